@@ -1,0 +1,204 @@
+/*
+ * zebra.h — C ABI of the Zebra3D multi-view global-attention library (sm_100a).
+ *
+ * Source of the method: the page "How Hybrid Attention Lets Feed-Forward 3D
+ * Models Scale to Many Views" (wispaper.ai), sections
+ *   "Linear-centered stages plus tile-sparse stages"   (tile-sparse stage, xL/yS)
+ *   "A closed-form fit avoids retraining from scratch"  (centered affine correction)
+ *   "Speedup scales with the number of input views"     (fused Q/K normalisation,
+ *       positional rotation and channel-softmax feature map; tile-major K/V packing)
+ *
+ * Token layout (all entry points). A layer sees V views; view v holds
+ * L = n_special + grid_h*grid_w tokens at token indices [v*L, (v+1)*L): first the
+ * n_special special tokens (camera, registers), then the patch grid in row-major
+ * order. Tokens are tiled per view into 8x8 patch blocks anchored at grid (0,0);
+ * bottom/right edge tiles are partial. Tile index
+ *   u = v*T_v + (row/8)*ceil(grid_w/8) + col/8,  T_v = ceil(grid_h/8)*ceil(grid_w/8),
+ * T = V*T_v tiles in all. Inside a tile, tokens are numbered row-major, 0..n_u-1.
+ *
+ * Q, K, V and outputs are [N, H, d] tensors: element (n, h, c) of a tensor with
+ * layout {tok_stride, head_stride} sits at ptr[n*tok_stride + h*head_stride + c]
+ * (strides in elements; channels contiguous). A NULL layout means contiguous
+ * [N, H, d] (tok_stride = H*d, head_stride = d). Outputs are always contiguous.
+ *
+ * Conventions.
+ *  - Ownership: the caller owns every buffer; all data pointers are DEVICE
+ *    pointers unless stated. The library allocates and frees no memory; scratch
+ *    comes from the caller's workspace (size: zebra_workspace_bytes).
+ *  - Streams: each call enqueues its kernels on `stream` (a cudaStream_t passed
+ *    as void*; NULL = legacy default stream) and returns without synchronising.
+ *  - Errors: argument errors return a nonzero status before anything is enqueued;
+ *    zebra_last_error() then describes the failure (thread-local). Launch errors
+ *    return ZEBRA_ERR_CUDA. Device-side failures (a bounded wait that ran out)
+ *    set a sticky device status word, read by zebra_sync_status().
+ *  - Inputs are never modified. Outputs are written completely.
+ */
+#ifndef ZEBRA_H
+#define ZEBRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZEBRA_API __attribute__((visibility("default")))
+#else
+#define ZEBRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-valued entry point. */
+#define ZEBRA_OK 0
+#define ZEBRA_ERR_INVALID_ARG 1   /* null pointer, bad size, y outside [0,1), ... */
+#define ZEBRA_ERR_UNSUPPORTED 2   /* d != 64, tile != 8, too many tiles, no sm_100 device */
+#define ZEBRA_ERR_WORKSPACE 3     /* workspace smaller than zebra_workspace_bytes() */
+#define ZEBRA_ERR_CUDA 4          /* a CUDA runtime or cuBLASLt call failed */
+#define ZEBRA_ERR_TIMEOUT 5       /* a device-side bounded wait gave up (sticky) */
+
+/* Element types of Q/K/V/out. bf16 is the production type; fp32 is accepted
+ * by the stage entry points for small, CPU-checkable runs. */
+typedef enum { ZEBRA_F32 = 0, ZEBRA_BF16 = 1 } zebra_dtype;
+
+/* Layer geometry. Constraints: views >= 0, grid_h >= 1, grid_w >= 1,
+ * 0 <= n_special <= 64, tile == 8, heads >= 1, head_dim == 64. */
+typedef struct zebra_geom {
+  int32_t views;
+  int32_t grid_h;
+  int32_t grid_w;
+  int32_t n_special;
+  int32_t tile;
+  int32_t heads;
+  int32_t head_dim;
+} zebra_geom;
+
+/* Strides (in elements) of a strided [N, H, d] input. */
+typedef struct zebra_layout {
+  int64_t tok_stride;
+  int64_t head_stride;
+} zebra_layout;
+
+/* Layer kinds of zebra_hybrid_layer ("xL/yS" allocation, section
+ * "Linear-centered stages plus tile-sparse stages"). */
+#define ZEBRA_LAYER_LINEAR 0
+#define ZEBRA_LAYER_SPARSE 1
+#define ZEBRA_LAYER_DENSE 2
+
+/* Operation ids of zebra_workspace_bytes. */
+#define ZEBRA_OP_SELECT 0
+#define ZEBRA_OP_SPARSE 1
+#define ZEBRA_OP_LINEAR 2
+#define ZEBRA_OP_HYBRID_LINEAR 3
+#define ZEBRA_OP_HYBRID_SPARSE 4
+#define ZEBRA_OP_HYBRID_DENSE 5
+
+/* Number of kept key tiles per query tile for sparsity y in [0,1):
+ * k = clamp(ceil((1-y)*T - 1e-6), 1, T) — the selector "retains a key-tile
+ * fraction of 1 minus y" (section "Linear-centered stages plus tile-sparse
+ * stages"); the ceiling and the 1e-6 guard are this library's reading.
+ * Returns -1 for y outside [0,1) or n_tiles < 1. Host only, no CUDA call. */
+ZEBRA_API int32_t zebra_keep_count(double y, int32_t n_tiles);
+
+/* Tile pooling and tile-major packing (sections "Linear-centered stages plus
+ * tile-sparse stages": omitted tiles become mean key/value landmarks; "Speedup
+ * scales with the number of input views": K/V packed in tile-major order).
+ *   x           [N, H, d] of type dt, strided by `layout` (NULL = contiguous)
+ *   x_mean      out [H, T, d] fp32: mean of each tile's n_u actual tokens (required)
+ *   x_packed    out [H, T, 64, d] of type dt, or NULL: tile u's tokens in row-major
+ *               tile order at rows 0..n_u-1, rows n_u..63 zero
+ *   tile_counts out [T] int32 n_u, or NULL
+ * T = 0 (views == 0) is a no-op. */
+ZEBRA_API int zebra_tile_pool(const zebra_geom* g, zebra_dtype dt, const void* x, const zebra_layout* layout,
+                    float* x_mean, void* x_packed, int32_t* tile_counts, void* stream);
+
+/* Per-query-tile key-tile selector (section "Linear-centered stages plus
+ * tile-sparse stages"). Scores key tile u for query tile t by the fp32 dot
+ * q_mean[h,t] . k_mean[h,u] over all T tiles (own tile included) and keeps the
+ * top k = zebra_keep_count(y, T); equal scores go to the lower tile index.
+ *   q_mean, k_mean [H, T, d] fp32 (from zebra_tile_pool)
+ *   mask      out [H, T, W] uint32, W = ceil(T/32): bit (u%32) of word u/32 of
+ *             row (h, t) is set iff key tile u is kept for query tile t
+ *   near_tie  out [H, T] uint8 or NULL: 1 where the k-th and (k+1)-th scores
+ *             differ by a relative gap < 1e-5 (0 when k == T)
+ *   k_out     HOST int32 out or NULL: the keep count
+ *   workspace device scratch of zebra_workspace_bytes(g, ZEBRA_OP_SELECT, ..) bytes
+ * Requires T <= 49152. */
+ZEBRA_API int zebra_tile_select(const zebra_geom* g, const float* q_mean, const float* k_mean, double y,
+                      uint32_t* mask, uint8_t* near_tie, int32_t* k_out,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Tile-sparse softmax attention of one layer (section "Linear-centered stages
+ * plus tile-sparse stages"). Per head, a patch query of tile t attends with
+ * scale 1/sqrt(d):
+ *   - every token of each kept key tile, exactly;
+ *   - every special-token key, exactly;
+ *   - its own key exactly, when its own tile t is not kept;
+ *   - one landmark per other unkept tile u: key = mean K, value = mean V of the
+ *     tile's tokens, logit q.k_mean/sqrt(d) + ln(m), m = n_u; for the own tile
+ *     (when unkept) the landmark covers its n_t - 1 other tokens (omitted if 0).
+ * Special-token queries attend all N keys densely.
+ *   q, k, v   [N, H, d] of type dt, strided by `layout` (NULL = contiguous)
+ *   y         sparsity in [0,1); y = 0 keeps every tile (dense attention)
+ *   mask      [H, T, W] selection from zebra_tile_select, or NULL to select here
+ *   out       [N, H, d] of type dt, contiguous
+ *   workspace zebra_workspace_bytes(g, ZEBRA_OP_SPARSE, dt, y) bytes */
+ZEBRA_API int zebra_sparse_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k, const void* v,
+                      const zebra_layout* layout, double y, const uint32_t* mask, void* out,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Linear global attention with the per-head centered affine correction
+ * (sections "Speedup scales with the number of input views" and "A closed-form
+ * fit avoids retraining from scratch"). Per head h and token n:
+ *   f(x) = phi(rope2d(x / sqrt(mean(x^2) + eps))), phi = softmax over the d channels,
+ *   rope2d turns channel pairs (j, j+16) of channels 0-31 by patch row * base^(-j/16)
+ *   and of channels 32-63 by patch column * base^(-j/16); special tokens unrotated;
+ *   S = sum_m f(k_m) v_m^T (d x d), z = sum_m f(k_m), over all N tokens;
+ *   out_n = A_h (S^T f(q_n) / (z . f(q_n))) + b_h.
+ *   A    [H, d, d] fp32 row-major (A[h][i][j] multiplies o_j into y_i), or NULL = identity
+ *   b    [H, d] fp32, or NULL = zero
+ *   out  [N, H, d] of type dt, contiguous
+ *   workspace zebra_workspace_bytes(g, ZEBRA_OP_LINEAR, dt, 0) bytes */
+ZEBRA_API int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k, const void* v,
+                      const zebra_layout* layout, const float* A, const float* b, float rope_base,
+                      float eps, void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* One stacked global-attention layer, bf16 only (section "Linear-centered
+ * stages plus tile-sparse stages": preserved QKV/output projections,
+ * normalisation and positional encoding):
+ *   x_out = x + concat_heads(Attn(Q, K, V)) W_o^T,  [Q|K|V] = x W_qkv^T,
+ * where Attn is the linear stage (kind ZEBRA_LAYER_LINEAR, with A, b), or the
+ * tile-sparse stage at sparsity y (ZEBRA_LAYER_SPARSE), or dense softmax
+ * attention (ZEBRA_LAYER_DENSE); the sparse and dense kinds first apply the
+ * RMS norm and 2D rotation of zebra_linear_attn to Q and K.
+ *   x      [N, D] bf16, D = heads*head_dim
+ *   w_qkv  [3D, D] bf16 row-major; w_o [D, D] bf16 row-major
+ *   x_out  [N, D] bf16 (may equal x)
+ *   workspace zebra_workspace_bytes(g, ZEBRA_OP_HYBRID_*, ZEBRA_BF16, y) bytes */
+ZEBRA_API int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void* w_qkv, const void* w_o,
+                       const float* A, const float* b, double y, float rope_base, float eps, void* x_out,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by operation `op` (ZEBRA_OP_*) for this geometry,
+ * element type and sparsity. Returns 0 and sets the last error on an invalid
+ * geometry or op. Host only. */
+ZEBRA_API size_t zebra_workspace_bytes(const zebra_geom* g, int op, zebra_dtype dt, double y);
+
+/* Description of the last error of the calling thread ("" if none). */
+ZEBRA_API const char* zebra_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns ZEBRA_OK, ZEBRA_ERR_TIMEOUT or ZEBRA_ERR_CUDA. */
+ZEBRA_API int zebra_sync_status(void* stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+ZEBRA_API uint64_t zebra_launch_count(void);
+
+/* Library version string. */
+ZEBRA_API const char* zebra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZEBRA_H */

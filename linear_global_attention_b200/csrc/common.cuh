@@ -1,0 +1,151 @@
+// Shared device/host helpers of the Zebra3D global-attention library.
+//
+// Token layout and tile partition follow the page "How Hybrid Attention Lets
+// Feed-Forward 3D Models Scale to Many Views", section "Linear-centered stages
+// plus tile-sparse stages" (8x8-patch tiles of 64 tokens per image; special
+// tokens per view), with partial bottom/right edge tiles.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "zebra.h"
+
+namespace zebra {
+
+constexpr int D = 64;      // head dimension (the only one supported)
+constexpr int TILE = 8;    // tile side in patches
+constexpr int TOK = 64;    // tokens in a complete tile / rows of a packed block
+
+// ---------------------------------------------------------------------------
+// geometry
+// ---------------------------------------------------------------------------
+struct Geo {
+  int V, Hp, Wp, S, H;   // views, grid rows, grid cols, special tokens/view, heads
+  int L;                 // tokens per view
+  int Tr, Tc, Tv, T;     // tile rows/cols per view, tiles per view, tiles
+  int W;                 // 32-bit mask words per selection row
+  int NS, NSp;           // special tokens (all views), padded to a multiple of 64
+  int Tpad;              // T padded to a multiple of 64
+  long long N;           // tokens
+};
+
+inline Geo make_geo(const zebra_geom& g) {
+  Geo o;
+  o.V = g.views; o.Hp = g.grid_h; o.Wp = g.grid_w; o.S = g.n_special; o.H = g.heads;
+  o.L = o.S + o.Hp * o.Wp;
+  o.Tr = (o.Hp + TILE - 1) / TILE;
+  o.Tc = (o.Wp + TILE - 1) / TILE;
+  o.Tv = o.Tr * o.Tc;
+  o.T = o.V * o.Tv;
+  o.W = (o.T + 31) / 32;
+  o.NS = o.S * o.V;
+  o.NSp = (o.NS + 63) / 64 * 64;
+  o.Tpad = (o.T + 63) / 64 * 64;
+  o.N = (long long)o.V * o.L;
+  return o;
+}
+
+struct TileShape {
+  int view, r0, c0, rows, cols;
+};
+
+__host__ __device__ __forceinline__ TileShape tile_shape(const Geo& g, int u) {
+  TileShape s;
+  s.view = u / g.Tv;
+  int p = u - s.view * g.Tv;
+  int br = p / g.Tc, bc = p - br * g.Tc;
+  s.r0 = br * TILE;
+  s.c0 = bc * TILE;
+  s.rows = min(TILE, g.Hp - s.r0);
+  s.cols = min(TILE, g.Wp - s.c0);
+  return s;
+}
+
+// token index of row a (row-major inside the tile) of tile shape s
+__host__ __device__ __forceinline__ long long tile_token(const Geo& g, const TileShape& s, int a) {
+  int rr = a / s.cols, cc = a - rr * s.cols;
+  return (long long)s.view * g.L + g.S + (long long)(s.r0 + rr) * g.Wp + (s.c0 + cc);
+}
+
+// token index of special token number i (0 <= i < NS): view i / S, slot i % S
+__host__ __device__ __forceinline__ long long special_token(const Geo& g, int i) {
+  int v = i / g.S;
+  return (long long)v * g.L + (i - v * g.S);
+}
+
+// ---------------------------------------------------------------------------
+// element helpers
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int PER16 = 4;  // elements per 16 bytes
+  __device__ static float to_f(float x) { return x; }
+  __device__ static float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int PER16 = 8;
+  __device__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  __device__ static __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// load 16 bytes as PER16 floats
+__device__ __forceinline__ void load16(const float* p, float* o) {
+  float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float* o) {
+  uint4 v = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    o[2 * i] = f.x; o[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store16(float* p, const float* o) {
+  *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float* o) {
+  uint4 v;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = v;
+}
+__device__ __forceinline__ void store16_zero(void* p) { *reinterpret_cast<uint4*>(p) = make_uint4(0, 0, 0, 0); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float LOG2E = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// host-side plumbing shared by the translation units
+// ---------------------------------------------------------------------------
+void set_error(const std::string& msg);
+void count_launch(int n = 1);
+int check_launch(const char* what);   // ZEBRA_OK or ZEBRA_ERR_CUDA (sets the message)
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Bump allocator over the caller's workspace.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T> T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align256(count * sizeof(T));
+    return p;
+  }
+  size_t used() const { return off; }
+};
+
+}  // namespace zebra

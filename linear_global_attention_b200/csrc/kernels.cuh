@@ -1,0 +1,88 @@
+// Kernel argument structs and launcher declarations (internal).
+#pragma once
+
+#include "common.cuh"
+
+namespace zebra {
+
+template <typename T>
+struct PoolArgs {
+  Geo g;
+  const T* x[3];        // up to three [N, H, d] inputs (Q, K, V); null = skip
+  long long ts, hs;     // token / head strides in elements (shared)
+  float* mean[3];       // [H, T, d] fp32 or null
+  T* packed[3];         // [H, T, 64, d] or null
+  T* lmk[3];            // [H, Tpad, d] landmark rows (mean rounded to T) or null
+  int norm_rope[3];     // apply RMS norm (+ rotation when rope != null)
+  const float2* rope;   // [maxpos, 16] cos/sin table or null
+  float eps;
+  int32_t* counts;      // [T] or null
+};
+
+template <typename T>
+struct SpecialArgs {
+  Geo g;
+  const T* x[3];
+  long long ts, hs;
+  T* out[3];            // [H, NSp, d]
+  int norm[3];
+  float eps;
+};
+
+template <typename T> int launch_pool_pack(const PoolArgs<T>& a, int ntensors, cudaStream_t st);
+template <typename T> int launch_pack_special(const SpecialArgs<T>& a, int ntensors, cudaStream_t st);
+int launch_rope_table(float2* tab, int maxpos, double base, cudaStream_t st);
+
+// ---- selector ----
+struct SelectArgs {
+  Geo g;
+  const float* qm;      // [H, T, d]
+  const float* km;
+  float* scores;        // [hc, T, Tld]
+  int Tld;
+  int h0, hc;           // head range of this pass
+  int keep;
+  uint32_t* mask;       // [H, T, W]
+  uint8_t* near_tie;    // [H, T] or null
+};
+int launch_scores(const SelectArgs& a, cudaStream_t st);
+int launch_select(const SelectArgs& a, cudaStream_t st);
+constexpr int SELECT_MAX_T = 49152;
+
+// ---- attention ----
+struct AttnArgs {
+  Geo g;
+  const void* Qp;  const void* Kp;  const void* Vp;   // [H, T, 64, d]
+  const void* Qs;  const void* Ks;  const void* Vs;   // [H, NSp, d]
+  const void* Kl;  const void* Vl;                    // [H, Tpad, d] landmark rows
+  const float* km; const float* vm;                   // [H, T, d] fp32 means (own-tile landmark)
+  const uint32_t* mask;                               // [H, T, W]
+  int keep;
+  void* out;                                          // [N, H, d]
+  // split-KV partials of the dense special-token rows
+  float* part_o;                                      // [splits, H, NSp, d]
+  float* part_ml;                                     // [splits, H, NSp, 2] (max in log2 units, sum)
+  int splits;
+  float ln_tab[TOK + 1];                              // ln(m), m = 0..64 (ln_tab[0] unused)
+};
+template <typename T> int launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
+template <typename T> int launch_special_rows(const AttnArgs& a, cudaStream_t st);
+
+// ---- linear stage ----
+struct LinearArgs {
+  Geo g;
+  const void* q; const void* k; const void* v;
+  long long ts, hs;
+  const float* A; const float* b;   // [H, d, d], [H, d] or null
+  float eps;
+  const float2* rope;               // [maxpos, 16]
+  float* part;                      // [chunks, H, d, 65] partial (S | z)
+  int chunks, chunk_tokens;
+  float* state;                     // [H, d, 65] fp32  S' = S A^T | z
+  void* state_b;                    // [H, 72, d] bf16 B operand (transposed) for the bf16 apply
+  void* out;                        // [N, H, d]
+};
+template <typename T> int launch_linear(const LinearArgs& a, cudaStream_t st);
+int linear_chunks(const Geo& g, int* chunk_tokens);
+
+}  // namespace zebra

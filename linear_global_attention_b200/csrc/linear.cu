@@ -1,0 +1,487 @@
+// Linear global attention with the per-head centered affine correction.
+//
+// Page "How Hybrid Attention Lets Feed-Forward 3D Models Scale to Many Views":
+//  - section "Speedup scales with the number of input views": the linear-stage
+//    kernels fuse Q/K normalisation, positional rotation and the channel-softmax
+//    feature map;
+//  - section "Linear-centered stages plus tile-sparse stages": linear-centered
+//    attention aggregates global context at linear cost;
+//  - section "A closed-form fit avoids retraining from scratch": a centered
+//    affine correction is applied to each linear stage's output.
+//
+// Per head h: f(x) = phi(rope2d(rmsnorm(x))), S = sum_n f(k_n) v_n^T, z = sum_n f(k_n),
+// y_n = A (S^T f(q_n)) / (z . f(q_n)) + b. Folding A into the state
+// (S' = S A^T) makes the epilogue one 64x65 contraction per token.
+//
+// Three kernels:
+//  1. state:  per (token chunk, head) CTA: prologue on K in registers (2 threads
+//     per token, 32 channels each), f(K) -> shared as bf16, then
+//     [S | z] += f(K)^T [V | 1] on mma.sync (M = 64 channels, N = 64 + 8 with a
+//     column of ones for z, K = 64 tokens), fp32 partials per chunk.
+//  2. reduce: per head, sums the chunk partials in a fixed order (deterministic),
+//     forms S' = S A^T, and writes the bf16 B operand [S' | z] of the apply kernel.
+//  3. apply:  per (token chunk, head) CTA: prologue on Q, f(Q) [S' | z] on
+//     mma.sync, divide by the z column, add b, store bf16.
+// The fp32 variants run the same three steps with plain fp32 arithmetic.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace zebra {
+
+constexpr int NB = 72;  // 64 state columns + z column, padded to a multiple of 8
+
+__device__ __forceinline__ void token_pos(const Geo& g, long long n, bool& special, int& row, int& col) {
+  const int j = (int)(n % g.L);
+  special = j < g.S;
+  const int p = j - g.S;
+  row = special ? 0 : p / g.Wp;
+  col = special ? 0 : p - (p / g.Wp) * g.Wp;
+}
+
+// Prologue on 32 channels (half 0: channels 0-31, rotated by row; half 1:
+// channels 32-63, rotated by column); the partner half lives in lane ^ 1.
+__device__ __forceinline__ void features_half(float* x, int half, bool special, int row, int col,
+                                              const float2* __restrict__ tab, float eps) {
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) ss = fmaf(x[c], x[c], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  const float sc = rsqrtf(ss * (1.0f / D) + eps);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) x[c] *= sc;
+  if (!special) {
+    const int pos = half ? col : row;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 cs = tab[pos * 16 + j];
+      const float a = x[j], b = x[j + 16];
+      x[j] = a * cs.x - b * cs.y;
+      x[j + 16] = b * cs.x + a * cs.y;
+    }
+  }
+  float mx = x[0];
+#pragma unroll
+  for (int c = 1; c < 32; ++c) mx = fmaxf(mx, x[c]);
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  float sum = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    x[c] = fast_exp2((x[c] - mx) * LOG2E);
+    sum += x[c];
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  const float inv = 1.0f / sum;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) x[c] *= inv;
+}
+
+// full 64-channel prologue in one thread (fp32 path)
+__device__ __forceinline__ void features_full(float* x, bool special, int row, int col,
+                                              const float2* __restrict__ tab, float eps) {
+  float ss = 0.f;
+  for (int c = 0; c < 64; ++c) ss = fmaf(x[c], x[c], ss);
+  const float sc = 1.0f / sqrtf(ss * (1.0f / D) + eps);
+  for (int c = 0; c < 64; ++c) x[c] *= sc;
+  if (!special) {
+    for (int half = 0; half < 2; ++half) {
+      const int pos = half ? col : row;
+      for (int j = 0; j < 16; ++j) {
+        const float2 cs = tab[pos * 16 + j];
+        const float a = x[32 * half + j], b = x[32 * half + j + 16];
+        x[32 * half + j] = a * cs.x - b * cs.y;
+        x[32 * half + j + 16] = b * cs.x + a * cs.y;
+      }
+    }
+  }
+  float mx = x[0];
+  for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+  float sum = 0.f;
+  for (int c = 0; c < 64; ++c) {
+    x[c] = expf(x[c] - mx);
+    sum += x[c];
+  }
+  for (int c = 0; c < 64; ++c) x[c] /= sum;
+}
+
+// --------------------------------------------------------------------------
+// mma helpers (same conventions as the attention kernels)
+// --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t lsmem(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ uint32_t lswz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
+__device__ __forceinline__ void l_ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void l_ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void l_ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void l_mma(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void store_row_half_bf16(unsigned char* tile, int row, int half, const float* x) {
+  // 32 channels = 4 chunks of 8, swizzled
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 v;
+    __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hv[i] = __floats2bfloat162_rn(x[8 * q + 2 * i], x[8 * q + 2 * i + 1]);
+    *reinterpret_cast<uint4*>(tile + lswz(row, half * 4 + q)) = v;
+  }
+}
+
+// --------------------------------------------------------------------------
+// 1. state (bf16)
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) linear_state_kernel(const __grid_constant__ LinearArgs a) {
+  __shared__ __align__(128) unsigned char phi_s[64 * 128];
+  __shared__ __align__(128) unsigned char v_s[64 * 128];
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const long long n0 = (long long)blockIdx.x * a.chunk_tokens;
+  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
+  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v);
+  const int tok = tid >> 1, half = tid & 1;
+
+  float acc[9][4];
+#pragma unroll
+  for (int j = 0; j < 9; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const int g4 = lane >> 2;
+  const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
+
+  for (long long nb = n0; nb < n1; nb += 64) {
+    const long long n = nb + tok;
+    const bool valid = n < n1;
+    float x[32];
+    uint4 vraw[4];
+    if (valid) {
+      const __nv_bfloat16* kp = K + n * a.ts + (long long)h * a.hs + half * 32;
+      const __nv_bfloat16* vp = Vt + n * a.ts + (long long)h * a.hs + half * 32;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        load16(kp + 8 * q, x + 8 * q);
+        vraw[q] = *reinterpret_cast<const uint4*>(vp + 8 * q);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) vraw[q] = make_uint4(0, 0, 0, 0);
+    }
+    {
+      // every lane runs the prologue (it shuffles with lane ^ 1); padding tokens are zeroed after
+      bool sp;
+      int row, col;
+      token_pos(g, valid ? n : 0, sp, row, col);
+      features_half(x, half, sp, row, col, a.rope, a.eps);
+      if (!valid) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = 0.f;
+      }
+    }
+    __syncthreads();  // previous MMA reads of phi_s / v_s are done
+    store_row_half_bf16(phi_s, tok, half, x);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(v_s + lswz(tok, half * 4 + q)) = vraw[q];
+    __syncthreads();
+    // [S | z] (rows = channels 16*warp..) += phi^T [V | 1]
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {  // 16 tokens per k-step
+      uint32_t af[4];
+      {
+        // A = phi^T: 8x8 blocks [tok, ch] read transposed
+        const int mi = lane >> 3, ri = lane & 7;
+        const int trow = ks * 16 + (mi >> 1) * 8 + ri;   // token
+        const int chk = warp * 2 + (mi & 1);             // channel chunk
+        l_ldsm_x4_t(lsmem(phi_s) + lswz(trow, chk), af[0], af[1], af[2], af[3]);
+      }
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        const int mi = lane >> 3, ri = lane & 7;
+        const int trow = ks * 16 + (mi & 1) * 8 + ri;
+        uint32_t b0, b1, b2, b3;
+        l_ldsm_x4_t(lsmem(v_s) + lswz(trow, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
+        l_mma(acc[2 * dp], af, b0, b1);
+        l_mma(acc[2 * dp + 1], af, b2, b3);
+      }
+      l_mma(acc[8], af, ones, ones);
+    }
+  }
+  // write partial [64][65]: row = channel, col = 0..63 (S), 64 (z)
+  float* part = a.part + ((size_t)blockIdx.x * g.H + h) * 64 * 65;
+  const int q4 = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 9; ++j) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = warp * 16 + g4 + (e >> 1) * 8;
+      const int c = 8 * j + 2 * q4 + (e & 1);
+      if (c <= 64) part[r * 65 + c] = acc[j][e];
+    }
+  }
+}
+
+// A-fragment note: for A = phi^T (M = channels, K = tokens) the 8x8 blocks are
+// stored [token][channel]; ldmatrix.trans of block (tokens 8i.., channels 8j..)
+// yields the fragment of rows (channels) 8j.., columns (tokens) 8i... The four
+// matrices are ordered (ch 0-7, tok 0-7), (ch 8-15, tok 0-7), (ch 0-7, tok 8-15),
+// (ch 8-15, tok 8-15) = a0..a3: matrix mi takes channel chunk warp*2 + (mi & 1)
+// and token rows (mi >> 1) * 8.
+
+// --------------------------------------------------------------------------
+// fp32 state
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) linear_state_simt_kernel(const __grid_constant__ LinearArgs a) {
+  __shared__ float phi_s[64][65];
+  __shared__ float v_s[64][64];
+  const Geo& g = a.g;
+  const int tid = threadIdx.x;
+  const int h = blockIdx.y;
+  const long long n0 = (long long)blockIdx.x * a.chunk_tokens;
+  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
+  const float* K = static_cast<const float*>(a.k);
+  const float* Vt = static_cast<const float*>(a.v);
+  const int c = tid >> 2, jb = (tid & 3) * 16;
+  float acc[16], zacc = 0.f;
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+  for (long long nb = n0; nb < n1; nb += 64) {
+    __syncthreads();
+    if (tid < 64) {
+      const long long n = nb + tid;
+      float x[64];
+      if (n < n1) {
+        for (int e = 0; e < 64; ++e) x[e] = K[n * a.ts + (long long)h * a.hs + e];
+        bool sp;
+        int row, col;
+        token_pos(g, n, sp, row, col);
+        features_full(x, sp, row, col, a.rope, a.eps);
+        for (int e = 0; e < 64; ++e) v_s[tid][e] = Vt[n * a.ts + (long long)h * a.hs + e];
+      } else {
+        for (int e = 0; e < 64; ++e) x[e] = 0.f, v_s[tid][e] = 0.f;
+      }
+      for (int e = 0; e < 64; ++e) phi_s[tid][e] = x[e];
+    }
+    __syncthreads();
+    for (int tk = 0; tk < 64; ++tk) {
+      const float p = phi_s[tk][c];
+      for (int j = 0; j < 16; ++j) acc[j] = fmaf(p, v_s[tk][jb + j], acc[j]);
+      zacc += p;
+    }
+  }
+  float* part = a.part + ((size_t)blockIdx.x * g.H + h) * 64 * 65;
+  for (int j = 0; j < 16; ++j) part[c * 65 + jb + j] = acc[j];
+  if ((tid & 3) == 0) part[c * 65 + 64] = zacc;
+}
+
+// --------------------------------------------------------------------------
+// 2. reduce + fold A: state[h][c][i] = sum_j S[c][j] A[i][j]; state[h][c][64] = z[c]
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constant__ LinearArgs a, int want_bf16) {
+  __shared__ float S[64][65];
+  __shared__ float As[64][65];
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const Geo& g = a.g;
+  for (int e = tid; e < 64 * 65; e += 256) {
+    float s = 0.f;
+    for (int ch = 0; ch < a.chunks; ++ch) s += a.part[((size_t)ch * g.H + h) * 64 * 65 + e];
+    S[e / 65][e % 65] = s;
+  }
+  for (int e = tid; e < 64 * 64; e += 256) {
+    const int i = e / 64, j = e % 64;
+    As[i][j] = a.A ? a.A[(size_t)h * 64 * 64 + e] : (i == j ? 1.f : 0.f);
+  }
+  __syncthreads();
+  float* st = a.state + (size_t)h * 64 * 65;
+  __nv_bfloat16* sb = want_bf16 ? static_cast<__nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64 : nullptr;
+  for (int e = tid; e < 64 * NB; e += 256) {
+    const int c = e / NB, i = e % NB;  // channel c, output column i
+    float val = 0.f;
+    if (i < 64) {
+      for (int j = 0; j < 64; ++j) val = fmaf(S[c][j], As[i][j], val);
+    } else if (i == 64) {
+      val = S[c][64];
+    }
+    if (i <= 64) st[c * 65 + i] = val;
+    if (sb) sb[(size_t)i * 64 + c] = __float2bfloat16_rn(val);  // B operand stored [n][k]
+  }
+}
+
+// --------------------------------------------------------------------------
+// 3. apply (bf16): CTA = 128 threads, 64 tokens per step, state B operand in smem
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) linear_apply_kernel(const __grid_constant__ LinearArgs a) {
+  __shared__ __align__(128) unsigned char phi_s[64 * 128];
+  __shared__ __align__(128) unsigned char b_s[NB * 128];
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const long long n0 = (long long)blockIdx.x * a.chunk_tokens;
+  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
+  for (int i = tid; i < NB * 8; i += 128) {
+    const int r = i >> 3, c = i & 7;
+    *reinterpret_cast<uint4*>(b_s + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
+  }
+  const int tok = tid >> 1, half = tid & 1;
+  const int g4 = lane >> 2, q4 = lane & 3;
+  float bias[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    bias[2 * j] = a.b ? a.b[h * 64 + 8 * j + 2 * q4] : 0.f;
+    bias[2 * j + 1] = a.b ? a.b[h * 64 + 8 * j + 2 * q4 + 1] : 0.f;
+  }
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+  for (long long nb = n0; nb < n1; nb += 64) {
+    const long long n = nb + tok;
+    const bool valid = n < n1;
+    float x[32];
+    if (valid) {
+      const __nv_bfloat16* qp = Q + n * a.ts + (long long)h * a.hs + half * 32;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) load16(qp + 8 * q, x + 8 * q);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = 0.f;
+    }
+    {
+      bool sp;
+      int row, col;
+      token_pos(g, valid ? n : 0, sp, row, col);
+      features_half(x, half, sp, row, col, a.rope, a.eps);
+      if (!valid) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = 0.f;
+      }
+    }
+    __syncthreads();
+    store_row_half_bf16(phi_s, tok, half, x);
+    __syncthreads();
+    float acc[9][4];
+#pragma unroll
+    for (int j = 0; j < 9; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {  // 16 channels per k-step
+      uint32_t af[4];
+      {
+        const int mi = lane >> 3, ri = lane & 7;
+        const int row = warp * 16 + (mi & 1) * 8 + ri;
+        l_ldsm_x4(lsmem(phi_s) + lswz(row, 2 * ks + (mi >> 1)), af[0], af[1], af[2], af[3]);
+      }
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int mi = lane >> 3, ri = lane & 7;
+        const int row = np * 16 + (mi >> 1) * 8 + ri;
+        uint32_t b0, b1, b2, b3;
+        l_ldsm_x4(lsmem(b_s) + lswz(row, 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        l_mma(acc[2 * np], af, b0, b1);
+        l_mma(acc[2 * np + 1], af, b2, b3);
+      }
+      {
+        const int mi = (lane >> 3) & 1, ri = lane & 7;
+        uint32_t b0, b1;
+        l_ldsm_x2(lsmem(b_s) + lswz(64 + ri, 2 * ks + mi), b0, b1);
+        l_mma(acc[8], af, b0, b1);
+      }
+    }
+    // column 64 (z . phi) sits in acc[8][0] / acc[8][2] of the q4 == 0 lane of each quad
+    const float den0 = __shfl_sync(0xffffffffu, acc[8][0], lane & ~3);
+    const float den1 = __shfl_sync(0xffffffffu, acc[8][2], lane & ~3);
+    const float i0 = 1.0f / den0, i1 = 1.0f / den1;
+#pragma unroll
+    for (int half2 = 0; half2 < 2; ++half2) {
+      const long long nn = nb + warp * 16 + g4 + half2 * 8;
+      if (nn >= n1) continue;
+      const float il = half2 ? i1 : i0;
+      __nv_bfloat16* dst = out + (nn * g.H + h) * D;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = 8 * j + 2 * q4;
+        *reinterpret_cast<__nv_bfloat162*>(dst + c) = __floats2bfloat162_rn(
+            fmaf(acc[j][half2 * 2], il, bias[2 * j]), fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
+      }
+    }
+  }
+}
+
+// fp32 apply: one thread per token
+__global__ void __launch_bounds__(128) linear_apply_simt_kernel(const __grid_constant__ LinearArgs a) {
+  __shared__ float st[64][65];
+  const Geo& g = a.g;
+  const int h = blockIdx.y;
+  for (int e = threadIdx.x; e < 64 * 65; e += blockDim.x) st[e / 65][e % 65] = a.state[(size_t)h * 64 * 65 + e];
+  __syncthreads();
+  const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= g.N) return;
+  const float* Q = static_cast<const float*>(a.q);
+  float x[64];
+  for (int e = 0; e < 64; ++e) x[e] = Q[n * a.ts + (long long)h * a.hs + e];
+  bool sp;
+  int row, col;
+  token_pos(g, n, sp, row, col);
+  features_full(x, sp, row, col, a.rope, a.eps);
+  float den = 0.f;
+  for (int c = 0; c < 64; ++c) den = fmaf(x[c], st[c][64], den);
+  float* dst = static_cast<float*>(a.out) + (n * g.H + h) * D;
+  for (int i = 0; i < 64; ++i) {
+    float num = 0.f;
+    for (int c = 0; c < 64; ++c) num = fmaf(x[c], st[c][i], num);
+    dst[i] = num / den + (a.b ? a.b[h * 64 + i] : 0.f);
+  }
+}
+
+// --------------------------------------------------------------------------
+int linear_chunks(const Geo& g, int* chunk_tokens) {
+  long long ct = 2048;
+  long long chunks = (g.N + ct - 1) / ct;
+  if (chunks > 256) {
+    chunks = 256;
+    ct = ((g.N + chunks - 1) / chunks + 63) / 64 * 64;
+    chunks = (g.N + ct - 1) / ct;
+  }
+  if (chunks < 1) chunks = 1;
+  *chunk_tokens = (int)ct;
+  return (int)chunks;
+}
+
+template <>
+int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
+  if (a.g.N == 0) return ZEBRA_OK;
+  linear_state_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  count_launch();
+  if (int rc = check_launch("linear_state_kernel")) return rc;
+  linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 1);
+  count_launch();
+  if (int rc = check_launch("linear_reduce_kernel")) return rc;
+  linear_apply_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  count_launch();
+  return check_launch("linear_apply_kernel");
+}
+
+template <>
+int launch_linear<float>(const LinearArgs& a, cudaStream_t st) {
+  if (a.g.N == 0) return ZEBRA_OK;
+  linear_state_simt_kernel<<<dim3(a.chunks, a.g.H), 256, 0, st>>>(a);
+  count_launch();
+  if (int rc = check_launch("linear_state_simt_kernel")) return rc;
+  linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 0);
+  count_launch();
+  if (int rc = check_launch("linear_reduce_kernel")) return rc;
+  linear_apply_simt_kernel<<<dim3((unsigned)((a.g.N + 127) / 128), a.g.H), 128, 0, st>>>(a);
+  count_launch();
+  return check_launch("linear_apply_simt_kernel");
+}
+
+}  // namespace zebra

@@ -1,0 +1,246 @@
+// Per-query-tile key-tile selector.
+//
+// Page "How Hybrid Attention Lets Feed-Forward 3D Models Scale to Many Views",
+// section "Linear-centered stages plus tile-sparse stages": the selector of a
+// sparse stage retains a key-tile fraction of 1 - y for every query tile.
+// This library scores key tile u for query tile t by the unscaled dot of their
+// mean-pooled query and key (fp32), keeps the top k, and breaks equal scores
+// toward the lower tile index.
+//
+// Two kernels per group of heads:
+//  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 64x64-tile
+//     fp32 GEMM (K = 64) written to scratch; each score is a fixed-order fma chain.
+//  2. select_kernel: one CTA per row (h, t) loads the row into shared memory as
+//     order-preserving 32-bit keys, finds the k-th largest key with four 8-bit
+//     radix passes (histograms replicated 8 ways to spread same-bin atomics over
+//     banks), then emits the bitmask: keys above the threshold, plus the
+//     lowest-index keys equal to it (block-wide scan over the mask words).
+//     It also flags near-ties: the k-th and (k+1)-th scores within a relative
+//     gap of 1e-5.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace zebra {
+
+__global__ void __launch_bounds__(256) scores_kernel(SelectArgs a) {
+  __shared__ float sq[64][65];
+  __shared__ float sk[64][65];
+  const int T = a.g.T;
+  const int hh = blockIdx.z;
+  const int h = a.h0 + hh;
+  const int t0 = blockIdx.y * 64, u0 = blockIdx.x * 64;
+  const float* qm = a.qm + (size_t)h * T * D;
+  const float* km = a.km + (size_t)h * T * D;
+  for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+    const int r = i / 16, c4 = (i % 16) * 4;
+    float4 q = make_float4(0, 0, 0, 0), k = q;
+    if (t0 + r < T) q = *reinterpret_cast<const float4*>(qm + (size_t)(t0 + r) * D + c4);
+    if (u0 + r < T) k = *reinterpret_cast<const float4*>(km + (size_t)(u0 + r) * D + c4);
+    sq[r][c4] = q.x; sq[r][c4 + 1] = q.y; sq[r][c4 + 2] = q.z; sq[r][c4 + 3] = q.w;
+    sk[r][c4] = k.x; sk[r][c4 + 1] = k.y; sk[r][c4 + 2] = k.z; sk[r][c4 + 3] = k.w;
+  }
+  __syncthreads();
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < D; ++c) {
+    float qv[4], kv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = sq[ty + 16 * i][c];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kv[j] = sk[tx + 16 * j][c];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
+  }
+  float* out = a.scores + (size_t)hh * T * a.Tld;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty + 16 * i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = u0 + tx + 16 * j;
+      if (u < T) out[(size_t)t * a.Tld + u] = acc[i][j];
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+  s = s + 0.0f;  // -0 -> +0: equal scores must map to equal keys
+  const uint32_t f = __float_as_uint(s);
+  return (f & 0x80000000u) ? ~f : (f | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+constexpr int SEL_THREADS = 512;
+constexpr int HCOPIES = 8;
+constexpr int HSTRIDE = 257;
+
+__global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ uint32_t hist[HCOPIES * HSTRIDE];
+  __shared__ uint32_t s_bin, s_need, s_eqtotal;
+  __shared__ uint32_t s_wsum[SEL_THREADS / 32];
+  __shared__ uint32_t s_max[SEL_THREADS / 32];
+  const int T = a.g.T, W = a.g.W;
+  const int t = blockIdx.x, hh = blockIdx.y, h = a.h0 + hh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* mrow = a.mask + ((size_t)h * T + t) * W;
+  if (a.keep >= T) {
+    for (int w = tid; w < W; w += SEL_THREADS) {
+      const int rem = T - w * 32;
+      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+    }
+    if (a.near_tie && tid == 0) a.near_tie[(size_t)h * T + t] = 0;
+    return;
+  }
+  const float* srow = a.scores + ((size_t)hh * T + t) * a.Tld;
+  for (int i = tid; i < T; i += SEL_THREADS) keys[i] = order_key(srow[i]);
+
+  uint32_t prefix = 0, pmask = 0, need = (uint32_t)a.keep;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < HCOPIES * HSTRIDE; i += SEL_THREADS) hist[i] = 0;
+    __syncthreads();
+    uint32_t* hc = hist + (lane & (HCOPIES - 1)) * HSTRIDE;
+    for (int i = tid; i < T; i += SEL_THREADS) {
+      const uint32_t k = keys[i];
+      if ((k & pmask) == prefix) atomicAdd(&hc[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t s = 0;
+#pragma unroll
+      for (int c = 0; c < HCOPIES; ++c) s += hist[c * HSTRIDE + tid];
+      hist[tid] = s;  // copy 0 slot tid: read by this thread only above
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t cum = 0;
+      int b = 255;
+      for (; b > 0; --b) {
+        if (cum + hist[b] >= need) break;
+        cum += hist[b];
+      }
+      s_bin = (uint32_t)b;
+      s_need = need - cum;
+      s_eqtotal = hist[b];
+    }
+    __syncthreads();
+    prefix |= s_bin << shift;
+    pmask |= 255u << shift;
+    need = s_need;
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;          // the k-th largest key
+  const uint32_t eq_take = need;        // how many keys equal to thr are kept (lowest index first)
+  const uint32_t eq_total = s_eqtotal;  // how many keys equal thr
+
+  // mask words: thread tid owns a contiguous run of words
+  const int per = (W + SEL_THREADS - 1) / SEL_THREADS;
+  const int w0 = tid * per, w1 = min(W, w0 + per);
+  uint32_t my_eq = 0;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t eqb = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int i = w * 32 + j;
+      if (i < T && keys[i] == thr) eqb |= 1u << j;
+    }
+    my_eq += __popc(eqb);
+  }
+  // exclusive scan of my_eq over threads
+  uint32_t incl = my_eq;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0;
+  for (int i = 0; i < warp; ++i) base += s_wsum[i];
+  uint32_t before = base + incl - my_eq;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t gt = 0, eqb = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int i = w * 32 + j;
+      if (i < T) {
+        const uint32_t k = keys[i];
+        if (k > thr) gt |= 1u << j;
+        else if (k == thr) eqb |= 1u << j;
+      }
+    }
+    uint32_t take = before >= eq_take ? 0u : min(eq_take - before, (uint32_t)__popc(eqb));
+    before += __popc(eqb);
+    uint32_t keepb = 0;
+    while (take--) {
+      const uint32_t low = eqb & (~eqb + 1u);
+      keepb |= low;
+      eqb ^= low;
+    }
+    mrow[w] = gt | keepb;
+  }
+
+  if (a.near_tie) {
+    // (k+1)-th largest: equal to thr if more keys equal it than were taken,
+    // otherwise the largest key below thr
+    uint32_t below = 0;
+    if (eq_total <= eq_take) {
+      for (int i = tid; i < T; i += SEL_THREADS) {
+        const uint32_t k = keys[i];
+        if (k < thr && k > below) below = k;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) below = max(below, __shfl_xor_sync(0xffffffffu, below, o));
+    if (lane == 0) s_max[warp] = below;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t nxt = 0;
+      for (int i = 0; i < SEL_THREADS / 32; ++i) nxt = max(nxt, s_max[i]);
+      uint8_t flag;
+      if (eq_total > eq_take) {
+        flag = 1;
+      } else {
+        const double s_a = key_value(thr), s_b = key_value(nxt);
+        const double den = fmax(fabs(s_a), fabs(s_b));
+        const double gap = den > 0 ? fabs(s_a - s_b) / den : 0.0;
+        flag = gap < 1e-5 ? 1 : 0;
+      }
+      a.near_tie[(size_t)h * T + t] = flag;
+    }
+  }
+}
+
+int launch_scores(const SelectArgs& a, cudaStream_t st) {
+  const int T = a.g.T;
+  if (T == 0 || a.keep >= T) return ZEBRA_OK;
+  dim3 grid((T + 63) / 64, (T + 63) / 64, a.hc);
+  scores_kernel<<<grid, 256, 0, st>>>(a);
+  count_launch();
+  return check_launch("scores_kernel");
+}
+
+int launch_select(const SelectArgs& a, cudaStream_t st) {
+  const int T = a.g.T;
+  if (T == 0) return ZEBRA_OK;
+  const size_t smem = (size_t)T * sizeof(uint32_t);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SELECT_MAX_T * 4);
+    attr_set = true;
+  }
+  dim3 grid(T, a.hc);
+  select_kernel<<<grid, SEL_THREADS, smem, st>>>(a);
+  count_launch();
+  return check_launch("select_kernel");
+}
+
+}  // namespace zebra

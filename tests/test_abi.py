@@ -1,0 +1,150 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/zebra.h, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_global_attention_b200 as zb
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(zb.LIB_PATH):
+        from linear_global_attention_b200 import build
+        build.build()
+    return zb.lib()
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "zebra.h")).read()
+    return re.findall(r"ZEBRA_API\s+[\w\s\*]+?\b(zebra_\w+)\s*\(", txt)
+
+
+def test_header_declares_the_entry_points():
+    names = set(_declared())
+    for n in ("zebra_tile_pool", "zebra_tile_select", "zebra_sparse_attn", "zebra_linear_attn",
+              "zebra_hybrid_layer", "zebra_workspace_bytes", "zebra_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 10
+    raw = ctypes.CDLL(zb.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_version_and_launch_count(L):
+    assert "sm_100a" in zb.zebra_version()
+    assert zb.zebra_launch_count() >= 0
+
+
+@pytest.mark.parametrize("T", [1, 7, 16, 512, 3200, 12800, 25600, 49152])
+@pytest.mark.parametrize("y", [0.0, 0.1, 0.5, 0.6, 0.8, 0.875, 0.9, 0.99, 0.9999])
+def test_keep_count_matches_oracle(L, y, T):
+    assert zb.zebra_keep_count(y, T) == oracle.keep_count(y, T)
+
+
+def test_keep_count_rejects_bad_y(L):
+    assert zb.zebra_keep_count(1.0, 16) == -1
+    assert zb.zebra_keep_count(-0.1, 16) == -1
+    assert zb.zebra_keep_count(float("nan"), 16) == -1
+
+
+def _g(**kw):
+    base = dict(views=4, grid_h=16, grid_w=16, heads=2)
+    base.update(kw)
+    return zb.geom(**base)
+
+
+def test_workspace_bytes(L):
+    g = _g()
+    for op in range(6):
+        assert zb.zebra_workspace_bytes(g, op, zb.ZEBRA_BF16, 0.6) > 0
+    bad = _g(head_dim=32)
+    with pytest.raises(zb.ZebraError):
+        zb.zebra_workspace_bytes(bad, zb.ZEBRA_OP_SPARSE)
+    with pytest.raises(zb.ZebraError):
+        zb.zebra_workspace_bytes(_g(), 17)
+
+
+def _sparse(L, g, dtype=zb.ZEBRA_BF16, y=0.6, ptr=4096, ws=4096, nbytes=1 << 40, layout=None):
+    p = ctypes.c_void_p(ptr)
+    return L.zebra_sparse_attn(ctypes.byref(g) if g is not None else None, dtype, p, p, p, layout, y, None, p,
+                               ctypes.c_void_p(ws) if ws else None, nbytes, None)
+
+
+def test_sparse_argument_errors(L):
+    assert _sparse(L, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(head_dim=128)) == zb.ZEBRA_ERR_UNSUPPORTED
+    assert _sparse(L, _g(tile=16)) == zb.ZEBRA_ERR_UNSUPPORTED
+    assert _sparse(L, _g(heads=0)) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(grid_h=0)) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(views=-1)) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(n_special=65)) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(), y=1.0) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(), y=-0.5) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(), dtype=7) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _sparse(L, _g(), ptr=0) == zb.ZEBRA_ERR_INVALID_ARG          # null q
+    assert _sparse(L, _g(), ptr=4100) == zb.ZEBRA_ERR_INVALID_ARG       # misaligned
+    assert _sparse(L, _g(), nbytes=16) == zb.ZEBRA_ERR_WORKSPACE
+    assert _sparse(L, _g(), ws=0) == zb.ZEBRA_ERR_WORKSPACE
+    bad_layout = zb.Layout(130, 64)
+    assert _sparse(L, _g(), layout=ctypes.byref(bad_layout)) == zb.ZEBRA_ERR_INVALID_ARG
+    assert "strides" in zb.zebra_last_error()
+    # more tiles than the selector handles
+    assert _sparse(L, _g(views=2000, grid_h=64, grid_w=64)) == zb.ZEBRA_ERR_UNSUPPORTED
+
+
+def test_empty_input_is_a_noop(L):
+    # views == 0: nothing to do, no device needed
+    assert _sparse(L, _g(views=0), ptr=0, ws=0, nbytes=0) == zb.ZEBRA_OK
+    p = ctypes.c_void_p(0)
+    g = _g(views=0)
+    assert L.zebra_linear_attn(ctypes.byref(g), zb.ZEBRA_BF16, p, p, p, None, None, None, 100.0, 1e-6, p, None, 0,
+                               None) == zb.ZEBRA_OK
+    assert L.zebra_hybrid_layer(ctypes.byref(g), 0, p, p, p, None, None, 0.0, 100.0, 1e-6, p, None, 0,
+                                None) == zb.ZEBRA_OK
+    assert L.zebra_tile_pool(ctypes.byref(g), zb.ZEBRA_BF16, p, None, p, None, None, None) == zb.ZEBRA_OK
+
+
+def test_linear_and_hybrid_argument_errors(L):
+    p = ctypes.c_void_p(4096)
+    g = _g()
+    assert L.zebra_linear_attn(ctypes.byref(g), zb.ZEBRA_BF16, p, p, p, None, None, None, 0.0, 1e-6, p, p, 1 << 40,
+                               None) == zb.ZEBRA_ERR_INVALID_ARG   # rope_base 0
+    assert L.zebra_linear_attn(ctypes.byref(g), zb.ZEBRA_BF16, p, p, p, None, None, None, 100.0, 1e-6, p, p, 8,
+                               None) == zb.ZEBRA_ERR_WORKSPACE
+    assert L.zebra_hybrid_layer(ctypes.byref(g), 9, p, p, p, None, None, 0.5, 100.0, 1e-6, p, p, 1 << 40,
+                                None) == zb.ZEBRA_ERR_INVALID_ARG  # kind
+    assert L.zebra_hybrid_layer(ctypes.byref(g), 1, p, p, p, None, None, 1.5, 100.0, 1e-6, p, p, 1 << 40,
+                                None) == zb.ZEBRA_ERR_INVALID_ARG  # y
+    assert L.zebra_hybrid_layer(ctypes.byref(g), 1, p, p, p, None, None, 0.5, 100.0, 1e-6, p, p, 8,
+                                None) == zb.ZEBRA_ERR_WORKSPACE
+
+
+def test_select_argument_errors(L):
+    p = ctypes.c_void_p(4096)
+    g = _g()
+    k = ctypes.c_int32(0)
+    assert L.zebra_tile_select(ctypes.byref(g), p, p, 1.0, p, None, ctypes.byref(k), p, 1 << 40,
+                               None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_tile_select(ctypes.byref(g), p, p, 0.6, None, None, ctypes.byref(k), p, 1 << 40,
+                               None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert k.value == 7   # keep count is reported before the mask check
+    assert L.zebra_tile_select(ctypes.byref(g), p, p, 0.6, p, None, ctypes.byref(k), p, 4,
+                               None) == zb.ZEBRA_ERR_WORKSPACE
+
+
+def test_no_gpu_gives_a_cuda_error_not_a_crash(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _sparse(L, _g()) == zb.ZEBRA_ERR_CUDA
+    assert "CUDA" in zb.zebra_last_error() or "device" in zb.zebra_last_error()
