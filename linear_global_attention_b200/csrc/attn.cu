@@ -42,6 +42,14 @@ struct BlockIter {
   int t_end;      // dense rows: end of the tile range
 };
 
+// word w of a selection row, with bits of tiles >= T cleared (a caller-supplied
+// mask may carry stray bits there)
+__device__ __forceinline__ uint32_t mask_word(const uint32_t* __restrict__ mrow, int w, int T) {
+  const uint32_t m = __ldg(mrow + w);
+  const int rem = T - w * 32;
+  return rem >= 32 ? m : (m & ((1u << rem) - 1u));
+}
+
 // MODE 0: the kept tiles of row `mrow`, then landmark blocks with at least one
 // visible landmark, then special blocks.
 __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, const uint32_t* __restrict__ mrow,
@@ -49,7 +57,7 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
   if (it.phase == 0) {
     while (it.bits == 0 && it.w + 1 < g.W) {
       ++it.w;
-      it.bits = __ldg(mrow + it.w);
+      it.bits = mask_word(mrow, it.w, g.T);
     }
     if (it.bits != 0) {
       const int b = __ffs(it.bits) - 1;
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   int n_t = 0;
   if (MODE == 0) {
     it.w = 0;
-    it.bits = __ldg(mrow);
+    it.bits = mask_word(mrow, 0, g.T);
     own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
     const TileShape s = tile_shape(g, t);
     n_t = s.rows * s.cols;
@@ -490,7 +498,7 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(const __grid_constant__ A
   bool with_special = true, own_kept = true;
   int n_t = 0;
   if (MODE == 0) {
-    it.bits = __ldg(mrow);
+    it.bits = mask_word(mrow, 0, g.T);
     own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
     const TileShape s = tile_shape(g, t);
     n_t = s.rows * s.cols;
