@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the Zebra3D hybrid global-attention stack on B200.
+
+Workload (the configuration the headline metric is quoted on): 1,024 views of
+a 37x37 patch grid plus 5 special tokens each (N = 1,406,976 tokens), model
+dim 1024, 16 heads of 64, 24 stacked global-attention layers allocated 0.7L/0.8S
+(layers 0-16 linear, 17-23 tile-sparse at y = 0.8), bf16, random-init
+projections ~ N(0, 0.02^2) and x0 ~ N(0, 1) from seed 4.
+
+One step = one pass of the whole stack (every step of the hot path: projections,
+pooling/packing, selection, sparse attention, dense special rows, linear
+state/apply, residual) over x0. Metric: tokens/s per layer = n_gpus * N * 24 /
+(device time of one step). Each step also copies x0 host->device before and
+x24 device->host after the stack inside the e2e timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zebra|reference]
+
+--impl reference times the CPU oracle (fp64 NumPy, this repository's test
+oracle) on bounded samples of the same workload, extrapolated to a full step.
+Multi-GPU (torchrun): every rank runs its own replica (weak scaling); times
+are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "global-attn tokens/s per layer at 1,024 views (sparse, linear, hybrid) + % roofline"
+UNIT = "tokens/s"
+WORKLOAD = "stack_v1024"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["zebra", "reference"], default="zebra")
+    p.add_argument("--views", type=int, default=None, help="override the view count (quick runs only)")
+    p.add_argument("--no-dense", action="store_true", help="skip the dense softmax baseline")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    p.add_argument("--json-extra", default=None, help="also write the full result dict to this file")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank float over all ranks (device-side all-reduce)."""
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    import torch
+    torch.cuda.synchronize()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        ident = str(device_index)
+        try:
+            import torch
+            ident = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-i", ident, "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == 7:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = [n for i, n in enumerate(names) if any(r[3 + i] == "Active" for r in rows)]
+        loaded = [x for x in sm if x > 500] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_zebra(args):
+    import numpy as np
+    import torch
+
+    import linear_global_attention_b200 as zb
+    import synth
+
+    ws_n, rank, local = dist_setup()
+    w = synth.WORKLOADS[WORKLOAD]
+    if args.views:
+        import dataclasses
+        w = dataclasses.replace(w, views=args.views)
+    V, Hp, Wp, H, D = w.views, w.grid_h, w.grid_w, w.heads, w.model_dim
+    g = zb.geom(V, Hp, Wp, H)
+    N, L = g.n_tokens, w.layers
+    kinds = synth.stack_layer_kinds(w)
+    y = w.y[0]
+
+    # inputs: x0 in pinned host memory; weights resident on the device
+    t0 = time.time()
+    x0_host = torch.from_numpy(synth.stack_x0(w)).to(torch.bfloat16).pin_memory()
+    wq, wo, As, bs = [], [], [], []
+    for layer in range(L):
+        a, b = synth.stack_layer_weights(w, layer)
+        wq.append(torch.from_numpy(a).to(torch.bfloat16).cuda())
+        wo.append(torch.from_numpy(b).to(torch.bfloat16).cuda())
+        if kinds[layer] == "linear":
+            A, bb = synth.affine(H, w.seed, layer)
+            As.append(torch.from_numpy(A).cuda())
+            bs.append(torch.from_numpy(bb).cuda())
+        else:
+            As.append(None)
+            bs.append(None)
+    gen_s = time.time() - t0
+    wsb = max(zb.zebra_workspace_bytes(g, zb.ZEBRA_OP_HYBRID_LINEAR, zb.ZEBRA_BF16, y),
+              zb.zebra_workspace_bytes(g, zb.ZEBRA_OP_HYBRID_SPARSE, zb.ZEBRA_BF16, y))
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    x0 = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+    xa = torch.empty_like(x0)
+    xb = torch.empty_like(x0)
+    out_host = torch.empty((N, D), dtype=torch.bfloat16).pin_memory()
+    kind_id = {"linear": zb.ZEBRA_LAYER_LINEAR, "sparse": zb.ZEBRA_LAYER_SPARSE}
+
+    def stack(layer_events=None):
+        src = x0
+        for layer in range(L):
+            dst = xa if layer % 2 == 0 else xb
+            zb.zebra_hybrid_layer(g, kind_id[kinds[layer]], src, wq[layer], wo[layer], As[layer], bs[layer], y, dst,
+                                  ws)
+            if layer_events is not None:
+                layer_events[layer].record()
+            src = dst
+        return src
+
+    def step(ev):
+        # ev: [e2e start, stack start, per-layer..., stack end(=last layer), e2e end]
+        ev[0].record()
+        x0.copy_(x0_host, non_blocking=True)
+        ev[1].record()
+        res = stack(ev[2:2 + L])
+        out_host.copy_(res, non_blocking=True)
+        ev[2 + L].record()
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(L + 3)]
+
+    for _ in range(args.warmup):
+        step(new_events())
+    assert zb.zebra_sync_status() == zb.ZEBRA_OK
+    barrier(ws_n)
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    zb.zebra_profile_enable(True)
+    launches0 = zb.zebra_launch_count()
+    evs = [new_events() for _ in range(args.steps)]
+    barrier(ws_n)
+    for i in range(args.steps):
+        step(evs[i])
+    barrier(ws_n)
+    launches = zb.zebra_launch_count() - launches0
+    clk = clocks.stop()
+    prof = zb.zebra_profile_report()
+    zb.zebra_profile_enable(False)
+    assert zb.zebra_sync_status() == zb.ZEBRA_OK
+
+    dev_ms = sum(e[1].elapsed_time(e[1 + L]) for e in evs)
+    e2e_ms = sum(e[0].elapsed_time(e[2 + L]) for e in evs)
+    per_layer = {"linear": [], "sparse": []}
+    for e in evs:
+        prev = e[1]
+        for layer in range(L):
+            per_layer[kinds[layer]].append(prev.elapsed_time(e[2 + layer]))
+            prev = e[2 + layer]
+    dev_ms = max_over_ranks(dev_ms, ws_n)
+    e2e_ms = max_over_ranks(e2e_ms, ws_n)
+    ms_step = dev_ms / args.steps
+    value = ws_n * N * L / (ms_step / 1e3)
+    e2e_value = ws_n * N * L / (e2e_ms / args.steps / 1e3)
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    kern = prof["kernels"]
+    dom = max(kern.items(), key=lambda kv: kv[1][1])
+    sparse_launches, sparse_ms = kern.get("attn_sparse_rows", (0, 0.0))
+    sparse_flops_launch = 4 * 64 * prof["logits"].get("sparse_rows", 0) / max(sparse_launches, 1)
+    achieved = sparse_flops_launch / (sparse_ms / max(sparse_launches, 1) / 1e3) / 1e12 if sparse_ms else 0.0
+    roofline = {"kernel": "attn_sparse_rows", "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sustained"], 4),
+                "traffic": None, "peak_source": f"{pk['source']} bf16 sustained",
+                "algorithmic_flops_per_launch": sparse_flops_launch,
+                "avg_launch_ms": sparse_ms / max(sparse_launches, 1)}
+    # linear stage: compulsory HBM bytes (Q, K, V read once, O written once, bf16)
+    lin_bytes = 8 * N * H * 64
+    lin_ms = sum(kern.get(n, (0, 0.0))[1] for n in ("linear_state", "linear_reduce", "linear_apply"))
+    lin_layers = max(kern.get("linear_state", (0, 0))[0], 1)
+    lin_gbs = lin_bytes / (lin_ms / lin_layers / 1e3) / 1e9 if lin_ms else 0.0
+    stages = {name: {"launches": n, "total_ms": round(ms, 3), "share": round(ms / sum(v[1] for v in kern.values()), 4)}
+              for name, (n, ms) in kern.items()}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded x0 ~ N(0,1), W ~ N(0,0.02^2))",
+        "config": {"workload": f"{WORKLOAD}: {V} views x (37x37 patches + 5 special) = {N:,} tokens, "
+                               f"{L} layers 0.7L/0.8S (17 linear + 7 tile-sparse y=0.8), dim 1024, 16 heads x 64",
+                   "views": V, "tokens": N, "layers": L, "allocation": "0.7L/0.8S", "parallelism": f"replica x{ws_n}",
+                   "l2": "inputs larger than L2 (x0 = %.2f GB bf16)" % (N * D * 2 / 1e9)},
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": N * D * 2,
+                "d2h_bytes_per_step": N * D * 2},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "layer_ms": {k: round(statistics.mean(v), 3) for k, v in per_layer.items() if v},
+        "linear_stage_hbm": {"gbs": round(lin_gbs, 1), "peak_gbs": pk["hbm_gbs"],
+                             "frac": round(lin_gbs / pk["hbm_gbs"], 4), "compulsory_bytes": lin_bytes},
+        "kernels": stages,
+        "dominant_kernel": dom[0],
+        "input_gen_s": round(gen_s, 1),
+    }
+
+    if not args.no_dense and rank == 0:
+        result["dense_baseline"] = dense_baseline(g, N, H, D, kern, ms_step, L)
+    if not args.no_cpu and rank == 0:
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, rank
+
+
+def dense_baseline(g, N, H, D, kern, ms_step, L):
+    """Same-GPU dense softmax layer on identical shapes: torch SDPA (flash/cuDNN,
+    bf16) over [1, 16, N, 64] plus this run's projection GEMM time per layer."""
+    import torch
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    q = torch.randn((1, H, N, 64), device="cuda", dtype=torch.bfloat16, generator=gen)
+    k = torch.randn_like(q)
+    v = torch.randn_like(q)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.nn.functional.scaled_dot_product_attention(q[:, :, :65536], k[:, :, :65536], v[:, :, :65536])
+    torch.cuda.synchronize()
+    e0.record()
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    e1.record()
+    torch.cuda.synchronize()
+    sdpa_ms = e0.elapsed_time(e1)
+    del q, k, v, o
+    gemm_n, gemm_ms = kern.get("cublasLt_gemm", (0, 0.0))
+    gemm_per_layer = gemm_ms / max(gemm_n, 1) * 2
+    layer_ms = sdpa_ms + gemm_per_layer
+    flops = 4 * 64 * N * N * H
+    return {"impl": "torch.nn.functional.scaled_dot_product_attention (bf16) + the stack's projection GEMMs",
+            "sdpa_ms": round(sdpa_ms, 1), "sdpa_tflops": round(flops / (sdpa_ms / 1e3) / 1e12, 1),
+            "layer_ms": round(layer_ms, 1), "stack_ms": round(layer_ms * L, 1),
+            "tokens_per_s_per_layer": round(N / (layer_ms / 1e3), 1),
+            "hybrid_speedup": round(layer_ms * L / ms_step, 3)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline)
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return None
+
+
+def cpu_baseline(w, budget_s=20.0, sample_tiles=4):
+    """The fp64 oracle on a bounded sample of one step, extrapolated to a step.
+
+    Sample (one head): the sparse stage for `sample_tiles` query tiles at the
+    full 1,024-view geometry (selection over all tiles, kept tokens, landmarks,
+    special keys), with iid N(0,1) Q/K/V; tile pooling and the linear stage on
+    a 1/8-size geometry (128 views), whose cost is linear in the token count;
+    the projections of 4,096 rows. Extrapolation: x8 for pooling and linear,
+    x(T / sample_tiles) for the sparse tiles, x16 heads, x(N / 4,096) rows,
+    then 17 linear + 7 sparse layers.
+    """
+    import dataclasses
+
+    import numpy as np
+
+    import oracle
+    import synth
+
+    g = oracle.Geom(w.views, w.grid_h, w.grid_w, 1)
+    N, T = g.n_tokens, g.n_tiles
+    scale = 8
+    gs = oracle.Geom(max(1, w.views // scale), w.grid_h, w.grid_w, 1)
+    ratio = N / gs.n_tokens
+    q, k, v = (synth.normal_blocks((1, 64), N, 777, i) for i in range(3))
+    qs, ks, vs = (x[:gs.n_tokens] for x in (q, k, v))
+    A, b = synth.affine(1, 777)
+    keep = oracle.keep_count(w.y[0], T)
+    rng = np.random.default_rng(0)
+    tiles = np.sort(rng.choice(T, sample_tiles, replace=False))
+    members_s = oracle.tile_members(gs)
+    t0 = time.perf_counter()
+    for x in (qs, ks, vs):
+        oracle.tile_means(x[:, 0], gs, members_s)
+    t_pool = (time.perf_counter() - t0) * ratio
+    t0 = time.perf_counter()
+    oracle.linear_stage(qs, ks, vs, gs, A, b)
+    t_lin = (time.perf_counter() - t0) * ratio
+    t0 = time.perf_counter()
+    oracle.sparse_stage(q, k, v, g, keep, query_tiles=tiles, special_rows=np.zeros(0, np.int64))
+    t_call = time.perf_counter() - t0
+    t_tiles = max(t_call - t_pool, 1e-9)          # the call pools every tile first
+    rows = 4096
+    xs = rng.standard_normal((rows, w.model_dim))
+    wqkv = rng.standard_normal((3 * w.model_dim, w.model_dim))
+    wo = rng.standard_normal((w.model_dim, w.model_dim))
+    t0 = time.perf_counter()
+    xs @ wqkv.T
+    xs @ wo.T
+    t_proj = (time.perf_counter() - t0) * N / rows
+    H = w.heads
+    sparse_layer = H * (t_pool + T / sample_tiles * t_tiles)
+    linear_layer = H * t_lin
+    n_lin = w.n_linear
+    step_s = n_lin * (linear_layer + t_proj) + (w.layers - n_lin) * (sparse_layer + t_proj)
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    return {"value": round(N * w.layers / step_s, 3), "unit": UNIT, "cores": cores, "blas_threads": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"1 head: {sample_tiles} sparse query tiles at the full {w.views}-view geometry, pooling and "
+                      f"the linear stage on {gs.views} views (x{ratio:.0f}), projections of {rows} rows; "
+                      f"extrapolated to 16 heads, all {T} tiles and the 24-layer step",
+            "step_s_extrapolated": round(step_s, 1),
+            "measured_s": {"sparse_call": round(t_call, 2), "pool_scaled": round(t_pool, 2),
+                           "linear_head_scaled": round(t_lin, 2), "proj": round(t_proj, 2)}}
+
+
+def run_reference(args):
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None, rank
+    w = synth.WORKLOADS[WORKLOAD]
+    if args.views:
+        import dataclasses
+        w = dataclasses.replace(w, views=args.views)
+    for _ in range(args.warmup):
+        cpu_baseline(w, sample_tiles=1)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(w)
+        vals.append(last["value"])
+    value = statistics.mean(vals)
+    N = w.n_tokens
+    res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(N * w.layers / value * 1e3, 1), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": f"{WORKLOAD}: {w.views} views, {N:,} tokens, {w.layers} layers 0.7L/0.8S"},
+           "impl": "reference",
+           "cpu_baseline": {"kind": "oracle", "cores": last["cores"], "sample": last["sample"], "value": value},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return res, rank
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        res, rank = run_reference(args)
+    else:
+        res, rank = run_zebra(args)
+    if rank == 0 and res is not None:
+        line = json.dumps(res)
+        print(line, flush=True)
+        if args.json_extra:
+            with open(args.json_extra, "w") as f:
+                f.write(json.dumps(res, indent=1))
+
+
+if __name__ == "__main__":
+    main()

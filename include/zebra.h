@@ -194,6 +194,20 @@ ZEBRA_API int zebra_sync_status(void* stream);
 /* Number of kernels this library has launched in this process (all devices). */
 ZEBRA_API uint64_t zebra_launch_count(void);
 
+/* Optional per-kernel timing. zebra_profile_enable(1) clears the record and
+ * from then on brackets every kernel this library launches with two CUDA events
+ * on the launching stream; it also zeroes the device counters of visible
+ * attention logits. zebra_profile_enable(0) stops recording. Returns a status. */
+ZEBRA_API int zebra_profile_enable(int on);
+
+/* Waits for the recorded events and writes a text report into buf (at most len
+ * bytes, NUL-terminated): one line "kernel <name> <launches> <total ms>" per
+ * kernel name in first-launch order, then "logits sparse_rows <n>" and
+ * "logits special_rows <n>", the number of unmasked query-key logits the
+ * attention kernels evaluated (4*d FLOPs each: QK^T and PV). Returns the full
+ * report length. Host pointer. */
+ZEBRA_API long long zebra_profile_report(char* buf, size_t len);
+
 /* Library version string. */
 ZEBRA_API const char* zebra_version(void);
 

@@ -15,7 +15,8 @@ __all__ = [
     "Geom", "Layout", "ZebraError", "lib", "geom",
     "zebra_keep_count", "zebra_tile_pool", "zebra_tile_select", "zebra_sparse_attn",
     "zebra_linear_attn", "zebra_hybrid_layer", "zebra_workspace_bytes", "zebra_last_error",
-    "zebra_sync_status", "zebra_launch_count", "zebra_version", "workspace",
+    "zebra_sync_status", "zebra_launch_count", "zebra_version", "workspace", "zebra_profile_enable",
+    "zebra_profile_report",
     "ZEBRA_OK", "ZEBRA_ERR_INVALID_ARG", "ZEBRA_ERR_UNSUPPORTED", "ZEBRA_ERR_WORKSPACE", "ZEBRA_ERR_CUDA",
     "ZEBRA_ERR_TIMEOUT", "ZEBRA_F32", "ZEBRA_BF16", "ZEBRA_LAYER_LINEAR", "ZEBRA_LAYER_SPARSE",
     "ZEBRA_LAYER_DENSE", "ZEBRA_OP_SELECT", "ZEBRA_OP_SPARSE", "ZEBRA_OP_LINEAR", "ZEBRA_OP_HYBRID_LINEAR",
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
             "zebra_sync_status": (ctypes.c_int, [_P]),
             "zebra_launch_count": (ctypes.c_uint64, []),
             "zebra_version": (ctypes.c_char_p, []),
+            "zebra_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+            "zebra_profile_report": (ctypes.c_longlong, [ctypes.c_char_p, ctypes.c_size_t]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -206,3 +209,22 @@ def zebra_hybrid_layer(g: Geom, kind: int, x, w_qkv, w_o, A, b, y, x_out, ws, ro
     _check(lib().zebra_hybrid_layer(ctypes.byref(g), kind, _ptr(x), _ptr(w_qkv), _ptr(w_o), _ptr(A), _ptr(b), y,
                                     rope_base, eps, _ptr(x_out), _ptr(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)))
+
+
+def zebra_profile_enable(on: bool = True):
+    _check(lib().zebra_profile_enable(1 if on else 0))
+
+
+def zebra_profile_report() -> dict:
+    """{"kernels": {name: (launches, total_ms)}, "logits": {"sparse_rows": n, "special_rows": n}}."""
+    n = lib().zebra_profile_report(None, 0)
+    buf = ctypes.create_string_buffer(int(n) + 1)
+    lib().zebra_profile_report(buf, len(buf))
+    rep = {"kernels": {}, "logits": {}}
+    for line in buf.value.decode().splitlines():
+        parts = line.split()
+        if parts[0] == "kernel":
+            rep["kernels"][parts[1]] = (int(parts[2]), float(parts[3]))
+        elif parts[0] == "logits":
+            rep["logits"][parts[1]] = int(parts[2])
+    return rep

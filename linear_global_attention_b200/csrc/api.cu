@@ -2,10 +2,14 @@
 // workspace carving and kernel orchestration. See include/zebra.h for the
 // contract of every entry point.
 #include <math.h>
+#include <string.h>
 
 #include <atomic>
 #include <cstdio>
+#include <map>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "gemm.cuh"
@@ -18,6 +22,42 @@ static std::atomic<unsigned long long> g_launches{0};
 
 void set_error(const std::string& msg) { g_err = msg; }
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+// ---- profiling records ----
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static std::atomic<bool> g_prof_on{false};
+static std::vector<ProfRec> g_recs;
+static std::vector<cudaEvent_t> g_event_pool;
+
+static cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+ProfScope::ProfScope(const char* name, cudaStream_t s) : st(s) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ProfRec r{name, take_event(), take_event()};
+  cudaEventRecord(r.a, st);
+  slot = (int)g_recs.size();
+  g_recs.push_back(r);
+}
+
+ProfScope::~ProfScope() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEventRecord(g_recs[slot].b, st);
+}
 
 int check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
@@ -511,6 +551,58 @@ int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void*
     ZTRY(run_sparse<__nv_bfloat16>(G, q, k, v, ts, hs, keep, nullptr, w.o, w.sp, true, rope_base, eps, st));
   }
   return gemm_bf16_nt(w.o, w_o, x, x_out, G.N, Dm, Dm, 1.f, w.gemm_ws, GEMM_WS_BYTES, st);
+}
+
+int zebra_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  g_prof_on.store(on != 0);
+  if (on) {
+    if (int rc = check_device()) return rc;
+    reset_logit_counters();
+    return check_launch("zebra_profile_enable");
+  }
+  return ZEBRA_OK;
+}
+
+long long zebra_profile_report(char* buf, size_t len) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  std::map<std::string, std::pair<long long, double>> acc;
+  std::vector<std::string> order;
+  for (auto& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    auto it = acc.find(r.name);
+    if (it == acc.end()) {
+      order.push_back(r.name);
+      acc[r.name] = {1, (double)ms};
+    } else {
+      it->second.first += 1;
+      it->second.second += ms;
+    }
+  }
+  std::string out;
+  char line[256];
+  for (auto& n : order) {
+    snprintf(line, sizeof(line), "kernel %s %lld %.6f\n", n.c_str(), acc[n].first, acc[n].second);
+    out += line;
+  }
+  unsigned long long cnt[2] = {0, 0};
+  if (check_device() == ZEBRA_OK) read_logit_counters(cnt);
+  snprintf(line, sizeof(line), "logits sparse_rows %llu\nlogits special_rows %llu\n", cnt[0], cnt[1]);
+  out += line;
+  if (buf && len) {
+    const size_t n = out.size() < len - 1 ? out.size() : len - 1;
+    memcpy(buf, out.data(), n);
+    buf[n] = 0;
+  }
+  return (long long)out.size();
 }
 
 int zebra_sync_status(void* stream) {

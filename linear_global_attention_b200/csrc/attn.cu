@@ -31,6 +31,16 @@
 
 namespace zebra {
 
+// Visible (unmasked) logits evaluated: [0] patch rows of the sparse kernel,
+// [1] special-token rows. Each costs 4*d FLOPs (QK^T and PV); one atomic per CTA.
+__device__ unsigned long long g_logits[2];
+
+void reset_logit_counters() {
+  const unsigned long long z[2] = {0, 0};
+  cudaMemcpyToSymbol(g_logits, z, sizeof(z));
+}
+void read_logit_counters(unsigned long long* out2) { cudaMemcpyFromSymbol(out2, g_logits, 2 * sizeof(unsigned long long)); }
+
 // ---------------------------------------------------------------------------
 // block stream
 // ---------------------------------------------------------------------------
@@ -53,7 +63,7 @@ __device__ __forceinline__ uint32_t mask_word(const uint32_t* __restrict__ mrow,
 // MODE 0: the kept tiles of row `mrow`, then landmark blocks with at least one
 // visible landmark, then special blocks.
 __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, const uint32_t* __restrict__ mrow,
-                                                  int t, bool has_lmk, int& kind, int& id) {
+                                                  int t, bool has_lmk, int& kind, int& id, int& nv) {
   if (it.phase == 0) {
     while (it.bits == 0 && it.w + 1 < g.W) {
       ++it.w;
@@ -64,6 +74,8 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
       it.bits &= it.bits - 1;
       kind = 0;
       id = it.w * 32 + b;
+      const TileShape ts = tile_shape(g, id);
+      nv = ts.rows * ts.cols;
       return true;
     }
     it.phase = 1;
@@ -74,6 +86,7 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
       while (it.lb < nlb) {
         const int lb = it.lb++;
         uint32_t vis = 0;
+        int nvis = 0;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int w = lb * 2 + k;
@@ -84,10 +97,12 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
           uint32_t v = ~__ldg(mrow + w) & inr;
           if ((t >> 5) == w) v &= ~(1u << (t & 31));
           vis |= v;
+          nvis += __popc(v);
         }
         if (vis) {
           kind = 1;
           id = lb;
+          nv = nvis;
           return true;
         }
       }
@@ -98,6 +113,7 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
     if (it.sb < g.NSp / 64) {
       kind = 2;
       id = it.sb++;
+      nv = min(64, g.NS - id * 64);
       return true;
     }
     it.phase = 3;
@@ -106,11 +122,14 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
 }
 
 // MODE 1: tiles [w, t_end), then the special blocks when `with_special`.
-__device__ __forceinline__ bool next_block_dense(BlockIter& it, const Geo& g, bool with_special, int& kind, int& id) {
+__device__ __forceinline__ bool next_block_dense(BlockIter& it, const Geo& g, bool with_special, int& kind, int& id,
+                                                 int& nv) {
   if (it.phase == 0) {
     if (it.w < it.t_end) {
       kind = 0;
       id = it.w++;
+      const TileShape ts = tile_shape(g, id);
+      nv = ts.rows * ts.cols;
       return true;
     }
     it.phase = 2;
@@ -118,6 +137,7 @@ __device__ __forceinline__ bool next_block_dense(BlockIter& it, const Geo& g, bo
   if (it.phase == 2 && with_special && it.sb < g.NSp / 64) {
     kind = 2;
     id = it.sb++;
+    nv = min(64, g.NS - id * 64);
     return true;
   }
   it.phase = 3;
@@ -189,8 +209,13 @@ __device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+// round a pair to bf16 in place and return it packed: the softmax sum then uses
+// exactly the weights that enter the PV product
+__device__ __forceinline__ uint32_t pack_round(float& lo, float& hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  const float2 f = __bfloat1622float2(v);
+  lo = f.x;
+  hi = f.y;
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -257,10 +282,14 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
     if (tid < 64) sm.bias[buf][tid] = block_bias(a, mrow, t, kind, id, tid);
   };
 
-  int kind = 0, id = 0;
-  bool have = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, kind, id)
-                        : next_block_dense(it, g, with_special, kind, id);
-  if (have) issue(kind, id, 0);
+  int kind = 0, id = 0, nv = 0;
+  long long keys = 0;  // visible keys per query row, summed over blocks
+  bool have = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, kind, id, nv)
+                        : next_block_dense(it, g, with_special, kind, id, nv);
+  if (have) {
+    issue(kind, id, 0);
+    keys += nv;
+  }
   cp_async_commit();
 
   const float sc = LOG2E * 0.125f;  // log2(e) / sqrt(64)
@@ -274,10 +303,13 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
 
   int buf = 0;
   while (have) {
-    int nkind = 0, nid = 0;
-    const bool nhave = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, nkind, nid)
-                                 : next_block_dense(it, g, with_special, nkind, nid);
-    if (nhave) issue(nkind, nid, buf ^ 1);
+    int nkind = 0, nid = 0, nnv = 0;
+    const bool nhave = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, nkind, nid, nnv)
+                                 : next_block_dense(it, g, with_special, nkind, nid, nnv);
+    if (nhave) {
+      issue(nkind, nid, buf ^ 1);
+      keys += nnv;
+    }
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
@@ -330,12 +362,15 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
     m0 = mn0;
     m1 = mn1;
     float rs0 = 0.f, rs1 = 0.f;
+    uint32_t pk[8][2];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       s[j][0] = fast_exp2(s[j][0] - base0);
       s[j][1] = fast_exp2(s[j][1] - base0);
       s[j][2] = fast_exp2(s[j][2] - base1);
       s[j][3] = fast_exp2(s[j][3] - base1);
+      pk[j][0] = pack_round(s[j][0], s[j][1]);
+      pk[j][1] = pack_round(s[j][2], s[j][3]);
       rs0 += s[j][0] + s[j][1];
       rs1 += s[j][2] + s[j][3];
     }
@@ -351,10 +386,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      pa[0] = pk[2 * kk][0];
+      pa[1] = pk[2 * kk][1];
+      pa[2] = pk[2 * kk + 1][0];
+      pa[3] = pk[2 * kk + 1][1];
 #pragma unroll
       for (int dp = 0; dp < 4; ++dp) {
         const int mi = lane >> 3, ri = lane & 7;
@@ -373,6 +408,11 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   }
   cp_async_wait<0>();
   if (!qloaded) __syncthreads();
+  if (tid == 0) {
+    const long long rows = MODE == 0 ? n_t : min(64, g.NS - t * 64);
+    const long long extra = (MODE == 0 && !own_kept) ? (n_t > 1 ? 2 : 1) : 0;
+    atomicAdd(&g_logits[MODE], (unsigned long long)(rows * (keys + extra)));
+  }
 
   const int r0 = warp * 16 + g4, r1 = r0 + 8;
   if (MODE == 0) {
@@ -508,8 +548,9 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(const __grid_constant__ A
     it.t_end = (int)((long long)g.T * (sp + 1) / a.splits);
     with_special = sp == 0;
   }
-  int kind, id;
-  while (MODE == 0 ? next_block_sparse(it, g, mrow, t, true, kind, id) : next_block_dense(it, g, with_special, kind, id)) {
+  int kind, id, nv;
+  while (MODE == 0 ? next_block_sparse(it, g, mrow, t, true, kind, id, nv)
+                   : next_block_dense(it, g, with_special, kind, id, nv)) {
     const float *ks, *vs;
     block_src<float>(a, h, kind, id, ks, vs);
     __syncthreads();
@@ -607,6 +648,7 @@ int launch_sparse_attn<__nv_bfloat16>(const AttnArgs& a, cudaStream_t st) {
   if (a.g.T == 0) return ZEBRA_OK;
   const size_t smem = sizeof(MmaSmem);
   cudaFuncSetAttribute(attn_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  ProfScope prof("attn_sparse_rows", st);
   attn_mma_kernel<0><<<dim3(a.g.T, a.g.H), 128, smem, st>>>(a);
   count_launch();
   return check_launch("attn_mma_kernel<sparse>");
@@ -614,6 +656,7 @@ int launch_sparse_attn<__nv_bfloat16>(const AttnArgs& a, cudaStream_t st) {
 template <>
 int launch_sparse_attn<float>(const AttnArgs& a, cudaStream_t st) {
   if (a.g.T == 0) return ZEBRA_OK;
+  ProfScope prof("attn_sparse_rows_f32", st);
   attn_simt_kernel<0><<<dim3(a.g.T, a.g.H), 64, 0, st>>>(a);
   count_launch();
   return check_launch("attn_simt_kernel<sparse>");
@@ -623,6 +666,8 @@ template <typename T>
 int launch_special_rows(const AttnArgs& a, cudaStream_t st) {
   if (a.g.NS == 0) return ZEBRA_OK;
   dim3 grid(a.g.NSp / 64, a.g.H, a.splits);
+  {
+  ProfScope prof("attn_special_rows", st);
   if (sizeof(T) == 2) {
     const size_t smem = sizeof(MmaSmem);
     cudaFuncSetAttribute(attn_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -630,10 +675,12 @@ int launch_special_rows(const AttnArgs& a, cudaStream_t st) {
   } else {
     attn_simt_kernel<1><<<grid, 64, 0, st>>>(a);
   }
+  }
   count_launch();
   int rc = check_launch("attn_kernel<special rows>");
   if (rc) return rc;
   const long long threads = (long long)a.g.NS * a.g.H * 32;
+  ProfScope prof("special_combine", st);
   special_combine_kernel<T><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(a);
   count_launch();
   return check_launch("special_combine_kernel");

@@ -133,6 +133,21 @@ void set_error(const std::string& msg);
 void count_launch(int n = 1);
 int check_launch(const char* what);   // ZEBRA_OK or ZEBRA_ERR_CUDA (sets the message)
 
+// Optional per-kernel timing: while profiling is on (zebra_profile_enable), a
+// ProfScope records a CUDA event on `st` when it is made and another when it
+// goes out of scope, around one kernel launch.
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st;
+  ProfScope(const char* name, cudaStream_t st);
+  ~ProfScope();
+};
+
+// visible-logit counters of the attention kernels (per device): [0] patch rows
+// of the sparse kernel, [1] special-token rows
+void reset_logit_counters();
+void read_logit_counters(unsigned long long* out2);
+
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Bump allocator over the caller's workspace.

@@ -52,9 +52,9 @@ int gemm_bf16_nt(const void* A, const void* B, const void* Cin, void* Cout, long
   if (s == CUBLAS_STATUS_SUCCESS && found == 0) s = CUBLAS_STATUS_NOT_SUPPORTED;
   if (s == CUBLAS_STATUS_SUCCESS) {
     const float alpha = 1.0f;
+    ProfScope prof("cublasLt_gemm", st);
     s = cublasLtMatmul(h, op, &alpha, B, la, A, lb, &beta, beta != 0.f ? Cin : Cout, lc, Cout, lc, &res.algo, ws,
                        ws_bytes, st);
-    count_launch();
   }
   if (s != CUBLAS_STATUS_SUCCESS) {
     set_error(std::string("cuBLASLt matmul failed, status ") + std::to_string((int)s));

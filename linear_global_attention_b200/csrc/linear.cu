@@ -459,13 +459,22 @@ int linear_chunks(const Geo& g, int* chunk_tokens) {
 template <>
 int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
-  linear_state_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  {
+    ProfScope prof("linear_state", st);
+    linear_state_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  }
   count_launch();
   if (int rc = check_launch("linear_state_kernel")) return rc;
-  linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 1);
+  {
+    ProfScope prof("linear_reduce", st);
+    linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 1);
+  }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
-  linear_apply_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  {
+    ProfScope prof("linear_apply", st);
+    linear_apply_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+  }
   count_launch();
   return check_launch("linear_apply_kernel");
 }
@@ -473,13 +482,22 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
 template <>
 int launch_linear<float>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
-  linear_state_simt_kernel<<<dim3(a.chunks, a.g.H), 256, 0, st>>>(a);
+  {
+    ProfScope prof("linear_state_simt", st);
+    linear_state_simt_kernel<<<dim3(a.chunks, a.g.H), 256, 0, st>>>(a);
+  }
   count_launch();
   if (int rc = check_launch("linear_state_simt_kernel")) return rc;
-  linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 0);
+  {
+    ProfScope prof("linear_reduce", st);
+    linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 0);
+  }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
-  linear_apply_simt_kernel<<<dim3((unsigned)((a.g.N + 127) / 128), a.g.H), 128, 0, st>>>(a);
+  {
+    ProfScope prof("linear_apply_simt", st);
+    linear_apply_simt_kernel<<<dim3((unsigned)((a.g.N + 127) / 128), a.g.H), 128, 0, st>>>(a);
+  }
   count_launch();
   return check_launch("linear_apply_simt_kernel");
 }

@@ -175,6 +175,7 @@ int launch_pool_pack(const PoolArgs<T>& a, int ntensors, cudaStream_t st) {
   if (a.g.T == 0) return ZEBRA_OK;
   constexpr int HPC = 128 / (D / Elem<T>::PER16);
   dim3 grid(a.g.Tpad, (a.g.H + HPC - 1) / HPC, ntensors);
+  ProfScope prof("pool_pack", st);
   pool_pack_kernel<T><<<grid, 128, 0, st>>>(a);
   count_launch();
   return check_launch("pool_pack_kernel");
@@ -185,6 +186,7 @@ int launch_pack_special(const SpecialArgs<T>& a, int ntensors, cudaStream_t st) 
   const long long threads = (long long)a.g.NSp * a.g.H * (D / Elem<T>::PER16);
   if (threads == 0) return ZEBRA_OK;
   dim3 grid((unsigned)((threads + 127) / 128), 1, ntensors);
+  ProfScope prof("pack_special", st);
   pack_special_kernel<T><<<grid, 128, 0, st>>>(a);
   count_launch();
   return check_launch("pack_special_kernel");
@@ -192,6 +194,7 @@ int launch_pack_special(const SpecialArgs<T>& a, int ntensors, cudaStream_t st) 
 
 int launch_rope_table(float2* tab, int maxpos, double base, cudaStream_t st) {
   const int n = maxpos * 16;
+  ProfScope prof("rope_table", st);
   rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, maxpos, base);
   count_launch();
   return check_launch("rope_table_kernel");

@@ -223,6 +223,7 @@ int launch_scores(const SelectArgs& a, cudaStream_t st) {
   const int T = a.g.T;
   if (T == 0 || a.keep >= T) return ZEBRA_OK;
   dim3 grid((T + 63) / 64, (T + 63) / 64, a.hc);
+  ProfScope prof("tile_scores", st);
   scores_kernel<<<grid, 256, 0, st>>>(a);
   count_launch();
   return check_launch("scores_kernel");
@@ -232,12 +233,9 @@ int launch_select(const SelectArgs& a, cudaStream_t st) {
   const int T = a.g.T;
   if (T == 0) return ZEBRA_OK;
   const size_t smem = (size_t)T * sizeof(uint32_t);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SELECT_MAX_T * 4);
-    attr_set = true;
-  }
+  cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SELECT_MAX_T * 4);
   dim3 grid(T, a.hc);
+  ProfScope prof("tile_select", st);
   select_kernel<<<grid, SEL_THREADS, smem, st>>>(a);
   count_launch();
   return check_launch("select_kernel");

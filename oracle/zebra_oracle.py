@@ -192,13 +192,15 @@ def _softmax_weighted_sum(logits: np.ndarray, values: np.ndarray) -> np.ndarray:
     return (p @ values) / p.sum(axis=-1, keepdims=True)
 
 
-def dense_attention(q_h, k_h, v_h, rows=None, chunk=1024) -> np.ndarray:
-    """Plain softmax(q k^T / sqrt(d)) v for one head; `rows` selects query rows."""
+def dense_attention(q_h, k_h, v_h, rows=None) -> np.ndarray:
+    """Plain softmax(q k^T / sqrt(d)) v for one head; `rows` selects query rows
+    (processed a few at a time so that one block of logits stays near 64 MB)."""
     k_h = np.asarray(k_h, np.float64)
     v_h = np.asarray(v_h, np.float64)
     q_h = np.asarray(q_h, np.float64)
     rows = np.arange(q_h.shape[0]) if rows is None else np.asarray(rows)
     d = q_h.shape[-1]
+    chunk = max(1, min(1024, (1 << 23) // max(k_h.shape[0], 1)))
     out = np.empty((len(rows), d))
     for a in range(0, len(rows), chunk):
         r = rows[a:a + chunk]
@@ -270,8 +272,9 @@ def sparse_stage(q, k, v, g: Geom, keep: int, query_tiles=None, special_rows=Non
             keys = np.concatenate([kh[exact], k_spec, k_mean[lm]])
             vals = np.concatenate([vh[exact], v_spec, v_mean[lm]])
             bias = np.concatenate([np.zeros(len(exact) + len(specials)), np.log(counts[lm])])
-            logits = Qt @ keys.T * scale + bias                         # [n_t, E]
-            values = np.broadcast_to(vals, (len(mine),) + vals.shape)   # [n_t, E, d]
+            logits = Qt @ keys.T * scale + bias                         # [n_t, E], shared entries
+            ex_logits = np.zeros((len(mine), 0))                        # per-query entries
+            ex_values = np.zeros((len(mine), 0, d))
             if not sel[a, t]:
                 # own tile unselected: exact self key + landmark of the other n_t - 1 tokens (R7)
                 n_t = counts[t]
@@ -284,11 +287,14 @@ def sparse_stage(q, k, v, g: Geom, keep: int, query_tiles=None, special_rows=Non
                     v_rest = (vh[mine].sum(0)[None, :] - vh[mine]) / m
                     extra_logits.append((np.einsum("ij,ij->i", Qt, k_rest) * scale + math.log(m))[:, None])
                     extra_values.append(v_rest[:, None, :])
-                logits = np.concatenate([logits] + extra_logits, axis=1)
-                values = np.concatenate([values] + extra_values, axis=1)
-            mx = logits.max(axis=1, keepdims=True)
+                ex_logits = np.concatenate(extra_logits, axis=1)
+                ex_values = np.concatenate(extra_values, axis=1)
+            # one softmax over the shared and the per-query entries together
+            mx = np.maximum(logits.max(axis=1, initial=-np.inf), ex_logits.max(axis=1, initial=-np.inf))[:, None]
             p = np.exp(logits - mx)
-            o = np.einsum("ie,ied->id", p, values) / p.sum(axis=1, keepdims=True)
+            pe = np.exp(ex_logits - mx)
+            num = p @ vals + np.einsum("ie,ied->id", pe, ex_values)
+            o = num / (p.sum(axis=1, keepdims=True) + pe.sum(axis=1, keepdims=True))
             for i, n in enumerate(mine):
                 out[pos[int(n)], h] = o[i]
 
