@@ -608,6 +608,9 @@ long long zebra_profile_report(char* buf, size_t len) {
 int zebra_sync_status(void* stream) {
   const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(ZEBRA_ERR_CUDA, cudaGetErrorString(e));
+  int st = 0;
+  if (read_and_clear_status(&st) != ZEBRA_OK) return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
+  if (st) return fail(ZEBRA_ERR_TIMEOUT, "a device-side wait gave up (kernel aborted; outputs are invalid)");
   return ZEBRA_OK;
 }
 

@@ -640,18 +640,18 @@ __global__ void special_combine_kernel(const __grid_constant__ AttnArgs a) {
   dst[1] = Elem<T>::from_f(o1 / l);
 }
 
+}  // namespace zebra
+
+#include "attn_tc.cuh"
+
+namespace zebra {
+
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
 template <>
 int launch_sparse_attn<__nv_bfloat16>(const AttnArgs& a, cudaStream_t st) {
-  if (a.g.T == 0) return ZEBRA_OK;
-  const size_t smem = sizeof(MmaSmem);
-  cudaFuncSetAttribute(attn_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  ProfScope prof("attn_sparse_rows", st);
-  attn_mma_kernel<0><<<dim3(a.g.T, a.g.H), 128, smem, st>>>(a);
-  count_launch();
-  return check_launch("attn_mma_kernel<sparse>");
+  return launch_sparse_attn_tc(a, st);
 }
 template <>
 int launch_sparse_attn<float>(const AttnArgs& a, cudaStream_t st) {

@@ -1,0 +1,567 @@
+// Tile-sparse softmax attention on the 5th-generation tensor cores (tcgen05).
+//
+// Page "How Hybrid Attention Lets Feed-Forward 3D Models Scale to Many Views",
+// section "Linear-centered stages plus tile-sparse stages": selected tiles keep
+// full softmax interactions, omitted tiles become mean key/value landmarks,
+// special-token keys stay visible and each patch query keeps its self key.
+// Section "Speedup scales with the number of input views": keys and values are
+// packed tile-major, so every kept tile is one contiguous 64x64 block.
+//
+// One CTA = one (query tile, head): a 64-row query block against the stream of
+// 64-key blocks (kept tiles, landmark blocks, special-key blocks) described in
+// attn.cu. Warp roles:
+//   warp 0      TMA producer: Q once, then K and V of each block into a
+//               3-stage ring (128-byte swizzled 64x64 bf16 tiles);
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
+//               score buffers (tcgen05.mma M=64 N=64, K-major A/B), then
+//               O += P V with P from shared memory (K-major) and V MN-major;
+//   warps 2..5  softmax warpgroup: tcgen05.ld of S (16x256b: rows spread over
+//               quads as in the m16n8 accumulator), scale + bias, running max,
+//               exp2, bf16 P into shared memory, and O rescaling in TMEM only
+//               when a row maximum grows by more than 2^8 (the stale maximum is
+//               exact as long as both the sum and O use it).
+// TMEM: S0 at column 0, S1 at 64, O at 128 (256 columns allocated); M=64
+// accumulators occupy lanes 0-15, 32-47, 64-79, 96-111, i.e. 16 rows per
+// softmax warp. Every mbarrier wait is bounded by the global timer; on expiry
+// the CTA records ZEBRA_ERR_TIMEOUT in a device status word, drains its own
+// copies and MMAs (bounded again), frees TMEM and exits.
+// Included by attn.cu (one translation unit with the block iterator and the
+// device counters).
+#pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace zebra {
+
+__device__ int g_status;   // sticky device status word (0 = ok)
+
+int read_and_clear_status(int* out) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e != cudaSuccess) return ZEBRA_ERR_CUDA;
+  const int z = 0;
+  e = cudaMemcpyToSymbol(g_status, &z, sizeof(int));
+  if (e != cudaSuccess) return ZEBRA_ERR_CUDA;
+  *out = v;
+  return ZEBRA_OK;
+}
+
+namespace tc {
+
+constexpr int STAGES = 3;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t COL_S0 = 0, COL_S1 = 64, COL_O = 128;
+constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
+
+struct __align__(1024) Smem {
+  __nv_bfloat16 q[64 * 64];
+  __nv_bfloat16 k[STAGES][64 * 64];
+  __nv_bfloat16 v[STAGES][64 * 64];
+  __nv_bfloat16 p[2][64 * 64];
+  uint64_t q_full;
+  uint64_t kv_full[STAGES];
+  uint64_t kv_empty[STAGES];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+// keep two CTAs per SM at most: their TMEM (2 x 256 columns) fills the SM
+constexpr size_t SMEM_BYTES = 80 * 1024;
+static_assert(sizeof(Smem) + 1024 <= SMEM_BYTES, "shared memory layout");
+
+struct alignas(64) Params {
+  CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs;
+  AttnArgs a;
+};
+
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long gtime() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete. Gives up after `limit_ns`, or
+// early once another warp has raised the abort flag; a timeout records the
+// error status and raises the flag. Returns true when the phase completed.
+__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                       unsigned long long limit_ns = WAIT_NS) {
+  if (mbar_try(b, parity)) return true;
+  const unsigned long long t0 = gtime();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(b, parity)) return true;
+    if ((i & 255) == 0) {
+      if (*abort_flag) return false;
+      if (gtime() - t0 > limit_ns) {
+        atomicExch(&g_status, ZEBRA_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// shared-memory matrix descriptors (sm_100 format: start>>4 at [0,14), LBO>>4 at
+// [16,30), SBO>>4 at [32,46), version 1 at [46,48), layout at [61,64): 2 = 128B swizzle)
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// K-major 64-row tile with 128-byte rows: 8-row groups 1024 bytes apart
+__device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return desc_sw128(addr, 16, 1024); }
+// MN-major tile: the 64 N values of a K row fill one 128-byte swizzle atom,
+// K rows 128 bytes apart, 8-row groups 1024 bytes apart
+__device__ __forceinline__ uint64_t desc_mn(uint32_t addr) { return desc_sw128(addr, 8192, 1024); }
+
+// instruction descriptor of kind::f16: D fp32, A/B bf16, M = 64, N = 64
+__host__ __device__ constexpr uint32_t idesc(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((64u >> 3) << 17) |
+         ((64u >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(accum));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(bar))
+               : "memory");
+}
+
+// 16 TMEM lanes x 64 fp32 columns -> 32 registers (m16n8 accumulator layout per 8 columns)
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* r) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+        "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+        "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+        "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* r) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+      "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15]), "r"(u[16]), "r"(u[17]),
+      "r"(u[18]), "r"(u[19]), "r"(u[20]), "r"(u[21]), "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]),
+      "r"(u[27]), "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_round(float& lo, float& hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  const float2 f = __bfloat1622float2(v);
+  lo = f.x;
+  hi = f.y;
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// rows of block `id` of `kind` in the 2D [rows, 64] tensor map of its source
+__device__ __forceinline__ int block_row(const Geo& g, int h, int kind, int id) {
+  if (kind == 0) return (h * g.T + id) * 64;
+  if (kind == 1) return h * g.Tpad + id * 64;
+  return h * g.NSp + id * 64;
+}
+
+__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_constant__ Params P) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const AttnArgs& a = P.a;
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = blockIdx.x, h = blockIdx.y;
+  const uint32_t* mrow = a.mask + ((size_t)h * g.T + t) * g.W;
+  volatile int* abort_flag = &sm.abort;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], 4);
+      mbar_init(&sm.p_full[b], 4);
+      mbar_init(&sm.pv_done[b], 1);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sm.tmem_base)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  const bool own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
+  const TileShape ts = tile_shape(g, t);
+  const int n_t = ts.rows * ts.cols;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
+      tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+      BlockIter it{};
+      it.bits = mask_word(mrow, 0, g.T);
+      int kind, id, nv;
+      while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+        const int s = issued % STAGES;
+        if (issued >= STAGES && !mbar_wait(&sm.kv_empty[s], ((issued / STAGES) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&sm.kv_full[s], 2 * 64 * 64 * 2);
+        const CUtensorMap* mk = kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks;
+        const CUtensorMap* mv = kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs;
+        const int row = block_row(g, h, kind, id);
+        tma_load_2d(sm.k[s], mk, 0, row, &sm.kv_full[s]);
+        tma_load_2d(sm.v[s], mv, 0, row, &sm.kv_full[s]);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA goes away
+        mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
+        for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+          mbar_wait(&sm.kv_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id_qk = idesc(false), id_pv = idesc(true);
+      const uint64_t dq = desc_k(saddr(sm.q));
+      bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+      int i = 0;
+      auto issue_pv = [&](int j) -> bool {
+        const int b = j & 1, s = j % STAGES;
+        if (!mbar_wait(&sm.p_full[b], (j >> 1) & 1, abort_flag)) return false;
+        fence_after();
+        const uint64_t dp = desc_k(saddr(sm.p[b]));
+        const uint64_t dv = desc_mn(saddr(sm.v[s]));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + COL_O, dp + 2 * kk, dv + (uint64_t)(2048 >> 4) * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.kv_empty[s]);
+        mma_commit(&sm.pv_done[b]);
+        return true;
+      };
+      if (ok) {
+        BlockIter it{};
+        it.bits = mask_word(mrow, 0, g.T);
+        int kind, id, nv;
+        while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+          const int s = i % STAGES, b = i & 1;
+          if (!mbar_wait(&sm.kv_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
+          if (i >= 2 && !mbar_wait(&sm.s_free[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          fence_after();
+          const uint64_t dk = desc_k(saddr(sm.k[s]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + (b ? COL_S1 : COL_S0), dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
+          mma_commit(&sm.s_full[b]);
+          if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+          ++i;
+        }
+        if (ok && i >= 1) issue_pv(i - 1);
+      }
+      // drain: every MMA this thread issued completes before TMEM is freed
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, abort_flag, *abort_flag ? DRAIN_NS : WAIT_NS);
+    }
+  } else {
+    // ---------------- softmax warpgroup ----------------
+    const int rb = warp & 3;                  // TMEM lane quarter this warp may access
+    const int g4 = lane >> 2, q4 = lane & 3;
+    const uint32_t lane_off = (uint32_t)(32 * rb) << 16;
+    const float sc = LOG2E * 0.125f;
+    const float NEG = -INFINITY;
+    float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
+    const int r0 = 16 * rb + g4, r1 = r0 + 8;  // query rows of this thread
+    unsigned char* pbase[2] = {reinterpret_cast<unsigned char*>(sm.p[0]), reinterpret_cast<unsigned char*>(sm.p[1])};
+    BlockIter it{};
+    it.bits = mask_word(mrow, 0, g.T);
+    int kind, id, nv;
+    int i = 0;
+    bool ok = true;
+    long long keys = 0;
+    while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+      keys += nv;
+      const int b = i & 1;
+      if (!mbar_wait(&sm.s_full[b], (i >> 1) & 1, abort_flag)) { ok = false; break; }
+      fence_after();
+      float s[32];
+      tmem_ld64(tmem + lane_off + (b ? COL_S1 : COL_S0), s);
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+
+      // scale, bias (log2 units) and row maxima
+      float mx0 = NEG, mx1 = NEG;
+      const bool full_tile = kind == 0 && nv == 64;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = 8 * j + 2 * q4 + e;
+          float bias = 0.f;
+          if (!full_tile) bias = kind == 1 ? block_bias(a, mrow, t, kind, id, col) : (col < nv ? 0.f : NEG);
+          s[4 * j + e] = fmaf(s[4 * j + e], sc, bias);
+          s[4 * j + 2 + e] = fmaf(s[4 * j + 2 + e], sc, bias);
+          mx0 = fmaxf(mx0, s[4 * j + e]);
+          mx1 = fmaxf(mx1, s[4 * j + 2 + e]);
+        }
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      // lazy maximum: move it only when the block exceeds it by more than 8 (x256)
+      const bool up0 = mx0 > m0 + 8.f, up1 = mx1 > m1 + 8.f;
+      const float mn0 = up0 ? mx0 : m0, mn1 = up1 ? mx1 : m1;
+      const float base0 = mn0 == NEG ? 0.f : mn0, base1 = mn1 == NEG ? 0.f : mn1;
+      const float al0 = up0 ? fast_exp2(m0 - base0) : 1.f, al1 = up1 ? fast_exp2(m1 - base1) : 1.f;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t pk[8][2];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        s[4 * j + 0] = fast_exp2(s[4 * j + 0] - base0);
+        s[4 * j + 1] = fast_exp2(s[4 * j + 1] - base0);
+        s[4 * j + 2] = fast_exp2(s[4 * j + 2] - base1);
+        s[4 * j + 3] = fast_exp2(s[4 * j + 3] - base1);
+        pk[j][0] = pack_round(s[4 * j + 0], s[4 * j + 1]);
+        pk[j][1] = pack_round(s[4 * j + 2], s[4 * j + 3]);
+        rs0 += s[4 * j + 0] + s[4 * j + 1];
+        rs1 += s[4 * j + 2] + s[4 * j + 3];
+      }
+      l0 = l0 * al0 + rs0;
+      l1 = l1 * al1 + rs1;
+      m0 = mn0;
+      m1 = mn1;
+      // P buffer b is free once PV of block i-2 has completed
+      if (i >= 2 && !mbar_wait(&sm.pv_done[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t cb = (uint32_t)(((j ^ (r0 & 7)) << 4) + 4 * q4);
+        *reinterpret_cast<uint32_t*>(pbase[b] + r0 * 128 + cb) = pk[j][0];
+        const uint32_t cb1 = (uint32_t)(((j ^ (r1 & 7)) << 4) + 4 * q4);
+        *reinterpret_cast<uint32_t*>(pbase[b] + r1 * 128 + cb1) = pk[j][1];
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // rescale O (TMEM) when any row of this warp moved its maximum
+      if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
+        const int jp = i - 1;
+        if (!mbar_wait(&sm.pv_done[jp & 1], (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+        fence_after();
+        float o[32];
+        tmem_ld64(tmem + lane_off + COL_O, o);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          o[4 * j + 0] *= al0;
+          o[4 * j + 1] *= al0;
+          o[4 * j + 2] *= al1;
+          o[4 * j + 3] *= al1;
+        }
+        tmem_st64(tmem + lane_off + COL_O, o);
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[b]);
+      ++i;
+    }
+    const int nb = i;
+    // ---------------- epilogue ----------------
+    if (ok && nb >= 1 && !mbar_wait(&sm.pv_done[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag)) ok = false;
+    if (ok) {
+      fence_after();
+      float o[32];
+      if (nb >= 1) {
+        tmem_ld64(tmem + lane_off + COL_O, o);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = 0.f;
+      }
+      if (!own_kept) {
+        // exact self key + landmark of the other n_t - 1 tokens of the own tile
+        const size_t tb = ((size_t)h * g.T + t) * TOK * D;
+        const __nv_bfloat16* Qp = static_cast<const __nv_bfloat16*>(a.Qp) + tb;
+        const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp) + tb;
+        const __nv_bfloat16* Vp = static_cast<const __nv_bfloat16*>(a.Vp) + tb;
+        const float* km = a.km + ((size_t)h * g.T + t) * D;
+        const float* vm = a.vm + ((size_t)h * g.T + t) * D;
+        const float nt = (float)n_t;
+        const float inv = n_t > 1 ? 1.0f / (float)(n_t - 1) : 0.f;
+        const float lnb = n_t > 1 ? a.ln_tab[n_t - 1] * LOG2E : 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = half ? r1 : r0;
+          float qk = 0.f, qm = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 8 * j + 2 * q4 + e;
+              const float qv = __bfloat162float(Qp[r * D + c]);
+              qk = fmaf(qv, __bfloat162float(Kp[r * D + c]), qk);
+              qm = fmaf(qv, km[c], qm);
+            }
+          }
+          qk += __shfl_xor_sync(0xffffffffu, qk, 1);
+          qk += __shfl_xor_sync(0xffffffffu, qk, 2);
+          qm += __shfl_xor_sync(0xffffffffu, qm, 1);
+          qm += __shfl_xor_sync(0xffffffffu, qm, 2);
+          const float s_self = qk * sc;
+          const float s_lm = n_t > 1 ? (nt * qm - qk) * inv * sc + lnb : NEG;
+          float& m = half ? m1 : m0;
+          float& l = half ? l1 : l0;
+          const float mn = fmaxf(m, fmaxf(s_self, s_lm));
+          const float al = fast_exp2(m - mn), ps = fast_exp2(s_self - mn);
+          const float pl = n_t > 1 ? fast_exp2(s_lm - mn) : 0.f;
+          m = mn;
+          l = l * al + (q4 == 0 ? ps + pl : 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 8 * j + 2 * q4 + e;
+              const float vv = __bfloat162float(Vp[r * D + c]);
+              const float vl = (nt * vm[c] - vv) * inv;
+              float& oo = o[4 * j + half * 2 + e];
+              oo = oo * al + ps * vv + pl * vl;
+            }
+          }
+        }
+      }
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = half ? r1 : r0;
+        if (r >= n_t) continue;
+        const float il = 1.0f / (half ? l1 : l0);
+        __nv_bfloat16* dst = out + (tile_token(g, ts, r) * g.H + h) * D;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = 8 * j + 2 * q4;
+          *reinterpret_cast<__nv_bfloat162*>(dst + c) =
+              __floats2bfloat162_rn(o[4 * j + half * 2] * il, o[4 * j + half * 2 + 1] * il);
+        }
+      }
+      if (tid == 64) {
+        const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);
+        atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (keys + extra)));
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 map over [rows, 64] with a 64 x 64 box and 128-byte swizzle
+static bool make_map(CUtensorMap* m, const void* base, unsigned long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (rows == 0) rows = 64;  // never read: keep the encoder happy
+  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) {
+  const Geo& g = a.g;
+  if (g.T == 0) return ZEBRA_OK;
+  tc::Params p;
+  p.a = a;
+  const unsigned long long tile_rows = (unsigned long long)g.H * g.T * 64;
+  bool ok = make_map(&p.tq, a.Qp, tile_rows) && make_map(&p.tk, a.Kp, tile_rows) && make_map(&p.tv, a.Vp, tile_rows) &&
+            make_map(&p.tkl, a.Kl, (unsigned long long)g.H * g.Tpad) &&
+            make_map(&p.tvl, a.Vl, (unsigned long long)g.H * g.Tpad) &&
+            make_map(&p.tks, a.Ks, (unsigned long long)g.H * g.NSp) &&
+            make_map(&p.tvs, a.Vs, (unsigned long long)g.H * g.NSp);
+  if (!ok) {
+    set_error("cuTensorMapEncodeTiled failed");
+    return ZEBRA_ERR_CUDA;
+  }
+  cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
+  ProfScope prof("attn_sparse_rows", st);
+  tc::attn_tc_kernel<<<dim3(g.T, g.H), tc::THREADS, tc::SMEM_BYTES, st>>>(p);
+  count_launch();
+  return check_launch("attn_tc_kernel");
+}
+
+}  // namespace zebra

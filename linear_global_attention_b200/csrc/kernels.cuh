@@ -66,6 +66,9 @@ struct AttnArgs {
   float ln_tab[TOK + 1];                              // ln(m), m = 0..64 (ln_tab[0] unused)
 };
 template <typename T> int launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
+int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st);
+// sticky device status word of the kernels with bounded waits (per device)
+int read_and_clear_status(int* out);
 template <typename T> int launch_special_rows(const AttnArgs& a, cudaStream_t st);
 
 // ---- linear stage ----
