@@ -42,15 +42,22 @@ def _newest_header() -> float:
     return max((os.path.getmtime(h) for h in hs), default=0.0)
 
 
-def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
+def build(verbose: bool = False, force: bool = False, extra_flags=None, out: str = None) -> str:
+    """Compile every csrc/*.cu and link the shared library (default: next to this file).
+
+    `extra_flags` (e.g. ["-DZEBRA_TC_STAGES=6"]) and `out` build a variant into
+    its own object directory and library path.
+    """
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    lib = out or LIB
+    build_dir = BUILD if not out else os.path.join(BUILD, "variant_" + os.path.basename(out).replace(".", "_"))
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = _newest_header()
     flags = NVCC_FLAGS + list(extra_flags or [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_t):
             return obj, ""
         cmd = [nvcc, *ARCH, *flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
@@ -68,15 +75,22 @@ def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
                 print(f"--- {os.path.basename(o)}\n{log}", file=sys.stderr)
     libdir = _cuda_lib_dir(nvcc)
     newest_obj = max(os.path.getmtime(o) for o in objs)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest_obj:
-        cmd = [nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *objs, "-L", libdir, "-lcublasLt",
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < newest_obj:
+        cmd = [nvcc, *ARCH, "-shared", "-o", lib + ".tmp", *objs, "-L", libdir, "-lcublasLt",
                "-Xlinker", f"-rpath,{libdir}"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+        os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv, force="-f" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("-v", action="store_true")
+    ap.add_argument("-f", action="store_true")
+    ap.add_argument("--define", action="append", default=[], help="extra -D definitions, e.g. ZEBRA_TC_STAGES=6")
+    ap.add_argument("--out", default=None, help="library path of a variant build")
+    a = ap.parse_args()
+    print(build(verbose=a.v, force=a.f, extra_flags=["-D" + d for d in a.define], out=a.out))

@@ -550,7 +550,14 @@ int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void*
     const int keep = kind == ZEBRA_LAYER_DENSE ? G.T : keep_of(y, G.T);
     ZTRY(run_sparse<__nv_bfloat16>(G, q, k, v, ts, hs, keep, nullptr, w.o, w.sp, true, rope_base, eps, st));
   }
-  return gemm_bf16_nt(w.o, w_o, x, x_out, G.N, Dm, Dm, 1.f, w.gemm_ws, GEMM_WS_BYTES, st);
+  if (x_out != x) return gemm_bf16_nt(w.o, w_o, x, x_out, G.N, Dm, Dm, 1.f, w.gemm_ws, GEMM_WS_BYTES, st);
+  // In place: a GEMM whose C and D alias may read C after writing D, so the
+  // result goes to the QKV scratch (no longer needed) and is then copied over x.
+  ZTRY(gemm_bf16_nt(w.o, w_o, x, w.qkv, G.N, Dm, Dm, 1.f, w.gemm_ws, GEMM_WS_BYTES, st));
+  const cudaError_t e = cudaMemcpyAsync(x_out, w.qkv, (size_t)G.N * Dm * sizeof(__nv_bfloat16),
+                                        cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(ZEBRA_ERR_CUDA, std::string("in-place copy: ") + cudaGetErrorString(e));
+  return ZEBRA_OK;
 }
 
 int zebra_profile_enable(int on) {

@@ -10,8 +10,10 @@
 // One CTA = one (query tile, head): a 64-row query block against the stream of
 // 64-key blocks (kept tiles, landmark blocks, special-key blocks) described in
 // attn.cu. Warp roles:
-//   warp 0      TMA producer: Q once, then K and V of each block into a
-//               3-stage ring (128-byte swizzled 64x64 bf16 tiles);
+//   warp 0      TMA producers: lane 0 loads Q once, then the K tile of each
+//               block into a ring of STAGES 128-byte-swizzled 64x64 bf16 tiles;
+//               lane 1 loads the V tiles into their own ring, so that K runs
+//               ahead of V (QK^T of a block needs K one block before PV needs V);
 //   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
 //               score buffers (tcgen05.mma M=64 N=64, K-major A/B), then
 //               O += P V with P from shared memory (K-major) and V MN-major;
@@ -48,7 +50,14 @@ int read_and_clear_status(int* out) {
 
 namespace tc {
 
-constexpr int STAGES = 3;
+#ifndef ZEBRA_TC_STAGES
+#define ZEBRA_TC_STAGES 5
+#endif
+#ifndef ZEBRA_TC_CTAS
+#define ZEBRA_TC_CTAS 2
+#endif
+constexpr int STAGES = ZEBRA_TC_STAGES;   // depth of each of the K and V rings
+constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_S0 = 0, COL_S1 = 64, COL_O = 128;
@@ -61,8 +70,10 @@ struct __align__(1024) Smem {
   __nv_bfloat16 v[STAGES][64 * 64];
   __nv_bfloat16 p[2][64 * 64];
   uint64_t q_full;
-  uint64_t kv_full[STAGES];
-  uint64_t kv_empty[STAGES];
+  uint64_t k_full[STAGES];
+  uint64_t k_empty[STAGES];
+  uint64_t v_full[STAGES];
+  uint64_t v_empty[STAGES];
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t p_full[2];
@@ -71,9 +82,14 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort;
 };
-// keep two CTAs per SM at most: their TMEM (2 x 256 columns) fills the SM
-constexpr size_t SMEM_BYTES = 80 * 1024;
-static_assert(sizeof(Smem) + 1024 <= SMEM_BYTES, "shared memory layout");
+// Shared memory per CTA: the layout, padded so that at most CTAS_PER_SM CTAs
+// fit on an SM (their TMEM, CTAS_PER_SM x 256 columns, must fit in 512).
+constexpr size_t SMEM_NEED = sizeof(Smem) + 1024;
+constexpr size_t SMEM_CAP = 227 * 1024;
+constexpr size_t SMEM_FLOOR = SMEM_CAP / (CTAS_PER_SM + 1) + 1024;
+constexpr size_t SMEM_BYTES = SMEM_NEED > SMEM_FLOOR ? SMEM_NEED : SMEM_FLOOR;
+static_assert(SMEM_BYTES * CTAS_PER_SM <= SMEM_CAP, "shared memory layout");
+static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "TMEM columns");
 
 struct alignas(64) Params {
   CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs;
@@ -220,8 +236,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
@@ -248,30 +266,33 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
   const int n_t = ts.rows * ts.cols;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // ---------------- TMA producers: lane 0 fills the K ring, lane 1 the V ring ----------------
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      uint64_t* full = is_k ? sm.k_full : sm.v_full;
+      uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
       int issued = 0;
-      mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
-      tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+      if (is_k) {
+        mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
+        tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+      }
       BlockIter it{};
       it.bits = mask_word(mrow, 0, g.T);
       int kind, id, nv;
       while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
         const int s = issued % STAGES;
-        if (issued >= STAGES && !mbar_wait(&sm.kv_empty[s], ((issued / STAGES) - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(&sm.kv_full[s], 2 * 64 * 64 * 2);
-        const CUtensorMap* mk = kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks;
-        const CUtensorMap* mv = kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs;
-        const int row = block_row(g, h, kind, id);
-        tma_load_2d(sm.k[s], mk, 0, row, &sm.kv_full[s]);
-        tma_load_2d(sm.v[s], mv, 0, row, &sm.kv_full[s]);
+        if (issued >= STAGES && !mbar_wait(&empty[s], ((issued / STAGES) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&full[s], 64 * 64 * 2);
+        const CUtensorMap* map = is_k ? (kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks)
+                                      : (kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs);
+        tma_load_2d(is_k ? (void*)sm.k[s] : (void*)sm.v[s], map, 0, block_row(g, h, kind, id), &full[s]);
         ++issued;
       }
       if (*abort_flag) {
         // let the copies already in flight land before the CTA goes away
-        mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
+        if (is_k) mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
         for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-          mbar_wait(&sm.kv_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
+          mbar_wait(&full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
       }
     }
   } else if (warp == 1) {
@@ -283,6 +304,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       int i = 0;
       auto issue_pv = [&](int j) -> bool {
         const int b = j & 1, s = j % STAGES;
+        if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, abort_flag)) return false;
         if (!mbar_wait(&sm.p_full[b], (j >> 1) & 1, abort_flag)) return false;
         fence_after();
         const uint64_t dp = desc_k(saddr(sm.p[b]));
@@ -290,7 +312,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(tmem + COL_O, dp + 2 * kk, dv + (uint64_t)(2048 >> 4) * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.kv_empty[s]);
+        mma_commit(&sm.v_empty[s]);
         mma_commit(&sm.pv_done[b]);
         return true;
       };
@@ -300,13 +322,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
         int kind, id, nv;
         while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
           const int s = i % STAGES, b = i & 1;
-          if (!mbar_wait(&sm.kv_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&sm.k_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
           if (i >= 2 && !mbar_wait(&sm.s_free[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
           fence_after();
           const uint64_t dk = desc_k(saddr(sm.k[s]));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_f16(tmem + (b ? COL_S1 : COL_S0), dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
+          mma_commit(&sm.k_empty[s]);
           mma_commit(&sm.s_full[b]);
           if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
           ++i;

@@ -389,8 +389,5 @@ def test_hybrid_in_place():
     zb.zebra_hybrid_layer(zg, zb.ZEBRA_LAYER_LINEAR, xd, W1, W2, None, None, 0.0, out, ws)
     zb.zebra_hybrid_layer(zg, zb.ZEBRA_LAYER_LINEAR, xd, W1, W2, None, None, 0.0, xd, ws)
     torch.cuda.synchronize()
-    d = (out.float() - xd.float()).abs()
-    ulp = torch.exp2(torch.floor(torch.log2(out.float().abs().clamp_min(1e-30))) - 7)
-    print("in-place max diff", float(d.max()), "differing", int((d > 0).sum()), "of", d.numel())
-    assert bool((d <= ulp).all()), "in-place result differs by more than one bf16 ulp"
+    assert torch.equal(out, xd)
 
