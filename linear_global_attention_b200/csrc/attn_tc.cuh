@@ -9,20 +9,25 @@
 //
 // One CTA = one (query tile, head): a 64-row query block against the stream of
 // 64-key blocks (kept tiles, landmark blocks, special-key blocks) described in
-// attn.cu. Warp roles:
-//   warp 0      TMA producers: lane 0 loads Q once, then the K tile of each
-//               block into a ring of STAGES 128-byte-swizzled 64x64 bf16 tiles;
-//               lane 1 loads the V tiles into their own ring, so that K runs
-//               ahead of V (QK^T of a block needs K one block before PV needs V);
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
-//               score buffers (tcgen05.mma M=64 N=64, K-major A/B), then
-//               O += P V with P from shared memory (K-major) and V MN-major;
-//   warps 2..5  softmax warpgroup: tcgen05.ld of S (16x256b: rows spread over
-//               quads as in the m16n8 accumulator), scale + bias, running max,
-//               exp2, bf16 P into shared memory, and O rescaling in TMEM only
-//               when a row maximum grows by more than 2^8 (the stale maximum is
-//               exact as long as both the sum and O use it).
-// TMEM: S0 at column 0, S1 at 64, O at 128 (256 columns allocated); M=64
+// attn.cu. The block count is known up front (a pre-pass over the selection
+// row), so only the producer walks the stream. Warp roles:
+//   warp 0      producer: lane 0 issues TMA loads of Q once and of the K and V
+//               tile of every block into rings of STAGES 128-byte-swizzled
+//               64x64 bf16 tiles (separate K and V barriers: QK^T may start as
+//               soon as K has landed); the whole warp writes the block's 64
+//               logit biases (log2 units: 0, ln(n_u) for landmarks, -inf for
+//               masked columns) into the stage's bias row;
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of NSBUF TMEM
+//               score buffers (tcgen05.mma M=64 N=64, K-major A/B), issued up
+//               to NSBUF blocks ahead of O += P V (P from shared memory,
+//               K-major; V MN-major);
+//   warps 2..5  softmax warpgroup, straight-line per block: tcgen05.ld of S
+//               (16x256b: rows spread over quads as in the m16n8 accumulator),
+//               scale + bias, running max, exp2, bf16 P into shared memory,
+//               and O rescaling in TMEM only when a row maximum grows by more
+//               than 2^8 (the stale maximum is exact as long as both the sum
+//               and O use it).
+// TMEM: S buffers at columns 0/64/128, O at 192 (256 columns allocated); M=64
 // accumulators occupy lanes 0-15, 32-47, 64-79, 96-111, i.e. 16 rows per
 // softmax warp. Every mbarrier wait is bounded by the global timer; on expiry
 // the CTA records ZEBRA_ERR_TIMEOUT in a device status word, drains its own
@@ -56,31 +61,38 @@ namespace tc {
 #ifndef ZEBRA_TC_CTAS
 #define ZEBRA_TC_CTAS 2
 #endif
-constexpr int STAGES = ZEBRA_TC_STAGES;   // depth of each of the K and V rings
+constexpr int STAGES = ZEBRA_TC_STAGES;   // depth of the K and V rings
+constexpr int NSBUF = 3;                  // TMEM score buffers (QK^T lookahead)
 constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_S0 = 0, COL_S1 = 64, COL_O = 128;
+constexpr uint32_t COL_O = 192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
+static_assert(NSBUF <= STAGES, "QK^T lookahead needs that many K stages");
 
 struct __align__(1024) Smem {
   __nv_bfloat16 q[64 * 64];
   __nv_bfloat16 k[STAGES][64 * 64];
   __nv_bfloat16 v[STAGES][64 * 64];
   __nv_bfloat16 p[2][64 * 64];
+  float bias[STAGES][64];       // logit bias row of the block in each stage (log2 units)
+  int all_zero[STAGES];         // 1 when every bias of the stage is 0 (a complete kept tile)
   uint64_t q_full;
   uint64_t k_full[STAGES];
   uint64_t k_empty[STAGES];
   uint64_t v_full[STAGES];
   uint64_t v_empty[STAGES];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
+  uint64_t b_full[STAGES];      // bias row written
+  uint64_t s_full[NSBUF];
+  uint64_t s_free[NSBUF];
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int nblocks;
+  long long keys;               // visible keys per query row over all blocks
 };
 // Shared memory per CTA: the layout, padded so that at most CTAS_PER_SM CTAs
 // fit on an SM (their TMEM, CTAS_PER_SM x 256 columns, must fit in 512).
@@ -113,34 +125,43 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
 }
+// One test of the phase; while it is incomplete the thread sleeps in hardware
+// (up to SUSPEND_NS) and wakes when the phase completes, so waiting warps do
+// not take issue slots from the softmax warps.
+constexpr uint32_t SUSPEND_NS = 100000;
 __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity)
+      : "r"(saddr(b)), "r"(parity), "r"(SUSPEND_NS)
       : "memory");
   return ok != 0;
 }
 
-// Wait for the phase of `parity` to complete. Gives up after `limit_ns`, or
-// early once another warp has raised the abort flag; a timeout records the
-// error status and raises the flag. Returns true when the phase completed.
-__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                       unsigned long long limit_ns = WAIT_NS) {
-  if (mbar_try(b, parity)) return true;
+// Slow path of mbar_wait: keep testing until the phase completes, another warp
+// raises the abort flag, or `limit_ns` passes (then record the error status
+// and raise the flag).
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                            unsigned long long limit_ns) {
   const unsigned long long t0 = gtime();
-  for (uint32_t i = 1;; ++i) {
+  while (true) {
     if (mbar_try(b, parity)) return true;
-    if ((i & 255) == 0) {
-      if (*abort_flag) return false;
-      if (gtime() - t0 > limit_ns) {
-        atomicExch(&g_status, ZEBRA_ERR_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
+    if (*abort_flag) return false;
+    if (gtime() - t0 > limit_ns) {
+      atomicExch(&g_status, ZEBRA_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
     }
   }
+}
+
+// Wait for the phase of `parity` to complete; true when it did.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = WAIT_NS) {
+  if (mbar_try(b, parity)) return true;
+  return mbar_wait_slow(b, parity, abort_flag, limit_ns);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -240,10 +261,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.b_full[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NSBUF; ++b) {
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.s_free[b], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.p_full[b], 4);
       mbar_init(&sm.pv_done[b], 1);
     }
@@ -251,7 +275,21 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 0) {
+    // pre-pass: number of blocks and visible keys per query row
+    BlockIter it{};
+    it.bits = mask_word(mrow, 0, g.T);
+    int kind, id, nv, n = 0;
+    long long keys = 0;
+    while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+      ++n;
+      keys += nv;
+    }
+    if (lane == 0) {
+      sm.nblocks = n;
+      sm.keys = keys;
+    }
+  } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sm.tmem_base)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -260,39 +298,67 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
   __syncthreads();
   fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const int nb = sm.nblocks;
 
   const bool own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
   const TileShape ts = tile_shape(g, t);
   const int n_t = ts.rows * ts.cols;
 
   if (warp == 0) {
-    // ---------------- TMA producers: lane 0 fills the K ring, lane 1 the V ring ----------------
-    if (lane < 2) {
-      const bool is_k = lane == 0;
-      uint64_t* full = is_k ? sm.k_full : sm.v_full;
-      uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
-      int issued = 0;
-      if (is_k) {
-        mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
-        tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+    // ---------------- producer ----------------
+    int issued = 0;
+    if (lane == 0) {
+      mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
+      tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+    }
+    BlockIter it{};
+    it.bits = mask_word(mrow, 0, g.T);
+    int kind, id, nv;
+    bool ok = true;
+    while (ok && next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+      const int s = issued % STAGES;
+      const uint32_t par = ((issued / STAGES) - 1) & 1;
+      const int row = block_row(g, h, kind, id);
+      if (lane == 0) {
+        if (issued >= STAGES && !mbar_wait(&sm.k_empty[s], par, abort_flag)) ok = false;
+        if (ok) {
+          mbar_expect_tx(&sm.k_full[s], 64 * 64 * 2);
+          tma_load_2d(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
+        }
+        // the V tile and the bias row of this stage are free once PV of block issued - STAGES is done
+        if (ok && issued >= STAGES && !mbar_wait(&sm.v_empty[s], par, abort_flag)) ok = false;
+        if (ok) {
+          mbar_expect_tx(&sm.v_full[s], 64 * 64 * 2);
+          tma_load_2d(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
+        }
       }
-      BlockIter it{};
-      it.bits = mask_word(mrow, 0, g.T);
-      int kind, id, nv;
-      while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
-        const int s = issued % STAGES;
-        if (issued >= STAGES && !mbar_wait(&empty[s], ((issued / STAGES) - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(&full[s], 64 * 64 * 2);
-        const CUtensorMap* map = is_k ? (kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks)
-                                      : (kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs);
-        tma_load_2d(is_k ? (void*)sm.k[s] : (void*)sm.v[s], map, 0, block_row(g, h, kind, id), &full[s]);
-        ++issued;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      // bias row: two columns per lane
+      float b0, b1;
+      if (kind == 1) {
+        b0 = block_bias(a, mrow, t, kind, id, 2 * lane);
+        b1 = block_bias(a, mrow, t, kind, id, 2 * lane + 1);
+      } else {
+        b0 = 2 * lane < nv ? 0.f : -INFINITY;
+        b1 = 2 * lane + 1 < nv ? 0.f : -INFINITY;
       }
-      if (*abort_flag) {
-        // let the copies already in flight land before the CTA goes away
-        if (is_k) mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
-        for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-          mbar_wait(&full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
+      *reinterpret_cast<float2*>(&sm.bias[s][2 * lane]) = make_float2(b0, b1);
+      const int zero = __all_sync(0xffffffffu, b0 == 0.f && b1 == 0.f);
+      __threadfence_block();   // every lane's row entries precede lane 0's release below
+      __syncwarp();
+      if (lane == 0) {
+        sm.all_zero[s] = zero;
+        mbar_arrive(&sm.b_full[s]);
+      }
+      ++issued;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let the copies already in flight land before the CTA goes away
+      mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
+      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i) {
+        mbar_wait(&sm.k_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
+        mbar_wait(&sm.v_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
       }
     }
   } else if (warp == 1) {
@@ -301,40 +367,35 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       const uint32_t id_qk = idesc(false), id_pv = idesc(true);
       const uint64_t dq = desc_k(saddr(sm.q));
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
-      int i = 0;
-      auto issue_pv = [&](int j) -> bool {
-        const int b = j & 1, s = j % STAGES;
-        if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(&sm.p_full[b], (j >> 1) & 1, abort_flag)) return false;
+      int qk = 0;
+      for (int j = 0; ok && j < nb; ++j) {
+        // S = Q K^T for up to NSBUF blocks ahead of this PV
+        while (ok && qk < nb && qk < j + NSBUF) {
+          const int s = qk % STAGES, b = qk % NSBUF;
+          if (!mbar_wait(&sm.k_full[s], (qk / STAGES) & 1, abort_flag)) { ok = false; break; }
+          if (qk >= NSBUF && !mbar_wait(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag)) { ok = false; break; }
+          fence_after();
+          const uint64_t dk = desc_k(saddr(sm.k[s]));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + 64u * b, dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
+          mma_commit(&sm.k_empty[s]);
+          mma_commit(&sm.s_full[b]);
+          ++qk;
+        }
+        if (!ok) break;
+        // O += P V of block j
+        const int s = j % STAGES, pb = j & 1;
+        if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&sm.p_full[pb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
         fence_after();
-        const uint64_t dp = desc_k(saddr(sm.p[b]));
+        const uint64_t dp = desc_k(saddr(sm.p[pb]));
         const uint64_t dv = desc_mn(saddr(sm.v[s]));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(tmem + COL_O, dp + 2 * kk, dv + (uint64_t)(2048 >> 4) * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.v_empty[s]);
-        mma_commit(&sm.pv_done[b]);
-        return true;
-      };
-      if (ok) {
-        BlockIter it{};
-        it.bits = mask_word(mrow, 0, g.T);
-        int kind, id, nv;
-        while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
-          const int s = i % STAGES, b = i & 1;
-          if (!mbar_wait(&sm.k_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&sm.s_free[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-          fence_after();
-          const uint64_t dk = desc_k(saddr(sm.k[s]));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + (b ? COL_S1 : COL_S0), dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
-          mma_commit(&sm.k_empty[s]);
-          mma_commit(&sm.s_full[b]);
-          if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
-          ++i;
-        }
-        if (ok && i >= 1) issue_pv(i - 1);
+        mma_commit(&sm.pv_done[pb]);
       }
       // drain: every MMA this thread issued completes before TMEM is freed
       mma_commit(&sm.drain);
@@ -349,43 +410,43 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
     const float NEG = -INFINITY;
     float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
     const int r0 = 16 * rb + g4, r1 = r0 + 8;  // query rows of this thread
-    unsigned char* pbase[2] = {reinterpret_cast<unsigned char*>(sm.p[0]), reinterpret_cast<unsigned char*>(sm.p[1])};
-    BlockIter it{};
-    it.bits = mask_word(mrow, 0, g.T);
-    int kind, id, nv;
-    int i = 0;
     bool ok = true;
-    long long keys = 0;
-    while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
-      keys += nv;
-      const int b = i & 1;
-      if (!mbar_wait(&sm.s_full[b], (i >> 1) & 1, abort_flag)) { ok = false; break; }
+    for (int i = 0; i < nb; ++i) {
+      const int s = i % STAGES, b = i % NSBUF, pb = i & 1;
+      if (!mbar_wait(&sm.s_full[b], (i / NSBUF) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&sm.b_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
       fence_after();
-      float s[32];
-      tmem_ld64(tmem + lane_off + (b ? COL_S1 : COL_S0), s);
+      float sv[32];
+      tmem_ld64(tmem + lane_off + 64u * b, sv);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[b]);
 
       // scale, bias (log2 units) and row maxima
       float mx0 = NEG, mx1 = NEG;
-      const bool full_tile = kind == 0 && nv == 64;
+      if (sm.all_zero[s]) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 8; ++j) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 8 * j + 2 * q4 + e;
-          float bias = 0.f;
-          if (!full_tile) bias = kind == 1 ? block_bias(a, mrow, t, kind, id, col) : (col < nv ? 0.f : NEG);
-          s[4 * j + e] = fmaf(s[4 * j + e], sc, bias);
-          s[4 * j + 2 + e] = fmaf(s[4 * j + 2 + e], sc, bias);
-          mx0 = fmaxf(mx0, s[4 * j + e]);
-          mx1 = fmaxf(mx1, s[4 * j + 2 + e]);
+          for (int e = 0; e < 4; ++e) sv[4 * j + e] *= sc;
+          mx0 = fmaxf(mx0, fmaxf(sv[4 * j], sv[4 * j + 1]));
+          mx1 = fmaxf(mx1, fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 bb = *reinterpret_cast<const float2*>(&sm.bias[s][8 * j + 2 * q4]);
+          sv[4 * j + 0] = fmaf(sv[4 * j + 0], sc, bb.x);
+          sv[4 * j + 1] = fmaf(sv[4 * j + 1], sc, bb.y);
+          sv[4 * j + 2] = fmaf(sv[4 * j + 2], sc, bb.x);
+          sv[4 * j + 3] = fmaf(sv[4 * j + 3], sc, bb.y);
+          mx0 = fmaxf(mx0, fmaxf(sv[4 * j], sv[4 * j + 1]));
+          mx1 = fmaxf(mx1, fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
         }
       }
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
       // lazy maximum: move it only when the block exceeds it by more than 8 (x256)
       const bool up0 = mx0 > m0 + 8.f, up1 = mx1 > m1 + 8.f;
@@ -396,27 +457,27 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       uint32_t pk[8][2];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        s[4 * j + 0] = fast_exp2(s[4 * j + 0] - base0);
-        s[4 * j + 1] = fast_exp2(s[4 * j + 1] - base0);
-        s[4 * j + 2] = fast_exp2(s[4 * j + 2] - base1);
-        s[4 * j + 3] = fast_exp2(s[4 * j + 3] - base1);
-        pk[j][0] = pack_round(s[4 * j + 0], s[4 * j + 1]);
-        pk[j][1] = pack_round(s[4 * j + 2], s[4 * j + 3]);
-        rs0 += s[4 * j + 0] + s[4 * j + 1];
-        rs1 += s[4 * j + 2] + s[4 * j + 3];
+        sv[4 * j + 0] = fast_exp2(sv[4 * j + 0] - base0);
+        sv[4 * j + 1] = fast_exp2(sv[4 * j + 1] - base0);
+        sv[4 * j + 2] = fast_exp2(sv[4 * j + 2] - base1);
+        sv[4 * j + 3] = fast_exp2(sv[4 * j + 3] - base1);
+        pk[j][0] = pack_round(sv[4 * j + 0], sv[4 * j + 1]);
+        pk[j][1] = pack_round(sv[4 * j + 2], sv[4 * j + 3]);
+        rs0 += sv[4 * j + 0] + sv[4 * j + 1];
+        rs1 += sv[4 * j + 2] + sv[4 * j + 3];
       }
       l0 = l0 * al0 + rs0;
       l1 = l1 * al1 + rs1;
       m0 = mn0;
       m1 = mn1;
-      // P buffer b is free once PV of block i-2 has completed
-      if (i >= 2 && !mbar_wait(&sm.pv_done[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      // P buffer pb is free once PV of block i-2 has completed
+      if (i >= 2 && !mbar_wait(&sm.pv_done[pb], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      unsigned char* pbuf = reinterpret_cast<unsigned char*>(sm.p[pb]);
+      const uint32_t x0 = (uint32_t)(r0 & 7), x1 = (uint32_t)(r1 & 7);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint32_t cb = (uint32_t)(((j ^ (r0 & 7)) << 4) + 4 * q4);
-        *reinterpret_cast<uint32_t*>(pbase[b] + r0 * 128 + cb) = pk[j][0];
-        const uint32_t cb1 = (uint32_t)(((j ^ (r1 & 7)) << 4) + 4 * q4);
-        *reinterpret_cast<uint32_t*>(pbase[b] + r1 * 128 + cb1) = pk[j][1];
+        *reinterpret_cast<uint32_t*>(pbuf + r0 * 128 + (((uint32_t)j ^ x0) << 4) + 4 * q4) = pk[j][0];
+        *reinterpret_cast<uint32_t*>(pbuf + r1 * 128 + (((uint32_t)j ^ x1) << 4) + 4 * q4) = pk[j][1];
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       // rescale O (TMEM) when any row of this warp moved its maximum
@@ -437,10 +498,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[b]);
-      ++i;
+      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
-    const int nb = i;
     // ---------------- epilogue ----------------
     if (ok && nb >= 1 && !mbar_wait(&sm.pv_done[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag)) ok = false;
     if (ok) {
@@ -523,7 +582,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       }
       if (tid == 64) {
         const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);
-        atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (keys + extra)));
+        atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (sm.keys + extra)));
       }
     }
   }
