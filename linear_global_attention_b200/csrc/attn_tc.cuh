@@ -27,7 +27,7 @@
 //               and O rescaling in TMEM only when a row maximum grows by more
 //               than 2^8 (the stale maximum is exact as long as both the sum
 //               and O use it).
-// TMEM: S buffers at columns 0/64/128, O at 192 (256 columns allocated); M=64
+// TMEM: NSBUF score buffers of 64 columns, then O (128 or 256 columns); M=64
 // accumulators occupy lanes 0-15, 32-47, 64-79, 96-111, i.e. 16 rows per
 // softmax warp. Every mbarrier wait is bounded by the global timer; on expiry
 // the CTA records ZEBRA_ERR_TIMEOUT in a device status word, drains its own
@@ -56,26 +56,33 @@ int read_and_clear_status(int* out) {
 namespace tc {
 
 #ifndef ZEBRA_TC_STAGES
-#define ZEBRA_TC_STAGES 5
+#define ZEBRA_TC_STAGES 2
 #endif
 #ifndef ZEBRA_TC_CTAS
-#define ZEBRA_TC_CTAS 2
+#define ZEBRA_TC_CTAS 4
 #endif
 constexpr int STAGES = ZEBRA_TC_STAGES;   // depth of the K and V rings
-constexpr int NSBUF = 3;                  // TMEM score buffers (QK^T lookahead)
+#ifndef ZEBRA_TC_NSBUF
+#define ZEBRA_TC_NSBUF 1
+#endif
+constexpr int NSBUF = ZEBRA_TC_NSBUF;     // TMEM score buffers (QK^T lookahead)
+#ifndef ZEBRA_TC_PBUF
+#define ZEBRA_TC_PBUF 1
+#endif
+constexpr int PBUF = ZEBRA_TC_PBUF;       // shared-memory P buffers (softmax lead over PV)
 constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_O = 192;
+constexpr uint32_t COL_O = 64 * NSBUF;   // O after the score buffers
+constexpr uint32_t TMEM_COLS = COL_O + 64 <= 128 ? 128 : 256;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
-static_assert(NSBUF <= STAGES, "QK^T lookahead needs that many K stages");
+static_assert(NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
 
 struct __align__(1024) Smem {
   __nv_bfloat16 q[64 * 64];
   __nv_bfloat16 k[STAGES][64 * 64];
   __nv_bfloat16 v[STAGES][64 * 64];
-  __nv_bfloat16 p[2][64 * 64];
+  __nv_bfloat16 p[PBUF][64 * 64];
   float bias[STAGES][64];       // logit bias row of the block in each stage (log2 units)
   int all_zero[STAGES];         // 1 when every bias of the stage is 0 (a complete kept tile)
   uint64_t q_full;
@@ -86,8 +93,8 @@ struct __align__(1024) Smem {
   uint64_t b_full[STAGES];      // bias row written
   uint64_t s_full[NSBUF];
   uint64_t s_free[NSBUF];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t p_full[PBUF];
+  uint64_t pv_done[PBUF];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -95,7 +102,7 @@ struct __align__(1024) Smem {
   long long keys;               // visible keys per query row over all blocks
 };
 // Shared memory per CTA: the layout, padded so that at most CTAS_PER_SM CTAs
-// fit on an SM (their TMEM, CTAS_PER_SM x 256 columns, must fit in 512).
+// fit on an SM (their TMEM, CTAS_PER_SM x TMEM_COLS columns, must fit in 512).
 constexpr size_t SMEM_NEED = sizeof(Smem) + 1024;
 constexpr size_t SMEM_CAP = 227 * 1024;
 constexpr size_t SMEM_FLOOR = SMEM_CAP / (CTAS_PER_SM + 1) + 1024;
@@ -131,12 +138,21 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
 constexpr uint32_t SUSPEND_NS = 100000;
 __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
+#ifdef ZEBRA_TC_WAIT_SPIN
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+#else
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(saddr(b)), "r"(parity), "r"(SUSPEND_NS)
       : "memory");
+#endif
   return ok != 0;
 }
 
@@ -244,7 +260,7 @@ __device__ __forceinline__ int block_row(const Geo& g, int h, int kind, int id) 
   return h * g.NSp + id * 64;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const AttnArgs& a = P.a;
@@ -264,10 +280,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       mbar_init(&sm.b_full[s], 1);
     }
     for (int b = 0; b < NSBUF; ++b) {
-      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_full[b], 2);   // MMA completion + the MMA thread's release after the bias row
       mbar_init(&sm.s_free[b], 4);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < PBUF; ++b) {
       mbar_init(&sm.p_full[b], 4);
       mbar_init(&sm.pv_done[b], 1);
     }
@@ -369,8 +385,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
       int qk = 0;
       for (int j = 0; ok && j < nb; ++j) {
-        // S = Q K^T for up to NSBUF blocks ahead of this PV
-        while (ok && qk < nb && qk < j + NSBUF) {
+        // S = Q K^T up to NSBUF blocks ahead of this PV (a score buffer is
+        // reusable as soon as the softmax has loaded it)
+        while (ok && qk < nb && qk <= j + NSBUF) {
           const int s = qk % STAGES, b = qk % NSBUF;
           if (!mbar_wait(&sm.k_full[s], (qk / STAGES) & 1, abort_flag)) { ok = false; break; }
           if (qk >= NSBUF && !mbar_wait(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag)) { ok = false; break; }
@@ -381,13 +398,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
             mma_f16(tmem + 64u * b, dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
           mma_commit(&sm.k_empty[s]);
           mma_commit(&sm.s_full[b]);
+          // forward the stage's bias row to the softmax through s_full: this
+          // thread acquires it here and releases it with its own arrival
+          if (!mbar_wait(&sm.b_full[s], (qk / STAGES) & 1, abort_flag)) { ok = false; break; }
+          mbar_arrive(&sm.s_full[b]);
           ++qk;
         }
         if (!ok) break;
         // O += P V of block j
-        const int s = j % STAGES, pb = j & 1;
+        const int s = j % STAGES, pb = j % PBUF;
         if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&sm.p_full[pb], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&sm.p_full[pb], (j / PBUF) & 1, abort_flag)) { ok = false; break; }
         fence_after();
         const uint64_t dp = desc_k(saddr(sm.p[pb]));
         const uint64_t dv = desc_mn(saddr(sm.v[s]));
@@ -412,9 +433,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
     const int r0 = 16 * rb + g4, r1 = r0 + 8;  // query rows of this thread
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
-      const int s = i % STAGES, b = i % NSBUF, pb = i & 1;
+      const int s = i % STAGES, b = i % NSBUF, pb = i % PBUF;
       if (!mbar_wait(&sm.s_full[b], (i / NSBUF) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&sm.b_full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
       fence_after();
       float sv[32];
       tmem_ld64(tmem + lane_off + 64u * b, sv);
@@ -424,14 +444,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
 
       // scale, bias (log2 units) and row maxima
       float mx0 = NEG, mx1 = NEG;
-      if (sm.all_zero[s]) {
+      const bool nobias = sm.all_zero[s] != 0;
+      if (nobias) {
+        // complete kept tile: maxima of the raw scores (the scale is positive)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sv[4 * j + e] *= sc;
           mx0 = fmaxf(mx0, fmaxf(sv[4 * j], sv[4 * j + 1]));
           mx1 = fmaxf(mx1, fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
         }
+        mx0 *= sc;
+        mx1 *= sc;
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -455,12 +477,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       const float al0 = up0 ? fast_exp2(m0 - base0) : 1.f, al1 = up1 ? fast_exp2(m1 - base1) : 1.f;
       float rs0 = 0.f, rs1 = 0.f;
       uint32_t pk[8][2];
+      // p = 2^(scaled score - base): one FFMA per element for complete tiles
+      const float ka = nobias ? sc : 1.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        sv[4 * j + 0] = fast_exp2(sv[4 * j + 0] - base0);
-        sv[4 * j + 1] = fast_exp2(sv[4 * j + 1] - base0);
-        sv[4 * j + 2] = fast_exp2(sv[4 * j + 2] - base1);
-        sv[4 * j + 3] = fast_exp2(sv[4 * j + 3] - base1);
+        sv[4 * j + 0] = fast_exp2(fmaf(sv[4 * j + 0], ka, -base0));
+        sv[4 * j + 1] = fast_exp2(fmaf(sv[4 * j + 1], ka, -base0));
+        sv[4 * j + 2] = fast_exp2(fmaf(sv[4 * j + 2], ka, -base1));
+        sv[4 * j + 3] = fast_exp2(fmaf(sv[4 * j + 3], ka, -base1));
         pk[j][0] = pack_round(sv[4 * j + 0], sv[4 * j + 1]);
         pk[j][1] = pack_round(sv[4 * j + 2], sv[4 * j + 3]);
         rs0 += sv[4 * j + 0] + sv[4 * j + 1];
@@ -470,8 +494,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       l1 = l1 * al1 + rs1;
       m0 = mn0;
       m1 = mn1;
-      // P buffer pb is free once PV of block i-2 has completed
-      if (i >= 2 && !mbar_wait(&sm.pv_done[pb], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      // P buffer pb is free once PV of block i-PBUF has completed
+      if (i >= PBUF && !mbar_wait(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
       unsigned char* pbuf = reinterpret_cast<unsigned char*>(sm.p[pb]);
       const uint32_t x0 = (uint32_t)(r0 & 7), x1 = (uint32_t)(r1 & 7);
 #pragma unroll
@@ -483,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       // rescale O (TMEM) when any row of this warp moved its maximum
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
-        if (!mbar_wait(&sm.pv_done[jp & 1], (jp >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag)) { ok = false; break; }
         fence_after();
         float o[32];
         tmem_ld64(tmem + lane_off + COL_O, o);
@@ -501,7 +525,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(const __grid_consta
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
     // ---------------- epilogue ----------------
-    if (ok && nb >= 1 && !mbar_wait(&sm.pv_done[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag)) ok = false;
+    if (ok && nb >= 1 && !mbar_wait(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag)) ok = false;
     if (ok) {
       fence_after();
       float o[32];
