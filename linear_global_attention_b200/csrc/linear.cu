@@ -143,13 +143,15 @@ __device__ __forceinline__ void store_row_half_bf16(unsigned char* tile, int row
 // --------------------------------------------------------------------------
 // 1. state (bf16)
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) linear_state_kernel(const __grid_constant__ LinearArgs a) {
+__global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_constant__ LinearArgs a) {
   __shared__ __align__(128) unsigned char phi_s[64 * 128];
-  __shared__ __align__(128) unsigned char v_s[64 * 128];
+  __shared__ __align__(128) unsigned char v_s[2][64 * 128];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const long long n0 = (long long)blockIdx.x * a.chunk_tokens;
+  // grid (head, chunk): the CTAs resident together cover all heads of the same
+  // tokens, so their 128-byte head slices of each token row are fetched together
+  const int h = blockIdx.x;
+  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
   const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v);
@@ -161,24 +163,50 @@ __global__ void __launch_bounds__(128) linear_state_kernel(const __grid_constant
   const int g4 = lane >> 2;
   const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
 
+  // K of this thread's token half: registers, one 64-token block ahead
+  auto fetch_k = [&](long long nb, uint4* kd) {
+    const long long n = nb + tok;
+    if (n < n1) {
+      const uint4* kp = reinterpret_cast<const uint4*>(K + n * a.ts + (long long)h * a.hs + half * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) kd[q] = __ldg(kp + q);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) kd[q] = make_uint4(0, 0, 0, 0);
+    }
+  };
+  // V of this thread's token half: straight into a swizzled shared tile (zeros past the chunk)
+  auto fetch_v = [&](long long nb, int buf) {
+    const long long n = nb + tok;
+    const bool ok = n < n1;
+    const __nv_bfloat16* vp = Vt + (ok ? n : n0) * a.ts + (long long)h * a.hs + half * 32;
+    const uint32_t dst = lsmem(v_s[buf]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst + lswz(tok, half * 4 + q)),
+                   "l"(vp + 8 * q), "r"(ok ? 16 : 0));
+    asm volatile("cp.async.commit_group;\n" ::);
+  };
+  uint4 kr[4];
+  fetch_k(n0, kr);
+  fetch_v(n0, 0);
+  int buf = 0;
   for (long long nb = n0; nb < n1; nb += 64) {
     const long long n = nb + tok;
     const bool valid = n < n1;
+    uint4 kn[4];
+    fetch_k(nb + 64, kn);
     float x[32];
-    uint4 vraw[4];
-    if (valid) {
-      const __nv_bfloat16* kp = K + n * a.ts + (long long)h * a.hs + half * 32;
-      const __nv_bfloat16* vp = Vt + n * a.ts + (long long)h * a.hs + half * 32;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        load16(kp + 8 * q, x + 8 * q);
-        vraw[q] = *reinterpret_cast<const uint4*>(vp + 8 * q);
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&kr[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hv[e]);
+        x[8 * q + 2 * e] = f.x;
+        x[8 * q + 2 * e + 1] = f.y;
       }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) vraw[q] = make_uint4(0, 0, 0, 0);
+      kr[q] = kn[q];
     }
     {
       // every lane runs the prologue (it shuffles with lane ^ 1); padding tokens are zeroed after
@@ -191,11 +219,13 @@ __global__ void __launch_bounds__(128) linear_state_kernel(const __grid_constant
         for (int c = 0; c < 32; ++c) x[c] = 0.f;
       }
     }
-    __syncthreads();  // previous MMA reads of phi_s / v_s are done
+    __syncthreads();  // the previous MMA has finished reading phi_s and v_s[buf ^ 1]
+    if (nb + 64 < n1) fetch_v(nb + 64, buf ^ 1);
+    else asm volatile("cp.async.commit_group;\n" ::);
     store_row_half_bf16(phi_s, tok, half, x);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(v_s + lswz(tok, half * 4 + q)) = vraw[q];
+    asm volatile("cp.async.wait_group 1;\n" ::);   // this block's V has landed
     __syncthreads();
+    const uint32_t vb = lsmem(v_s[buf]);
     // [S | z] (rows = channels 16*warp..) += phi^T [V | 1]
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {  // 16 tokens per k-step
@@ -212,15 +242,17 @@ __global__ void __launch_bounds__(128) linear_state_kernel(const __grid_constant
         const int mi = lane >> 3, ri = lane & 7;
         const int trow = ks * 16 + (mi & 1) * 8 + ri;
         uint32_t b0, b1, b2, b3;
-        l_ldsm_x4_t(lsmem(v_s) + lswz(trow, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
+        l_ldsm_x4_t(vb + lswz(trow, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
         l_mma(acc[2 * dp], af, b0, b1);
         l_mma(acc[2 * dp + 1], af, b2, b3);
       }
       l_mma(acc[8], af, ones, ones);
     }
+    buf ^= 1;
   }
+  asm volatile("cp.async.wait_group 0;\n" ::);
   // write partial [64][65]: row = channel, col = 0..63 (S), 64 (z)
-  float* part = a.part + ((size_t)blockIdx.x * g.H + h) * 64 * 65;
+  float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
   const int q4 = lane & 3;
 #pragma unroll
   for (int j = 0; j < 9; ++j) {
@@ -321,13 +353,13 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constan
 // --------------------------------------------------------------------------
 // 3. apply (bf16): CTA = 128 threads, 64 tokens per step, state B operand in smem
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) linear_apply_kernel(const __grid_constant__ LinearArgs a) {
+__global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_constant__ LinearArgs a) {
   __shared__ __align__(128) unsigned char phi_s[64 * 128];
   __shared__ __align__(128) unsigned char b_s[NB * 128];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const long long n0 = (long long)blockIdx.x * a.chunk_tokens;
+  const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
+  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
@@ -344,17 +376,36 @@ __global__ void __launch_bounds__(128) linear_apply_kernel(const __grid_constant
     bias[2 * j + 1] = a.b ? a.b[h * 64 + 8 * j + 2 * q4 + 1] : 0.f;
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+  // raw Q of this thread's token half, loaded one 64-token block ahead
+  uint4 qr[4];
+  auto fetch = [&](long long nb, uint4* qd) {
+    const long long n = nb + tok;
+    if (n < n1) {
+      const uint4* qp = reinterpret_cast<const uint4*>(Q + n * a.ts + (long long)h * a.hs + half * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) qd[q] = __ldg(qp + q);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) qd[q] = make_uint4(0, 0, 0, 0);
+    }
+  };
+  fetch(n0, qr);
   for (long long nb = n0; nb < n1; nb += 64) {
     const long long n = nb + tok;
     const bool valid = n < n1;
+    uint4 qn[4];
+    fetch(nb + 64, qn);
     float x[32];
-    if (valid) {
-      const __nv_bfloat16* qp = Q + n * a.ts + (long long)h * a.hs + half * 32;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) load16(qp + 8 * q, x + 8 * q);
-    } else {
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&qr[q]);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = 0.f;
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hv[e]);
+        x[8 * q + 2 * e] = f.x;
+        x[8 * q + 2 * e + 1] = f.y;
+      }
+      qr[q] = qn[q];
     }
     {
       bool sp;
@@ -461,7 +512,7 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
   {
     ProfScope prof("linear_state", st);
-    linear_state_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+    linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
   }
   count_launch();
   if (int rc = check_launch("linear_state_kernel")) return rc;
@@ -473,7 +524,7 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
   {
     ProfScope prof("linear_apply", st);
-    linear_apply_kernel<<<dim3(a.chunks, a.g.H), 128, 0, st>>>(a);
+    linear_apply_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
   }
   count_launch();
   return check_launch("linear_apply_kernel");
