@@ -163,6 +163,26 @@ ZEBRA_API int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void*
                       const zebra_layout* layout, const float* A, const float* b, float rope_base,
                       float eps, void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* The linear stage of zebra_linear_attn (same arguments, same result) for
+ * callers that cannot allocate device memory: code whose device memory is
+ * owned by another framework's allocator or a fixed reservation (so a
+ * cudaMalloc of a workspace would fail or fragment it), latency-critical paths
+ * that must not risk an allocation stalling the device, and thin C or FFI
+ * clients with no allocator at hand. The paper has no counterpart of this
+ * entry point; it only changes where the scratch memory comes from.
+ * Scratch: a built-in device array of 16 MiB (every GPU that loads the
+ * library holds it until the process exits); no cudaMalloc, cudaFree or
+ * allocating library routine is called. Geometries whose per-head state and
+ * per-chunk partials do not fit in it return ZEBRA_ERR_UNSUPPORTED (at 16
+ * heads any token count fits). The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) and caches it; make that first call
+ * before any stream capture. Every call uses the same array, so calls that
+ * overlap on the GPU (e.g. on two streams) race; serialise them. Nothing in
+ * the array has to start at zero: each call overwrites what it reads. */
+ZEBRA_API int zebra_linear_attn_noalloc(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k,
+                                        const void* v, const zebra_layout* layout, const float* A, const float* b,
+                                        float rope_base, float eps, void* out, void* stream);
+
 /* One stacked global-attention layer, bf16 only (section "Linear-centered
  * stages plus tile-sparse stages": preserved QKV/output projections,
  * normalisation and positional encoding):

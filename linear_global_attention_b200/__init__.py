@@ -16,7 +16,7 @@ __all__ = [
     "zebra_keep_count", "zebra_tile_pool", "zebra_tile_select", "zebra_sparse_attn",
     "zebra_linear_attn", "zebra_hybrid_layer", "zebra_workspace_bytes", "zebra_last_error",
     "zebra_sync_status", "zebra_launch_count", "zebra_version", "workspace", "zebra_profile_enable",
-    "zebra_profile_report",
+    "zebra_profile_report", "zebra_linear_attn_noalloc",
     "ZEBRA_OK", "ZEBRA_ERR_INVALID_ARG", "ZEBRA_ERR_UNSUPPORTED", "ZEBRA_ERR_WORKSPACE", "ZEBRA_ERR_CUDA",
     "ZEBRA_ERR_TIMEOUT", "ZEBRA_F32", "ZEBRA_BF16", "ZEBRA_LAYER_LINEAR", "ZEBRA_LAYER_SPARSE",
     "ZEBRA_LAYER_DENSE", "ZEBRA_OP_SELECT", "ZEBRA_OP_SPARSE", "ZEBRA_OP_LINEAR", "ZEBRA_OP_HYBRID_LINEAR",
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
             "zebra_sync_status": (ctypes.c_int, [_P]),
             "zebra_launch_count": (ctypes.c_uint64, []),
             "zebra_version": (ctypes.c_char_p, []),
+            "zebra_linear_attn_noalloc": (ctypes.c_int, [_G, ctypes.c_int, _P, _P, _P, _L, _P, _P, ctypes.c_float,
+                                                         ctypes.c_float, _P, _P]),
             "zebra_profile_enable": (ctypes.c_int, [ctypes.c_int]),
             "zebra_profile_report": (ctypes.c_longlong, [ctypes.c_char_p, ctypes.c_size_t]),
         }
@@ -202,6 +204,13 @@ def zebra_linear_attn(g: Geom, q, k, v, A, b, out, ws, rope_base=100.0, eps=1e-6
     _check(lib().zebra_linear_attn(ctypes.byref(g), _dtype(q), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay),
                                    _ptr(A), _ptr(b), rope_base, eps, _ptr(out), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def zebra_linear_attn_noalloc(g: Geom, q, k, v, A, b, out, rope_base=100.0, eps=1e-6, stream=None):
+    """zebra_linear_attn with its scratch in the library's built-in device array (no workspace)."""
+    lay = _layout(q, k, v)
+    _check(lib().zebra_linear_attn_noalloc(ctypes.byref(g), _dtype(q), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay),
+                                           _ptr(A), _ptr(b), rope_base, eps, _ptr(out), _stream(stream)))
 
 
 def zebra_hybrid_layer(g: Geom, kind: int, x, w_qkv, w_o, A, b, y, x_out, ws, rope_base=100.0, eps=1e-6,
