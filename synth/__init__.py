@@ -82,11 +82,31 @@ WORKLOADS = {
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bfloat16 (ties to even); returns float32."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    """Round float32 values to the nearest bfloat16 (ties to even); returns a new float32 array.
+
+    uint32 arithmetic, exact for every finite input (the rounding increment
+    cannot carry past the exponent of a finite float); large arrays are
+    processed in threaded chunks.
+    """
+    out = np.array(x, dtype=np.float32, copy=True, order="C")
+    u = out.reshape(-1).view(np.uint32)
+    step = 1 << 24
+
+    def work(lo):
+        seg = u[lo:lo + step]
+        inc = (seg >> 16) & 1
+        inc += 0x7FFF
+        seg += inc
+        seg &= 0xFFFF0000
+
+    starts = range(0, u.size, step)
+    if u.size > step:
+        with _cf.ThreadPoolExecutor(min(_threads(), len(starts))) as ex:
+            list(ex.map(work, starts))
+    else:
+        for lo in starts:
+            work(lo)
+    return out
 
 
 def _rng(*key: int) -> np.random.Generator:
