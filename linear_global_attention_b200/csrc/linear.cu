@@ -143,9 +143,49 @@ __device__ __forceinline__ void store_row_half_bf16(unsigned char* tile, int row
 // --------------------------------------------------------------------------
 // 1. state (bf16)
 // --------------------------------------------------------------------------
+// Raw bf16 rows of a 64-token block, one 128-byte head slice per token, land in
+// a 3-deep ring of swizzled shared tiles through cp.async, two blocks ahead of
+// the block being computed (padding tokens are zero-filled).
+constexpr int LSTAGES = 3;
+
+__device__ __forceinline__ void fetch_rows(uint32_t tile, const __nv_bfloat16* base, long long nb, long long n1,
+                                           long long ts, int tok, int half) {
+  const long long n = nb + tok;
+  const bool ok = n < n1;
+  const __nv_bfloat16* p = base + (ok ? n : 0) * ts + half * 32;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, half * 4 + q)),
+                 "l"(p + 8 * q), "r"(ok ? 16 : 0));
+}
+
+// this thread's 32 channels of its token, from a swizzled raw tile
+__device__ __forceinline__ void read_half(const unsigned char* tile, int tok, int half, float* x) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + lswz(tok, half * 4 + q));
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(hv[e]);
+      x[8 * q + 2 * e] = f.x;
+      x[8 * q + 2 * e + 1] = f.y;
+    }
+  }
+}
+
+struct StateSmem {
+  unsigned char phi[64 * 128];
+  unsigned char k[LSTAGES][64 * 128];
+  unsigned char v[LSTAGES][64 * 128];
+};
+
 __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_constant__ LinearArgs a) {
-  __shared__ __align__(128) unsigned char phi_s[64 * 128];
-  __shared__ __align__(128) unsigned char v_s[2][64 * 128];
+  extern __shared__ __align__(128) unsigned char state_smem[];
+  StateSmem& ss = *reinterpret_cast<StateSmem*>(state_smem);
+  unsigned char* phi_s = ss.phi;
+  auto& k_s = ss.k;
+  auto& v_s = ss.v;
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // grid (head, chunk): the CTAs resident together cover all heads of the same
@@ -153,8 +193,8 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
   const int h = blockIdx.x;
   const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
-  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v);
+  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
+  const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v) + (long long)h * a.hs;
   const int tok = tid >> 1, half = tid & 1;
 
   float acc[9][4];
@@ -163,51 +203,31 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
   const int g4 = lane >> 2;
   const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
 
-  // K of this thread's token half: registers, one 64-token block ahead
-  auto fetch_k = [&](long long nb, uint4* kd) {
-    const long long n = nb + tok;
-    if (n < n1) {
-      const uint4* kp = reinterpret_cast<const uint4*>(K + n * a.ts + (long long)h * a.hs + half * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) kd[q] = __ldg(kp + q);
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) kd[q] = make_uint4(0, 0, 0, 0);
+  const int nblk = (int)((n1 - n0 + 63) / 64);
+  for (int i = 0; i < LSTAGES - 1; ++i) {
+    if (i < nblk) {
+      fetch_rows(lsmem(k_s[i]), K, n0 + 64LL * i, n1, a.ts, tok, half);
+      fetch_rows(lsmem(v_s[i]), Vt, n0 + 64LL * i, n1, a.ts, tok, half);
     }
-  };
-  // V of this thread's token half: straight into a swizzled shared tile (zeros past the chunk)
-  auto fetch_v = [&](long long nb, int buf) {
-    const long long n = nb + tok;
-    const bool ok = n < n1;
-    const __nv_bfloat16* vp = Vt + (ok ? n : n0) * a.ts + (long long)h * a.hs + half * 32;
-    const uint32_t dst = lsmem(v_s[buf]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst + lswz(tok, half * 4 + q)),
-                   "l"(vp + 8 * q), "r"(ok ? 16 : 0));
     asm volatile("cp.async.commit_group;\n" ::);
-  };
-  uint4 kr[4];
-  fetch_k(n0, kr);
-  fetch_v(n0, 0);
-  int buf = 0;
-  for (long long nb = n0; nb < n1; nb += 64) {
-    const long long n = nb + tok;
-    const bool valid = n < n1;
-    uint4 kn[4];
-    fetch_k(nb + 64, kn);
-    float x[32];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&kr[q]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        x[8 * q + 2 * e] = f.x;
-        x[8 * q + 2 * e + 1] = f.y;
+  }
+  for (int i = 0; i < nblk; ++i) {
+    const int st = i % LSTAGES;
+    __syncthreads();   // every warp is done with the stage refilled below and with phi_s
+    {
+      const int f = i + LSTAGES - 1;
+      if (f < nblk) {
+        fetch_rows(lsmem(k_s[f % LSTAGES]), K, n0 + 64LL * f, n1, a.ts, tok, half);
+        fetch_rows(lsmem(v_s[f % LSTAGES]), Vt, n0 + 64LL * f, n1, a.ts, tok, half);
       }
-      kr[q] = kn[q];
+      asm volatile("cp.async.commit_group;\n" ::);
     }
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));   // block i has landed (own copies)
+    __syncthreads();                                                 // ... and everyone's
+    const long long n = n0 + 64LL * i + tok;
+    const bool valid = n < n1;
+    float x[32];
+    read_half(k_s[st], tok, half, x);
     {
       // every lane runs the prologue (it shuffles with lane ^ 1); padding tokens are zeroed after
       bool sp;
@@ -219,13 +239,9 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
         for (int c = 0; c < 32; ++c) x[c] = 0.f;
       }
     }
-    __syncthreads();  // the previous MMA has finished reading phi_s and v_s[buf ^ 1]
-    if (nb + 64 < n1) fetch_v(nb + 64, buf ^ 1);
-    else asm volatile("cp.async.commit_group;\n" ::);
     store_row_half_bf16(phi_s, tok, half, x);
-    asm volatile("cp.async.wait_group 1;\n" ::);   // this block's V has landed
     __syncthreads();
-    const uint32_t vb = lsmem(v_s[buf]);
+    const uint32_t vb = lsmem(v_s[st]);
     // [S | z] (rows = channels 16*warp..) += phi^T [V | 1]
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {  // 16 tokens per k-step
@@ -248,7 +264,6 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
       }
       l_mma(acc[8], af, ones, ones);
     }
-    buf ^= 1;
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
   // write partial [64][65]: row = channel, col = 0..63 (S), 64 (z)
@@ -264,13 +279,6 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
     }
   }
 }
-
-// A-fragment note: for A = phi^T (M = channels, K = tokens) the 8x8 blocks are
-// stored [token][channel]; ldmatrix.trans of block (tokens 8i.., channels 8j..)
-// yields the fragment of rows (channels) 8j.., columns (tokens) 8i... The four
-// matrices are ordered (ch 0-7, tok 0-7), (ch 8-15, tok 0-7), (ch 0-7, tok 8-15),
-// (ch 8-15, tok 8-15) = a0..a3: matrix mi takes channel chunk warp*2 + (mi & 1)
-// and token rows (mi >> 1) * 8.
 
 // --------------------------------------------------------------------------
 // fp32 state
@@ -354,14 +362,15 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constan
 // 3. apply (bf16): CTA = 128 threads, 64 tokens per step, state B operand in smem
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_constant__ LinearArgs a) {
-  __shared__ __align__(128) unsigned char phi_s[64 * 128];
+  __shared__ __align__(128) unsigned char phi_s[64 * 128];   // f(Q) block, then the bf16 output block
+  __shared__ __align__(128) unsigned char q_s[LSTAGES][64 * 128];
   __shared__ __align__(128) unsigned char b_s[NB * 128];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
   const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q) + (long long)h * a.hs;
   const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
   for (int i = tid; i < NB * 8; i += 128) {
     const int r = i >> 3, c = i & 7;
@@ -376,37 +385,26 @@ __global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_const
     bias[2 * j + 1] = a.b ? a.b[h * 64 + 8 * j + 2 * q4 + 1] : 0.f;
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-  // raw Q of this thread's token half, loaded one 64-token block ahead
-  uint4 qr[4];
-  auto fetch = [&](long long nb, uint4* qd) {
-    const long long n = nb + tok;
-    if (n < n1) {
-      const uint4* qp = reinterpret_cast<const uint4*>(Q + n * a.ts + (long long)h * a.hs + half * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) qd[q] = __ldg(qp + q);
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) qd[q] = make_uint4(0, 0, 0, 0);
+  const int nblk = (int)((n1 - n0 + 63) / 64);
+  for (int i = 0; i < LSTAGES - 1; ++i) {
+    if (i < nblk) fetch_rows(lsmem(q_s[i]), Q, n0 + 64LL * i, n1, a.ts, tok, half);
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
+  for (int i = 0; i < nblk; ++i) {
+    const int st = i % LSTAGES;
+    const long long nb = n0 + 64LL * i;
+    __syncthreads();   // the stage refilled below and phi_s (last block's output) are free
+    {
+      const int f = i + LSTAGES - 1;
+      if (f < nblk) fetch_rows(lsmem(q_s[f % LSTAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half);
+      asm volatile("cp.async.commit_group;\n" ::);
     }
-  };
-  fetch(n0, qr);
-  for (long long nb = n0; nb < n1; nb += 64) {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
+    __syncthreads();
     const long long n = nb + tok;
     const bool valid = n < n1;
-    uint4 qn[4];
-    fetch(nb + 64, qn);
     float x[32];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&qr[q]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        x[8 * q + 2 * e] = f.x;
-        x[8 * q + 2 * e + 1] = f.y;
-      }
-      qr[q] = qn[q];
-    }
+    read_half(q_s[st], tok, half, x);
     {
       bool sp;
       int row, col;
@@ -417,7 +415,6 @@ __global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_const
         for (int c = 0; c < 32; ++c) x[c] = 0.f;
       }
     }
-    __syncthreads();
     store_row_half_bf16(phi_s, tok, half, x);
     __syncthreads();
     float acc[9][4];
@@ -451,20 +448,30 @@ __global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_const
     const float den0 = __shfl_sync(0xffffffffu, acc[8][0], lane & ~3);
     const float den1 = __shfl_sync(0xffffffffu, acc[8][2], lane & ~3);
     const float i0 = 1.0f / den0, i1 = 1.0f / den1;
+    __syncthreads();   // every warp has read phi_s: reuse it for the output block
 #pragma unroll
     for (int half2 = 0; half2 < 2; ++half2) {
-      const long long nn = nb + warp * 16 + g4 + half2 * 8;
-      if (nn >= n1) continue;
+      const int r = warp * 16 + g4 + half2 * 8;
       const float il = half2 ? i1 : i0;
-      __nv_bfloat16* dst = out + (nn * g.H + h) * D;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int c = 8 * j + 2 * q4;
-        *reinterpret_cast<__nv_bfloat162*>(dst + c) = __floats2bfloat162_rn(
-            fmaf(acc[j][half2 * 2], il, bias[2 * j]), fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
+                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
+        *reinterpret_cast<__nv_bfloat162*>(phi_s + lswz(r, j) + 4 * q4) = v2;
       }
     }
+    __syncthreads();
+    // 64 tokens x 128 bytes, written as whole 16-byte chunks of each token's head row
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int idx = tid + 128 * c, r = idx >> 3, ch = idx & 7;
+      const long long nn = nb + r;
+      if (nn < n1)
+        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
+    }
   }
+  asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
 // fp32 apply: one thread per token
@@ -512,7 +519,8 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
   {
     ProfScope prof("linear_state", st);
-    linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
+    cudaFuncSetAttribute(linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
+    linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, sizeof(StateSmem), st>>>(a);
   }
   count_launch();
   if (int rc = check_launch("linear_state_kernel")) return rc;
