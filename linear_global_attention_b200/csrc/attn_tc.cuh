@@ -23,13 +23,17 @@
 //               K-major; V MN-major);
 //   warps 2..5  softmax warpgroup, straight-line per block: tcgen05.ld of S
 //               (16x256b: rows spread over quads as in the m16n8 accumulator),
-//               scale + bias, running max, exp2, bf16 P into shared memory,
-//               and O rescaling in TMEM only when a row maximum grows by more
-//               than 2^8 (the stale maximum is exact as long as both the sum
-//               and O use it).
+//               scale + bias (packed f32x2 FMA), running max (3-input max),
+//               exp2, bf16 P into shared memory (stmatrix), and O rescaling in
+//               TMEM only when a row maximum grows by more than 2^8 (the stale
+//               maximum is exact as long as both the sum and O use it).
+// Row sums: the MMA warp also accumulates L += P x ones (N = 16) on the tensor
+// cores, so the denominator adds exactly the bf16 P values that O adds and the
+// softmax warps spend no instructions on it.
 // TMEM: NSBUF score buffers of 64 columns, then O (128 or 256 columns); M=64
 // accumulators occupy lanes 0-15, 32-47, 64-79, 96-111, i.e. 16 rows per
-// softmax warp. Every mbarrier wait is bounded by the global timer; on expiry
+// softmax warp. L sits in the other half of each lane quarter (lane offset 16)
+// of O's first 16 columns. Every mbarrier wait is bounded by the global timer; on expiry
 // the CTA records ZEBRA_ERR_TIMEOUT in a device status word, drains its own
 // copies and MMAs (bounded again), frees TMEM and exits.
 // Included by attn.cu (one translation unit with the block iterator and the
@@ -74,6 +78,7 @@ constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
 constexpr int THREADS = 192;
 constexpr uint32_t COL_O = 64 * NSBUF;   // O after the score buffers
 constexpr uint32_t TMEM_COLS = COL_O + 64 <= 128 ? 128 : 256;
+constexpr uint32_t LANE_L = 16u << 16;   // TMEM lane offset of the row-sum accumulator L
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
 static_assert(NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
@@ -83,6 +88,7 @@ struct __align__(1024) Smem {
   __nv_bfloat16 k[STAGES][64 * 64];
   __nv_bfloat16 v[STAGES][64 * 64];
   __nv_bfloat16 p[PBUF][64 * 64];
+  __nv_bfloat16 ones[16 * 64];  // B operand of the row-sum MMA (N = 16, K = 64), all 1.0
   float bias[STAGES][64];       // logit bias row of the block in each stage (log2 units)
   int all_zero[STAGES];         // 1 when every bias of the stage is 0 (a complete kept tile)
   uint64_t q_full;
@@ -202,9 +208,9 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return desc_sw128(ad
 // K rows 128 bytes apart, 8-row groups 1024 bytes apart
 __device__ __forceinline__ uint64_t desc_mn(uint32_t addr) { return desc_sw128(addr, 8192, 1024); }
 
-// instruction descriptor of kind::f16: D fp32, A/B bf16, M = 64, N = 64
-__host__ __device__ constexpr uint32_t idesc(bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((64u >> 3) << 17) |
+// instruction descriptor of kind::f16: D fp32, A/B bf16, M = 64, N = n
+__host__ __device__ constexpr uint32_t idesc(bool b_mn_major, uint32_t n = 64) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) |
          ((64u >> 4) << 24);
 }
 
@@ -245,12 +251,59 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* r) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_round(float& lo, float& hi) {
+// 16 TMEM lanes x 8 fp32 columns -> 4 registers (rows g4 and g4 + 8, columns 2 q4 and 2 q4 + 1)
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* r) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(u[0]), "r"(u[1]),
+               "r"(u[2]), "r"(u[3])
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  const float2 f = __bfloat1622float2(v);
-  lo = f.x;
-  hi = f.y;
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// (a.x, a.y) * (b.x, b.y) + (c.x, c.y) as one packed fp32 instruction
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n mov.b64 rc, {%6,%7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0,%1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// maximum of one row's 16 values in the 16x256b fragment (sv[4j + O], sv[4j + O + 1], j < 8),
+// as a tree of 3-input maxima
+template <int O>
+__device__ __forceinline__ float max_row(const float* sv) {
+  const float a = fmax3(sv[O + 0], sv[O + 1], sv[O + 4]), b = fmax3(sv[O + 5], sv[O + 8], sv[O + 9]);
+  const float c = fmax3(sv[O + 12], sv[O + 13], sv[O + 16]), d = fmax3(sv[O + 17], sv[O + 20], sv[O + 21]);
+  const float e = fmax3(sv[O + 24], sv[O + 25], sv[O + 28]);
+  return fmaxf(fmax3(a, b, c), fmax3(d, e, sv[O + 29]));
+}
+
+// four 8x8 bf16 matrices from mma-fragment registers to shared memory; this
+// thread gives the row address of row (lane & 7) of matrix (lane >> 3)
+__device__ __forceinline__ void stmatrix4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
 }
 
 // rows of block `id` of `kind` in the 2D [rows, 64] tensor map of its source
@@ -291,6 +344,9 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // the all-ones operand of the row-sum MMA (read by the tensor cores: async proxy)
+  for (int i = tid; i < 16 * 64 / 2; i += THREADS) reinterpret_cast<uint32_t*>(sm.ones)[i] = 0x3F803F80u;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
     // pre-pass: number of blocks and visible keys per query row
     BlockIter it{};
@@ -380,8 +436,9 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t id_qk = idesc(false), id_pv = idesc(true);
+      const uint32_t id_qk = idesc(false), id_pv = idesc(true), id_sum = idesc(false, 16);
       const uint64_t dq = desc_k(saddr(sm.q));
+      const uint64_t d1 = desc_k(saddr(sm.ones));
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
       int qk = 0;
       for (int j = 0; ok && j < nb; ++j) {
@@ -415,6 +472,10 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(tmem + COL_O, dp + 2 * kk, dv + (uint64_t)(2048 >> 4) * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        // L += P ones: the row sums of exactly the bf16 P that O accumulated
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + LANE_L + COL_O, dp + 2 * kk, d1 + 2 * kk, id_sum, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.v_empty[s]);
         mma_commit(&sm.pv_done[pb]);
       }
@@ -428,9 +489,20 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     const int g4 = lane >> 2, q4 = lane & 3;
     const uint32_t lane_off = (uint32_t)(32 * rb) << 16;
     const float sc = LOG2E * 0.125f;
+    const float2 sc2 = make_float2(sc, sc);
     const float NEG = -INFINITY;
-    float m0 = NEG, m1 = NEG, l0 = 0.f, l1 = 0.f;
+    float m0 = NEG, m1 = NEG;
     const int r0 = 16 * rb + g4, r1 = r0 + 8;  // query rows of this thread
+    // stmatrix row address in P buffer 0: matrix mi = lane >> 3 of store jj
+    // covers rows 16 rb + 8 (mi & 1) .. + 7 and 16-byte chunk 2 jj + (mi >> 1),
+    // placed by the 128-byte swizzle at chunk ^ (row & 7); the buffer is
+    // 1024-byte aligned, so store jj's address is p_addr ^ (jj << 5)
+    uint32_t p_addr;
+    {
+      const uint32_t mi = (uint32_t)lane >> 3, rr = (uint32_t)lane & 7;
+      const uint32_t R = (uint32_t)(16 * rb) + (mi & 1) * 8 + rr;
+      p_addr = saddr(sm.p[0]) + R * 128u + (((mi >> 1) ^ rr) << 4);
+    }
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int s = i % STAGES, b = i % NSBUF, pb = i % PBUF;
@@ -442,29 +514,27 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[b]);
 
-      // scale, bias (log2 units) and row maxima
-      float mx0 = NEG, mx1 = NEG;
+      // scale, bias (log2 units) and row maxima; sv[4j], sv[4j+1] belong to
+      // row r0 and sv[4j+2], sv[4j+3] to row r1
+      float mx0, mx1;
       const bool nobias = sm.all_zero[s] != 0;
       if (nobias) {
         // complete kept tile: maxima of the raw scores (the scale is positive)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          mx0 = fmaxf(mx0, fmaxf(sv[4 * j], sv[4 * j + 1]));
-          mx1 = fmaxf(mx1, fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
-        }
-        mx0 *= sc;
-        mx1 *= sc;
+        mx0 = max_row<0>(sv) * sc;
+        mx1 = max_row<2>(sv) * sc;
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float2 bb = *reinterpret_cast<const float2*>(&sm.bias[s][8 * j + 2 * q4]);
-          sv[4 * j + 0] = fmaf(sv[4 * j + 0], sc, bb.x);
-          sv[4 * j + 1] = fmaf(sv[4 * j + 1], sc, bb.y);
-          sv[4 * j + 2] = fmaf(sv[4 * j + 2], sc, bb.x);
-          sv[4 * j + 3] = fmaf(sv[4 * j + 3], sc, bb.y);
-          mx0 = fmaxf(mx0, fmaxf(sv[4 * j], sv[4 * j + 1]));
-          mx1 = fmaxf(mx1, fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
+          const float2 t0 = ffma2(make_float2(sv[4 * j + 0], sv[4 * j + 1]), sc2, bb);
+          const float2 t1 = ffma2(make_float2(sv[4 * j + 2], sv[4 * j + 3]), sc2, bb);
+          sv[4 * j + 0] = t0.x;
+          sv[4 * j + 1] = t0.y;
+          sv[4 * j + 2] = t1.x;
+          sv[4 * j + 3] = t1.y;
         }
+        mx0 = max_row<0>(sv);
+        mx1 = max_row<2>(sv);
       }
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -475,36 +545,29 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       const float mn0 = up0 ? mx0 : m0, mn1 = up1 ? mx1 : m1;
       const float base0 = mn0 == NEG ? 0.f : mn0, base1 = mn1 == NEG ? 0.f : mn1;
       const float al0 = up0 ? fast_exp2(m0 - base0) : 1.f, al1 = up1 ? fast_exp2(m1 - base1) : 1.f;
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pk[8][2];
-      // p = 2^(scaled score - base): one FFMA per element for complete tiles
+      // p = 2^(scaled score - base): one packed FMA per two elements
       const float ka = nobias ? sc : 1.f;
+      const float2 ka2 = make_float2(ka, ka);
+      const float2 nb0 = make_float2(-base0, -base0), nb1 = make_float2(-base1, -base1);
+      uint32_t pk[8][2];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        sv[4 * j + 0] = fast_exp2(fmaf(sv[4 * j + 0], ka, -base0));
-        sv[4 * j + 1] = fast_exp2(fmaf(sv[4 * j + 1], ka, -base0));
-        sv[4 * j + 2] = fast_exp2(fmaf(sv[4 * j + 2], ka, -base1));
-        sv[4 * j + 3] = fast_exp2(fmaf(sv[4 * j + 3], ka, -base1));
-        pk[j][0] = pack_round(sv[4 * j + 0], sv[4 * j + 1]);
-        pk[j][1] = pack_round(sv[4 * j + 2], sv[4 * j + 3]);
-        rs0 += sv[4 * j + 0] + sv[4 * j + 1];
-        rs1 += sv[4 * j + 2] + sv[4 * j + 3];
+        const float2 e0 = ffma2(make_float2(sv[4 * j + 0], sv[4 * j + 1]), ka2, nb0);
+        const float2 e1 = ffma2(make_float2(sv[4 * j + 2], sv[4 * j + 3]), ka2, nb1);
+        pk[j][0] = pack_bf16(fast_exp2(e0.x), fast_exp2(e0.y));
+        pk[j][1] = pack_bf16(fast_exp2(e1.x), fast_exp2(e1.y));
       }
-      l0 = l0 * al0 + rs0;
-      l1 = l1 * al1 + rs1;
       m0 = mn0;
       m1 = mn1;
       // P buffer pb is free once PV of block i-PBUF has completed
       if (i >= PBUF && !mbar_wait(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
-      unsigned char* pbuf = reinterpret_cast<unsigned char*>(sm.p[pb]);
-      const uint32_t x0 = (uint32_t)(r0 & 7), x1 = (uint32_t)(r1 & 7);
+      const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<uint32_t*>(pbuf + r0 * 128 + (((uint32_t)j ^ x0) << 4) + 4 * q4) = pk[j][0];
-        *reinterpret_cast<uint32_t*>(pbuf + r1 * 128 + (((uint32_t)j ^ x1) << 4) + 4 * q4) = pk[j][1];
-      }
+      for (int jj = 0; jj < 4; ++jj)
+        stmatrix4((p_addr ^ ((uint32_t)jj << 5)) + poff, pk[2 * jj][0], pk[2 * jj][1], pk[2 * jj + 1][0],
+                  pk[2 * jj + 1][1]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      // rescale O (TMEM) when any row of this warp moved its maximum
+      // rescale O and L (TMEM) when any row of this warp moved its maximum
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
         if (!mbar_wait(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag)) { ok = false; break; }
@@ -519,6 +582,13 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           o[4 * j + 3] *= al1;
         }
         tmem_st64(tmem + lane_off + COL_O, o);
+        float lv[4];
+        tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
+        lv[0] *= al0;
+        lv[1] *= al0;
+        lv[2] *= al1;
+        lv[3] *= al1;
+        tmem_st8(tmem + lane_off + LANE_L + COL_O, lv);
       }
       fence_before();
       __syncwarp();
@@ -529,8 +599,13 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     if (ok) {
       fence_after();
       float o[32];
+      float l0 = 0.f, l1 = 0.f;   // row sums (every column of L holds the row's sum)
       if (nb >= 1) {
         tmem_ld64(tmem + lane_off + COL_O, o);
+        float lv[4];
+        tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
+        l0 = lv[0];
+        l1 = lv[2];
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
@@ -572,7 +647,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           const float al = fast_exp2(m - mn), ps = fast_exp2(s_self - mn);
           const float pl = n_t > 1 ? fast_exp2(s_lm - mn) : 0.f;
           m = mn;
-          l = l * al + (q4 == 0 ? ps + pl : 0.f);
+          l = l * al + ps + pl;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
 #pragma unroll
@@ -586,10 +661,6 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           }
         }
       }
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
