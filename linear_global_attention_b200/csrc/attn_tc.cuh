@@ -11,16 +11,19 @@
 // 64-key blocks (kept tiles, landmark blocks, special-key blocks) described in
 // attn.cu. The block count is known up front (a pre-pass over the selection
 // row), so only the producer walks the stream. Warp roles:
-//   warp 0      producer: lane 0 issues TMA loads of Q once and of the K and V
-//               tile of every block into rings of STAGES 128-byte-swizzled
-//               64x64 bf16 tiles (separate K and V barriers: QK^T may start as
-//               soon as K has landed); the whole warp writes the block's 64
-//               logit biases (log2 units: 0, ln(n_u) for landmarks, -inf for
-//               masked columns) into the stage's bias row;
+//   warp 0      producer: one elected lane issues TMA loads of Q once and of
+//               the K and V tile of every block into rings of STAGES
+//               128-byte-swizzled 64x64 bf16 tiles (separate K and V barriers:
+//               QK^T may start as soon as K has landed); the whole warp writes
+//               the block's 64 logit biases (log2 units: 0, ln(n_u) for
+//               landmarks, -inf for masked columns) into the stage's bias row;
 //   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of NSBUF TMEM
 //               score buffers (tcgen05.mma M=64 N=64, K-major A/B), issued up
 //               to NSBUF blocks ahead of O += P V (P from shared memory,
-//               K-major; V MN-major);
+//               K-major; V MN-major). The whole warp runs the loop and waits;
+//               one elected lane issues each group of MMAs and its commits
+//               from a single asm block (a lane-0 branch with one MMA per
+//               statement costs several times more issue cycles per MMA);
 //   warps 2..5  softmax warpgroup, straight-line per block: tcgen05.ld of S
 //               (16x256b: rows spread over quads as in the m16n8 accumulator),
 //               scale + bias (packed f32x2 FMA), running max (3-input max),
@@ -186,10 +189,45 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
   return mbar_wait_slow(b, parity, abort_flag, limit_ns);
 }
 
+// Whole-warp form (all 32 lanes call it): the result is the same in every lane,
+// so the loops around it stay converged for the elected issues below.
+__device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                                 unsigned long long limit_ns) {
+  const unsigned long long t0 = gtime();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
+    const bool late = gtime() - t0 > limit_ns;
+    if (__any_sync(0xffffffffu, late || *abort_flag)) {
+      if (late) {
+        atomicExch(&g_status, ZEBRA_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                               unsigned long long limit_ns = WAIT_NS) {
+  if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
+  return mbar_wait_warp_slow(b, parity, abort_flag, limit_ns);
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar))
+      : "memory");
+}
+
+// One elected lane of the (converged) warp arms `bar` with the tile's bytes and
+// starts the copy.
+__device__ __forceinline__ void tma_load_2d_elect(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%4], %5;\n"
+      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n}\n"
+      ::"r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar)), "r"(64 * 64 * 2)
       : "memory");
 }
 
@@ -220,6 +258,51 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(accum));
 }
+// S = Q K^T (K = 64: four K = 16 steps) issued by one elected lane of the
+// converged warp, then commits to `bar0` and `bar1`. One asm block keeps the
+// issue cost per MMA low.
+__device__ __forceinline__ void mma_qk_elect(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint64_t* bar0,
+                                             uint64_t* bar1) {
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, 0, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %9, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%10];\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n}\n"
+      ::"r"(d), "l"(a), "l"(b), "l"(a + 2), "l"(b + 2), "l"(a + 4), "l"(b + 4), "l"(a + 6), "l"(b + 6), "r"(id),
+      "r"(saddr(bar0)), "r"(saddr(bar1))
+      : "memory");
+}
+// O += P V (V MN-major: K steps 2048 bytes apart) and L += P ones, then commits
+// to `bar0` and `bar1`; `acc` = 0 starts both accumulators.
+__device__ __forceinline__ void mma_pv_elect(uint32_t d_o, uint32_t d_l, uint64_t p, uint64_t v, uint64_t ones,
+                                             uint32_t id_pv, uint32_t id_sum, uint32_t acc, uint64_t* bar0,
+                                             uint64_t* bar1) {
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, %16, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %14, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %9, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %2, %10, %15, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %3, %11, %15, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %4, %12, %15, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %5, %13, %15, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%17];\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%18];\n}\n"
+      ::"r"(d_o), "r"(d_l), "l"(p), "l"(p + 2), "l"(p + 4), "l"(p + 6), "l"(v), "l"(v + 128), "l"(v + 256),
+      "l"(v + 384), "l"(ones), "l"(ones + 2), "l"(ones + 4), "l"(ones + 6), "r"(id_pv), "r"(id_sum), "r"(acc),
+      "r"(saddr(bar0)), "r"(saddr(bar1))
+      : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(bar))
                : "memory");
@@ -377,12 +460,9 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   const int n_t = ts.rows * ts.cols;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
+    // ---------------- producer (whole warp; one elected lane issues) ----------------
     int issued = 0;
-    if (lane == 0) {
-      mbar_expect_tx(&sm.q_full, 64 * 64 * 2);
-      tma_load_2d(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
-    }
+    tma_load_2d_elect(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
     BlockIter it{};
     it.bits = mask_word(mrow, 0, g.T);
     int kind, id, nv;
@@ -391,21 +471,13 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       const int s = issued % STAGES;
       const uint32_t par = ((issued / STAGES) - 1) & 1;
       const int row = block_row(g, h, kind, id);
-      if (lane == 0) {
-        if (issued >= STAGES && !mbar_wait(&sm.k_empty[s], par, abort_flag)) ok = false;
-        if (ok) {
-          mbar_expect_tx(&sm.k_full[s], 64 * 64 * 2);
-          tma_load_2d(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
-        }
-        // the V tile and the bias row of this stage are free once PV of block issued - STAGES is done
-        if (ok && issued >= STAGES && !mbar_wait(&sm.v_empty[s], par, abort_flag)) ok = false;
-        if (ok) {
-          mbar_expect_tx(&sm.v_full[s], 64 * 64 * 2);
-          tma_load_2d(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag);
       if (!ok) break;
+      tma_load_2d_elect(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
+      // the V tile and the bias row of this stage are free once PV of block issued - STAGES is done
+      if (issued >= STAGES) ok = mbar_wait_warp(&sm.v_empty[s], par, abort_flag);
+      if (!ok) break;
+      tma_load_2d_elect(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
       // bias row: two columns per lane
       float b0, b1;
       if (kind == 1) {
@@ -434,55 +506,44 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t id_qk = idesc(false), id_pv = idesc(true), id_sum = idesc(false, 16);
-      const uint64_t dq = desc_k(saddr(sm.q));
-      const uint64_t d1 = desc_k(saddr(sm.ones));
-      bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
-      int qk = 0;
-      for (int j = 0; ok && j < nb; ++j) {
-        // S = Q K^T up to NSBUF blocks ahead of this PV (a score buffer is
-        // reusable as soon as the softmax has loaded it)
-        while (ok && qk < nb && qk <= j + NSBUF) {
-          const int s = qk % STAGES, b = qk % NSBUF;
-          if (!mbar_wait(&sm.k_full[s], (qk / STAGES) & 1, abort_flag)) { ok = false; break; }
-          if (qk >= NSBUF && !mbar_wait(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag)) { ok = false; break; }
-          fence_after();
-          const uint64_t dk = desc_k(saddr(sm.k[s]));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem + 64u * b, dq + 2 * kk, dk + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
-          mma_commit(&sm.k_empty[s]);
-          mma_commit(&sm.s_full[b]);
-          // forward the stage's bias row to the softmax through s_full: this
-          // thread acquires it here and releases it with its own arrival
-          if (!mbar_wait(&sm.b_full[s], (qk / STAGES) & 1, abort_flag)) { ok = false; break; }
-          mbar_arrive(&sm.s_full[b]);
-          ++qk;
-        }
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    const uint32_t id_qk = idesc(false), id_pv = idesc(true), id_sum = idesc(false, 16);
+    const uint64_t dq = desc_k(saddr(sm.q));
+    const uint64_t d1 = desc_k(saddr(sm.ones));
+    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
+    int qk = 0;
+    for (int j = 0; ok && j < nb; ++j) {
+      // S = Q K^T up to NSBUF blocks ahead of this PV (a score buffer is
+      // reusable as soon as the softmax has loaded it)
+      while (qk < nb && qk <= j + NSBUF) {
+        const int s = qk % STAGES, b = qk % NSBUF;
+        ok = mbar_wait_warp(&sm.k_full[s], (qk / STAGES) & 1, abort_flag);
+        if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag);
         if (!ok) break;
-        // O += P V of block j
-        const int s = j % STAGES, pb = j % PBUF;
-        if (!mbar_wait(&sm.v_full[s], (j / STAGES) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&sm.p_full[pb], (j / PBUF) & 1, abort_flag)) { ok = false; break; }
         fence_after();
-        const uint64_t dp = desc_k(saddr(sm.p[pb]));
-        const uint64_t dv = desc_mn(saddr(sm.v[s]));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem + COL_O, dp + 2 * kk, dv + (uint64_t)(2048 >> 4) * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        // L += P ones: the row sums of exactly the bf16 P that O accumulated
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem + LANE_L + COL_O, dp + 2 * kk, d1 + 2 * kk, id_sum, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.v_empty[s]);
-        mma_commit(&sm.pv_done[pb]);
+        mma_qk_elect(tmem + 64u * b, dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
+        // forward the stage's bias row to the softmax through s_full: this
+        // warp acquires it here and releases it with one arrival
+        ok = mbar_wait_warp(&sm.b_full[s], (qk / STAGES) & 1, abort_flag);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive(&sm.s_full[b]);
+        __syncwarp();
+        ++qk;
       }
-      // drain: every MMA this thread issued completes before TMEM is freed
-      mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0, abort_flag, *abort_flag ? DRAIN_NS : WAIT_NS);
+      if (!ok) break;
+      // O += P V and L += P ones of block j
+      const int s = j % STAGES, pb = j % PBUF;
+      ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag);
+      if (ok) ok = mbar_wait_warp(&sm.p_full[pb], (j / PBUF) & 1, abort_flag);
+      if (!ok) break;
+      fence_after();
+      mma_pv_elect(tmem + COL_O, tmem + LANE_L + COL_O, desc_k(saddr(sm.p[pb])), desc_mn(saddr(sm.v[s])), d1, id_pv,
+                   id_sum, j > 0 ? 1u : 0u, &sm.v_empty[s], &sm.pv_done[pb]);
     }
+    // drain: every MMA this warp issued completes before TMEM is freed
+    if (elect_one()) mma_commit(&sm.drain);
+    __syncwarp();
+    mbar_wait_warp(&sm.drain, 0, abort_flag, *abort_flag ? DRAIN_NS : WAIT_NS);
   } else {
     // ---------------- softmax warpgroup ----------------
     const int rb = warp & 3;                  // TMEM lane quarter this warp may access
@@ -506,7 +567,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int s = i % STAGES, b = i % NSBUF, pb = i % PBUF;
-      if (!mbar_wait(&sm.s_full[b], (i / NSBUF) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&sm.s_full[b], (i / NSBUF) & 1, abort_flag)) { ok = false; break; }
       fence_after();
       float sv[32];
       tmem_ld64(tmem + lane_off + 64u * b, sv);
@@ -560,7 +621,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       m0 = mn0;
       m1 = mn1;
       // P buffer pb is free once PV of block i-PBUF has completed
-      if (i >= PBUF && !mbar_wait(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
+      if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
       const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
@@ -570,7 +631,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       // rescale O and L (TMEM) when any row of this warp moved its maximum
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
-        if (!mbar_wait(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag)) { ok = false; break; }
         fence_after();
         float o[32];
         tmem_ld64(tmem + lane_off + COL_O, o);
@@ -595,7 +656,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
     // ---------------- epilogue ----------------
-    if (ok && nb >= 1 && !mbar_wait(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag)) ok = false;
+    if (ok && nb >= 1 && !mbar_wait_warp(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag)) ok = false;
     if (ok) {
       fence_after();
       float o[32];
