@@ -48,6 +48,7 @@ struct BlockIter {
   int phase;      // 0 kept tiles, 1 landmark blocks, 2 special blocks, 3 done
   int w;          // mask word (phase 0) / tile cursor (dense rows)
   uint32_t bits;
+  uint32_t nxt;   // word w + 1, loaded one word ahead
   int lb, sb;
   int t_end;      // dense rows: end of the tile range
 };
@@ -60,14 +61,43 @@ __device__ __forceinline__ uint32_t mask_word(const uint32_t* __restrict__ mrow,
   return rem >= 32 ? m : (m & ((1u << rem) - 1u));
 }
 
+// start the kept-tile walk of selection row `mrow`
+__device__ __forceinline__ void iter_init(BlockIter& it, const uint32_t* __restrict__ mrow, const Geo& g) {
+  it.bits = mask_word(mrow, 0, g.T);
+  it.nxt = g.W > 1 ? mask_word(mrow, 1, g.T) : 0u;
+}
+
+// Landmarks of block lb (landmarks 64 lb .. 64 lb + 63) visible to query tile
+// t: tiles below T, not selected, not t itself. Returns their bit set over the
+// two mask words; `nvis` gets their count.
+__device__ __forceinline__ uint32_t lmk_visible(const uint32_t* __restrict__ mrow, const Geo& g, int t, int lb,
+                                                int& nvis) {
+  uint32_t vis = 0;
+  nvis = 0;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int w = lb * 2 + k;
+    if (w >= g.W) continue;
+    uint32_t inr = 0xffffffffu;
+    const int rem = g.T - w * 32;
+    if (rem < 32) inr = (1u << rem) - 1u;
+    uint32_t v = ~__ldg(mrow + w) & inr;
+    if ((t >> 5) == w) v &= ~(1u << (t & 31));
+    vis |= v;
+    nvis += __popc(v);
+  }
+  return vis;
+}
+
 // MODE 0: the kept tiles of row `mrow`, then landmark blocks with at least one
-// visible landmark, then special blocks.
+// visible landmark, then special blocks. `it` starts from iter_init.
 __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, const uint32_t* __restrict__ mrow,
                                                   int t, bool has_lmk, int& kind, int& id, int& nv) {
   if (it.phase == 0) {
     while (it.bits == 0 && it.w + 1 < g.W) {
       ++it.w;
-      it.bits = mask_word(mrow, it.w, g.T);
+      it.bits = it.nxt;
+      it.nxt = it.w + 1 < g.W ? mask_word(mrow, it.w + 1, g.T) : 0u;
     }
     if (it.bits != 0) {
       const int b = __ffs(it.bits) - 1;
@@ -85,20 +115,8 @@ __device__ __forceinline__ bool next_block_sparse(BlockIter& it, const Geo& g, c
       const int nlb = g.Tpad / 64;
       while (it.lb < nlb) {
         const int lb = it.lb++;
-        uint32_t vis = 0;
-        int nvis = 0;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int w = lb * 2 + k;
-          if (w >= g.W) continue;
-          uint32_t inr = 0xffffffffu;
-          const int rem = g.T - w * 32;
-          if (rem < 32) inr = (1u << rem) - 1u;
-          uint32_t v = ~__ldg(mrow + w) & inr;
-          if ((t >> 5) == w) v &= ~(1u << (t & 31));
-          vis |= v;
-          nvis += __popc(v);
-        }
+        int nvis;
+        const uint32_t vis = lmk_visible(mrow, g, t, lb, nvis);
         if (vis) {
           kind = 1;
           id = lb;
@@ -258,7 +276,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   int n_t = 0;
   if (MODE == 0) {
     it.w = 0;
-    it.bits = mask_word(mrow, 0, g.T);
+    iter_init(it, mrow, g);
     own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
     const TileShape s = tile_shape(g, t);
     n_t = s.rows * s.cols;
@@ -538,7 +556,7 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(const __grid_constant__ A
   bool with_special = true, own_kept = true;
   int n_t = 0;
   if (MODE == 0) {
-    it.bits = mask_word(mrow, 0, g.T);
+    iter_init(it, mrow, g);
     own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
     const TileShape s = tile_shape(g, t);
     n_t = s.rows * s.cols;

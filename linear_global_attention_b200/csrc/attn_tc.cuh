@@ -108,7 +108,6 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort;
   int nblocks;
-  long long keys;               // visible keys per query row over all blocks
 };
 // Shared memory per CTA: the layout, padded so that at most CTAS_PER_SM CTAs
 // fit on an SM (their TMEM, CTAS_PER_SM x TMEM_COLS columns, must fit in 512).
@@ -431,19 +430,17 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   for (int i = tid; i < 16 * 64 / 2; i += THREADS) reinterpret_cast<uint32_t*>(sm.ones)[i] = 0x3F803F80u;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
-    // pre-pass: number of blocks and visible keys per query row
-    BlockIter it{};
-    it.bits = mask_word(mrow, 0, g.T);
-    int kind, id, nv, n = 0;
-    long long keys = 0;
-    while (next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
-      ++n;
-      keys += nv;
+    // pre-pass, lane-parallel: the number of blocks the walk below will
+    // produce (kept tiles, landmark blocks with a visible landmark, special
+    // blocks)
+    int n = 0;
+    for (int w = lane; w < g.W; w += 32) n += __popc(mask_word(mrow, w, g.T));
+    for (int lb = lane; lb < g.Tpad / 64; lb += 32) {
+      int nvis;
+      n += lmk_visible(mrow, g, t, lb, nvis) != 0u ? 1 : 0;
     }
-    if (lane == 0) {
-      sm.nblocks = n;
-      sm.keys = keys;
-    }
+    n = __reduce_add_sync(0xffffffffu, n);
+    if (lane == 0) sm.nblocks = n + g.NSp / 64;
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sm.tmem_base)),
                  "r"(TMEM_COLS));
@@ -464,10 +461,12 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     int issued = 0;
     tma_load_2d_elect(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
     BlockIter it{};
-    it.bits = mask_word(mrow, 0, g.T);
+    iter_init(it, mrow, g);
     int kind, id, nv;
+    long long keys = 0;   // visible keys per query row (for the logit counter)
     bool ok = true;
     while (ok && next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+      keys += nv;
       const int s = issued % STAGES;
       const uint32_t par = ((issued / STAGES) - 1) & 1;
       const int row = block_row(g, h, kind, id);
@@ -496,6 +495,10 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         mbar_arrive(&sm.b_full[s]);
       }
       ++issued;
+    }
+    if (lane == 0 && ok && issued == nb) {
+      const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);   // the own-tile extras of the epilogue
+      atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (keys + extra)));
     }
     if (lane == 0 && *abort_flag) {
       // let the copies already in flight land before the CTA goes away
@@ -735,10 +738,6 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           *reinterpret_cast<__nv_bfloat162*>(dst + c) =
               __floats2bfloat162_rn(o[4 * j + half * 2] * il, o[4 * j + half * 2 + 1] * il);
         }
-      }
-      if (tid == 64) {
-        const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);
-        atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (sm.keys + extra)));
       }
     }
   }

@@ -23,6 +23,30 @@ constexpr int TOK = 64;    // tokens in a complete tile / rows of a packed block
 // ---------------------------------------------------------------------------
 // geometry
 // ---------------------------------------------------------------------------
+// Division by a fixed divisor d >= 1 as a multiply and a shift, exact for
+// dividends in [0, 2^31): with s = ceil(log2 d) and m = ceil(2^(31+s) / d),
+// m < 2^32 and m d - 2^(31+s) < d <= 2^s, so n m / 2^(31+s) exceeds n / d by
+// less than 1/d and its floor is floor(n / d).
+struct FastDiv {
+  uint32_t m;
+  int s;   // 0 for d = 1
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  int s = 0;
+  while ((1ull << s) < d) ++s;
+  if (s == 0) return FastDiv{0u, 0};
+  const unsigned long long m = ((1ull << (31 + s)) + d - 1) / d;
+  return FastDiv{(uint32_t)m, s};
+}
+__host__ __device__ __forceinline__ int fdiv(int n, FastDiv f) {
+  if (f.s == 0) return n;
+#ifdef __CUDA_ARCH__
+  return (int)(__umulhi((uint32_t)n, f.m) >> (f.s - 1));
+#else
+  return (int)((((unsigned long long)(uint32_t)n * f.m) >> 32) >> (f.s - 1));
+#endif
+}
+
 struct Geo {
   int V, Hp, Wp, S, H;   // views, grid rows, grid cols, special tokens/view, heads
   int L;                 // tokens per view
@@ -31,6 +55,7 @@ struct Geo {
   int NS, NSp;           // special tokens (all views), padded to a multiple of 64
   int Tpad;              // T padded to a multiple of 64
   long long N;           // tokens
+  FastDiv fTv, fTc;      // division by Tv and Tc
 };
 
 inline Geo make_geo(const zebra_geom& g) {
@@ -46,6 +71,8 @@ inline Geo make_geo(const zebra_geom& g) {
   o.NSp = (o.NS + 63) / 64 * 64;
   o.Tpad = (o.T + 63) / 64 * 64;
   o.N = (long long)o.V * o.L;
+  o.fTv = make_fastdiv((uint32_t)(o.Tv > 0 ? o.Tv : 1));
+  o.fTc = make_fastdiv((uint32_t)(o.Tc > 0 ? o.Tc : 1));
   return o;
 }
 
@@ -55,9 +82,9 @@ struct TileShape {
 
 __host__ __device__ __forceinline__ TileShape tile_shape(const Geo& g, int u) {
   TileShape s;
-  s.view = u / g.Tv;
+  s.view = fdiv(u, g.fTv);
   int p = u - s.view * g.Tv;
-  int br = p / g.Tc, bc = p - br * g.Tc;
+  int br = fdiv(p, g.fTc), bc = p - br * g.Tc;
   s.r0 = br * TILE;
   s.c0 = bc * TILE;
   s.rows = min(TILE, g.Hp - s.r0);
