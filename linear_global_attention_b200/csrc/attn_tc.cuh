@@ -121,6 +121,7 @@ static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "TMEM columns");
 struct alignas(64) Params {
   CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs;
   AttnArgs a;
+  int item0;   // first work item (h * T + t) of this launch; CTA b takes item0 + b
 };
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -401,7 +402,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   const AttnArgs& a = P.a;
   const Geo& g = a.g;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = blockIdx.x, h = blockIdx.y;
+  const int item = P.item0 + (int)blockIdx.x;
+  const int h = item / g.T, t = item - h * g.T;
   const uint32_t* mrow = a.mask + ((size_t)h * g.T + t) * g.W;
   volatile int* abort_flag = &sm.abort;
 
@@ -795,10 +797,34 @@ int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) {
     return ZEBRA_ERR_CUDA;
   }
   cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
+  // Work items (h, t) go out in launches of one resident wave each. All CTAs
+  // of a launch start together and walk their kept tiles in ascending order at
+  // about the same rate, so at any moment they read K/V tiles from a narrow
+  // window of tile indices that stays in L2. In one launch of all items the
+  // CTAs of later waves start whenever a slot frees up, their positions spread
+  // over the whole key range, and most K/V reads go to DRAM (at 1,024 views x
+  // 16 heads: 25% slower, the extra DRAM power pulling the clock down under
+  // the board's power limit).
+  const long long items = (long long)g.T * g.H;
+  long long wave = items;
+  {
+    // the kernel is built for CTAS_PER_SM resident CTAs per SM (registers,
+    // shared memory and TMEM columns are sized for it)
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        sms > 0)
+      wave = (long long)tc::CTAS_PER_SM * sms;
+    cudaGetLastError();
+  }
   ProfScope prof("attn_sparse_rows", st);
-  tc::attn_tc_kernel<<<dim3(g.T, g.H), tc::THREADS, tc::SMEM_BYTES, st>>>(p);
-  count_launch();
-  return check_launch("attn_tc_kernel");
+  for (long long base = 0; base < items; base += wave) {
+    p.item0 = (int)base;
+    const unsigned n = (unsigned)(items - base < wave ? items - base : wave);
+    tc::attn_tc_kernel<<<n, tc::THREADS, tc::SMEM_BYTES, st>>>(p);
+    count_launch();
+    if (int rc = check_launch("attn_tc_kernel")) return rc;
+  }
+  return ZEBRA_OK;
 }
 
 }  // namespace zebra
