@@ -65,6 +65,31 @@ def peaks():
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
+# DRAM traffic of the sparse attention kernel, from an ncu capture of
+# dram__bytes_read.sum + dram__bytes_write.sum over every launch of one call
+# (profiles/attn_tc_dram_v1024_h1.md): bytes per (head, query tile) work item.
+# Valid only for the kernel sources it was taken on; otherwise traffic is null.
+SPARSE_TRAFFIC = {"bytes_per_item": None, "sources_sha1": None}
+SPARSE_SOURCES = ("linear_global_attention_b200/csrc/attn_tc.cuh", "linear_global_attention_b200/csrc/attn.cu")
+
+
+def sparse_sources_sha1() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for rel in SPARSE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def sparse_traffic_per_launch(items_per_launch: float):
+    """Measured DRAM bytes per launch of the sparse kernel, or None when not measured for these sources."""
+    t = SPARSE_TRAFFIC
+    if t["bytes_per_item"] is None or t["sources_sha1"] != sparse_sources_sha1():
+        return None
+    return round(t["bytes_per_item"] * items_per_launch)
+
+
 def dist_setup():
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -259,14 +284,19 @@ def run_zebra(args):
     pk = peaks()
     kern = prof["kernels"]
     dom = max(kern.items(), key=lambda kv: kv[1][1])
-    sparse_launches, sparse_ms = kern.get("attn_sparse_rows", (0, 0.0))
-    sparse_flops_launch = 4 * 64 * prof["logits"].get("sparse_rows", 0) / max(sparse_launches, 1)
-    achieved = sparse_flops_launch / (sparse_ms / max(sparse_launches, 1) / 1e3) / 1e12 if sparse_ms else 0.0
-    roofline = {"kernel": "attn_sparse_rows", "bound": "tensor", "achieved": round(achieved, 2),
+    sparse_calls, sparse_ms = kern.get("attn_sparse_rows", (0, 0.0))
+    sparse_launches = max(prof["launches"].get("attn_sparse_rows", 0), 1)
+    sparse_flops = 4 * 64 * prof["logits"].get("sparse_rows", 0)
+    achieved = sparse_flops / (sparse_ms / 1e3) / 1e12 if sparse_ms else 0.0
+    items_per_launch = H * g.n_tiles * max(sparse_calls, 1) / sparse_launches
+    roofline = {"kernel": "attn_sparse_rows (attn_tc_kernel)", "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sustained"], 4),
-                "traffic": None, "peak_source": f"{pk['source']} bf16 sustained",
-                "algorithmic_flops_per_launch": sparse_flops_launch,
-                "avg_launch_ms": sparse_ms / max(sparse_launches, 1)}
+                "traffic": sparse_traffic_per_launch(items_per_launch),
+                "peak_source": f"{pk['source']} bf16 sustained",
+                "algorithmic_flops_per_launch": sparse_flops / sparse_launches,
+                "avg_launch_ms": sparse_ms / sparse_launches,
+                "launches_per_call": sparse_launches / max(sparse_calls, 1),
+                "work_items_per_launch": round(items_per_launch, 1)}
     # linear stage: compulsory HBM bytes (Q, K, V read once, O written once, bf16)
     lin_bytes = 8 * N * H * 64
     lin_ms = sum(kern.get(n, (0, 0.0))[1] for n in ("linear_state", "linear_reduce", "linear_apply"))

@@ -215,14 +215,17 @@ ZEBRA_API int zebra_sync_status(void* stream);
 ZEBRA_API uint64_t zebra_launch_count(void);
 
 /* Optional per-kernel timing. zebra_profile_enable(1) clears the record and
- * from then on brackets every kernel this library launches with two CUDA events
+ * from then on brackets every kernel this library launches (or, for the sparse
+ * attention kernel, the sequence of launches of one call) with two CUDA events
  * on the launching stream; it also zeroes the device counters of visible
  * attention logits. zebra_profile_enable(0) stops recording. Returns a status. */
 ZEBRA_API int zebra_profile_enable(int on);
 
 /* Waits for the recorded events and writes a text report into buf (at most len
- * bytes, NUL-terminated): one line "kernel <name> <launches> <total ms>" per
- * kernel name in first-launch order, then "logits sparse_rows <n>" and
+ * bytes, NUL-terminated): one line "kernel <name> <records> <total ms>
+ * <launches>" per kernel name in first-launch order (records = bracketed
+ * intervals, launches = kernel launches inside them), then
+ * "logits sparse_rows <n>" and
  * "logits special_rows <n>", the number of unmasked query-key logits the
  * attention kernels evaluated (4*d FLOPs each: QK^T and PV). Returns the full
  * report length. Host pointer. */

@@ -225,15 +225,22 @@ def zebra_profile_enable(on: bool = True):
 
 
 def zebra_profile_report() -> dict:
-    """{"kernels": {name: (launches, total_ms)}, "logits": {"sparse_rows": n, "special_rows": n}}."""
+    """{"kernels": {name: (records, total_ms)}, "launches": {name: kernel launches},
+    "logits": {"sparse_rows": n, "special_rows": n}}.
+
+    A record is one bracketed interval: one kernel launch, or for the sparse
+    attention kernel the launches of one call (its work goes out in rounds of
+    one resident wave).
+    """
     n = lib().zebra_profile_report(None, 0)
     buf = ctypes.create_string_buffer(int(n) + 1)
     lib().zebra_profile_report(buf, len(buf))
-    rep = {"kernels": {}, "logits": {}}
+    rep = {"kernels": {}, "launches": {}, "logits": {}}
     for line in buf.value.decode().splitlines():
         parts = line.split()
         if parts[0] == "kernel":
             rep["kernels"][parts[1]] = (int(parts[2]), float(parts[3]))
+            rep["launches"][parts[1]] = int(parts[4])
         elif parts[0] == "logits":
             rep["logits"][parts[1]] = int(parts[2])
     return rep

@@ -27,6 +27,7 @@ void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memo
 struct ProfRec {
   const char* name;
   cudaEvent_t a, b;
+  int launches;
 };
 static std::mutex g_prof_mu;
 static std::atomic<bool> g_prof_on{false};
@@ -47,7 +48,7 @@ static cudaEvent_t take_event() {
 ProfScope::ProfScope(const char* name, cudaStream_t s) : st(s) {
   if (!g_prof_on.load(std::memory_order_relaxed)) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  ProfRec r{name, take_event(), take_event()};
+  ProfRec r{name, take_event(), take_event(), 1};
   cudaEventRecord(r.a, st);
   slot = (int)g_recs.size();
   g_recs.push_back(r);
@@ -57,6 +58,12 @@ ProfScope::~ProfScope() {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   cudaEventRecord(g_recs[slot].b, st);
+}
+
+void ProfScope::set_launches(int n) {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_recs[slot].launches = n;
 }
 
 int check_launch(const char* what) {
@@ -579,25 +586,26 @@ int zebra_profile_enable(int on) {
 
 long long zebra_profile_report(char* buf, size_t len) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  std::map<std::string, std::pair<long long, double>> acc;
+  struct Acc {
+    long long records = 0, launches = 0;
+    double ms = 0.0;
+  };
+  std::map<std::string, Acc> acc;
   std::vector<std::string> order;
   for (auto& r : g_recs) {
     cudaEventSynchronize(r.b);
     float ms = 0.f;
     cudaEventElapsedTime(&ms, r.a, r.b);
-    auto it = acc.find(r.name);
-    if (it == acc.end()) {
-      order.push_back(r.name);
-      acc[r.name] = {1, (double)ms};
-    } else {
-      it->second.first += 1;
-      it->second.second += ms;
-    }
+    if (acc.find(r.name) == acc.end()) order.push_back(r.name);
+    Acc& x = acc[r.name];
+    x.records += 1;
+    x.launches += r.launches;
+    x.ms += ms;
   }
   std::string out;
   char line[256];
   for (auto& n : order) {
-    snprintf(line, sizeof(line), "kernel %s %lld %.6f\n", n.c_str(), acc[n].first, acc[n].second);
+    snprintf(line, sizeof(line), "kernel %s %lld %.6f %lld\n", n.c_str(), acc[n].records, acc[n].ms, acc[n].launches);
     out += line;
   }
   unsigned long long cnt[2] = {0, 0};

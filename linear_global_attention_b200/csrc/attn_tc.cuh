@@ -817,6 +817,7 @@ int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) {
     cudaGetLastError();
   }
   ProfScope prof("attn_sparse_rows", st);
+  prof.set_launches((int)((items + wave - 1) / wave));
   for (long long base = 0; base < items; base += wave) {
     p.item0 = (int)base;
     const unsigned n = (unsigned)(items - base < wave ? items - base : wave);

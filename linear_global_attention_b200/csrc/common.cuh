@@ -162,12 +162,13 @@ int check_launch(const char* what);   // ZEBRA_OK or ZEBRA_ERR_CUDA (sets the me
 
 // Optional per-kernel timing: while profiling is on (zebra_profile_enable), a
 // ProfScope records a CUDA event on `st` when it is made and another when it
-// goes out of scope, around one kernel launch.
+// goes out of scope, around one kernel launch (or set_launches(n) launches).
 struct ProfScope {
   int slot = -1;
   cudaStream_t st;
   ProfScope(const char* name, cudaStream_t st);
   ~ProfScope();
+  void set_launches(int n);
 };
 
 // visible-logit counters of the attention kernels (per device): [0] patch rows
