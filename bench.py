@@ -69,7 +69,7 @@ def peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum over every launch of one call
 # (profiles/attn_tc_dram_v1024_h1.md): bytes per (head, query tile) work item.
 # Valid only for the kernel sources it was taken on; otherwise traffic is null.
-SPARSE_TRAFFIC = {"bytes_per_item": 1660215, "sources_sha1": "311a2e06f090e3c445395575dc5bd1dbe9ba395f"}
+SPARSE_TRAFFIC = {"bytes_per_item": 1660215, "sources_sha1": "cb380bcb8ca331aa170f31c9948d0d842fab10b2"}
 SPARSE_SOURCES = ("linear_global_attention_b200/csrc/attn_tc.cuh", "linear_global_attention_b200/csrc/attn.cu")
 
 

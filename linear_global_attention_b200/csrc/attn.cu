@@ -17,13 +17,14 @@
 // All logits carry the 1/sqrt(d) scale; exponentials are base 2 with log2(e)
 // folded into the scale and biases.
 //
-// bf16 path: 4 warps x 16 query rows, QK^T and PV on mma.sync m16n8k16 with
-// fp32 accumulation; K/V blocks double-buffered in shared memory by cp.async
-// with an XOR swizzle on 16-byte chunks so ldmatrix reads are conflict-free.
+// bf16 patch rows run on the tcgen05 kernel (attn_tc.cuh, included below).
 // fp32 path: one thread per query row, plain fp32 arithmetic (small inputs).
 //
 // Special-token query rows attend all N keys: split-KV over key-tile ranges,
-// partial (max, sum, unnormalised output) per split, then a combine kernel.
+// partial (max, sum, unnormalised output) per split, then a combine kernel. In
+// bf16 they run on mma.sync m16n8k16 with fp32 accumulation, 4 warps x 16
+// query rows, K/V blocks double-buffered in shared memory by cp.async with an
+// XOR swizzle on 16-byte chunks so ldmatrix reads are conflict-free.
 #include <math.h>
 
 #include "common.cuh"
@@ -249,20 +250,24 @@ struct MmaSmem {
   float bias[2][64];
 };
 
+// Dense rows of the special-token queries (mma.sync, bf16): CTA = one block of
+// 64 special queries x one head x one key split (blockIdx.z of a.splits); the
+// key range is the split's share of the patch tiles, plus every special key in
+// split 0. Writes unnormalised partial O, row maximum and row sum for
+// special_combine_kernel. (MODE 1 is the only mode: the sparse patch rows run
+// on the tcgen05 kernel.)
 template <int MODE>
 __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
+  static_assert(MODE == 1, "dense special-token rows only");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   MmaSmem& sm = *reinterpret_cast<MmaSmem*>(smem_raw);
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y;
-  const int t = blockIdx.x;  // MODE 0: query tile; MODE 1: special query block
-  const uint32_t* mrow = MODE == 0 ? a.mask + ((size_t)h * g.T + t) * g.W : nullptr;
+  const int t = blockIdx.x;  // special query block
 
   // query rows -> shared (swizzled)
-  const __nv_bfloat16* qsrc = MODE == 0
-      ? static_cast<const __nv_bfloat16*>(a.Qp) + ((size_t)h * g.T + t) * TOK * D
-      : static_cast<const __nv_bfloat16*>(a.Qs) + ((size_t)h * g.NSp + (size_t)t * 64) * D;
+  const __nv_bfloat16* qsrc = static_cast<const __nv_bfloat16*>(a.Qs) + ((size_t)h * g.NSp + (size_t)t * 64) * D;
   for (int i = tid; i < 512; i += 128) {
     const int r = i >> 3, c = i & 7;
     cp_async16(smem_u32(sm.q) + swz(r, c), qsrc + r * D + c * 8);
@@ -271,23 +276,10 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
 
   BlockIter it{};
   it.phase = 0;
-  bool with_special = true;
-  bool own_kept = true;
-  int n_t = 0;
-  if (MODE == 0) {
-    it.w = 0;
-    iter_init(it, mrow, g);
-    own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
-    const TileShape s = tile_shape(g, t);
-    n_t = s.rows * s.cols;
-  } else {
-    const int sp = blockIdx.z;
-    it.w = (int)((long long)g.T * sp / a.splits);
-    it.t_end = (int)((long long)g.T * (sp + 1) / a.splits);
-    with_special = sp == 0;
-  }
-  // a caller-supplied mask may keep every tile: then no landmark is visible
-  const bool has_lmk = MODE == 0;
+  const int sp = blockIdx.z;
+  it.w = (int)((long long)g.T * sp / a.splits);
+  it.t_end = (int)((long long)g.T * (sp + 1) / a.splits);
+  const bool with_special = sp == 0;
 
   auto issue = [&](int kind, int id, int buf) {
     const __nv_bfloat16 *ks, *vs;
@@ -297,13 +289,12 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
       cp_async16(smem_u32(sm.k[buf]) + swz(r, c), ks + r * D + c * 8);
       cp_async16(smem_u32(sm.v[buf]) + swz(r, c), vs + r * D + c * 8);
     }
-    if (tid < 64) sm.bias[buf][tid] = block_bias(a, mrow, t, kind, id, tid);
+    if (tid < 64) sm.bias[buf][tid] = block_bias(a, nullptr, t, kind, id, tid);   // kinds 0 and 2 only
   };
 
   int kind = 0, id = 0, nv = 0;
   long long keys = 0;  // visible keys per query row, summed over blocks
-  bool have = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, kind, id, nv)
-                        : next_block_dense(it, g, with_special, kind, id, nv);
+  bool have = next_block_dense(it, g, with_special, kind, id, nv);
   if (have) {
     issue(kind, id, 0);
     keys += nv;
@@ -322,8 +313,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   int buf = 0;
   while (have) {
     int nkind = 0, nid = 0, nnv = 0;
-    const bool nhave = MODE == 0 ? next_block_sparse(it, g, mrow, t, has_lmk, nkind, nid, nnv)
-                                 : next_block_dense(it, g, with_special, nkind, nid, nnv);
+    const bool nhave = next_block_dense(it, g, with_special, nkind, nid, nnv);
     if (nhave) {
       issue(nkind, nid, buf ^ 1);
       keys += nnv;
@@ -427,89 +417,16 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   cp_async_wait<0>();
   if (!qloaded) __syncthreads();
   if (tid == 0) {
-    const long long rows = MODE == 0 ? n_t : min(64, g.NS - t * 64);
-    const long long extra = (MODE == 0 && !own_kept) ? (n_t > 1 ? 2 : 1) : 0;
-    atomicAdd(&g_logits[MODE], (unsigned long long)(rows * (keys + extra)));
+    const long long rows = min(64, g.NS - t * 64);
+    atomicAdd(&g_logits[1], (unsigned long long)(rows * keys));
   }
 
   const int r0 = warp * 16 + g4, r1 = r0 + 8;
-  if (MODE == 0) {
-    if (!own_kept) {
-      // exact self key + landmark of the other n_t - 1 tokens of the own tile
-      const size_t tb = ((size_t)h * g.T + t) * TOK * D;
-      const __nv_bfloat16* Qp = static_cast<const __nv_bfloat16*>(a.Qp) + tb;
-      const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp) + tb;
-      const __nv_bfloat16* Vp = static_cast<const __nv_bfloat16*>(a.Vp) + tb;
-      const float* km = a.km + ((size_t)h * g.T + t) * D;
-      const float* vm = a.vm + ((size_t)h * g.T + t) * D;
-      const float nt = (float)n_t;
-      const float inv = n_t > 1 ? 1.0f / (float)(n_t - 1) : 0.f;
-      const float lnb = n_t > 1 ? a.ln_tab[n_t - 1] * LOG2E : 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = half ? r1 : r0;
-        float qk = 0.f, qm = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 8 * j + 2 * q4 + e;
-            const float qv = __bfloat162float(Qp[r * D + c]);
-            qk = fmaf(qv, __bfloat162float(Kp[r * D + c]), qk);
-            qm = fmaf(qv, km[c], qm);
-          }
-        }
-        qk += __shfl_xor_sync(0xffffffffu, qk, 1);
-        qk += __shfl_xor_sync(0xffffffffu, qk, 2);
-        qm += __shfl_xor_sync(0xffffffffu, qm, 1);
-        qm += __shfl_xor_sync(0xffffffffu, qm, 2);
-        const float s_self = qk * sc;
-        const float s_lm = n_t > 1 ? (nt * qm - qk) * inv * sc + lnb : -INFINITY;
-        float& m = half ? m1 : m0;
-        float& l = half ? l1 : l0;
-        const float mn = fmaxf(m, fmaxf(s_self, s_lm));
-        const float al = fast_exp2(m - mn), ps = fast_exp2(s_self - mn);
-        const float pl = n_t > 1 ? fast_exp2(s_lm - mn) : 0.f;
-        m = mn;
-        l = l * al + (q4 == 0 ? ps + pl : 0.f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 8 * j + 2 * q4 + e;
-            const float vv = __bfloat162float(Vp[r * D + c]);
-            const float vl = (nt * vm[c] - vv) * inv;
-            float& oo = o[j][half * 2 + e];
-            oo = oo * al + ps * vv + pl * vl;
-          }
-        }
-      }
-    }
+  {
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    const TileShape s = tile_shape(g, t);
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = half ? r1 : r0;
-      if (r >= n_t) continue;
-      const float il = 1.0f / (half ? l1 : l0);
-      __nv_bfloat16* dst = out + (tile_token(g, s, r) * g.H + h) * D;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 8 * j + 2 * q4;
-        *reinterpret_cast<__nv_bfloat162*>(dst + c) =
-            __floats2bfloat162_rn(o[j][half * 2] * il, o[j][half * 2 + 1] * il);
-      }
-    }
-  } else {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    const int sp = blockIdx.z;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int r = half ? r1 : r0;
