@@ -46,6 +46,15 @@ Readings of points the page leaves open (each marked READING below):
   R16 in a stacked layer all three kinds (linear, sparse, dense) apply the
      Q/K RMS norm and the rotation before attention.
   R17 stacked layer body: x + W_o Attn(split(W_qkv x)); no bias, no MLP.
+  R20 affine fit samples [CF]: one sample per (token, view, scene, head) is
+     the pair (x, y) of 64-vectors, x the converted linear output before the
+     correction and y the teacher (dense softmax) output; samples of all heads
+     are pooled into one fit ("accumulated across ... heads"), and a per-head
+     fit is offered as an option.
+  R21 centred regularised least squares [CF]: with means mu_x, mu_y and
+     covariances C_xx = mean((x-mu_x)(x-mu_x)^T), C_xy = mean((x-mu_x)(y-mu_y)^T)
+     over the n accumulated samples, A^T = (C_xx + lam I)^-1 C_xy and
+     b = mu_y - A mu_x; lam >= 0 is a parameter (the page gives no value).
 """
 from __future__ import annotations
 
@@ -413,3 +422,58 @@ def hybrid_layer(x, w_qkv, w_o, kind: str, g: Geom, A=None, b=None, keep=None,
         else:
             raise ValueError(kind)
     return x + o.reshape(N, -1) @ np.asarray(w_o, np.float64).T
+
+
+# ----------------------------------------------------------------------------
+# closed-form centred affine fit [CF]
+# ----------------------------------------------------------------------------
+def affine_moments(x, y, per_head: bool = False) -> dict:
+    """Accumulable raw moments of the fit samples (READING R20).
+
+    x, y: [n, H, d] (any float type, taken as float64). Returns float64 arrays
+    n [G], sx [G, d], sy [G, d], sxx [G, d, d], sxy [G, d, d] with G = H for a
+    per-head fit and G = 1 when the heads are pooled. Moments of several calls
+    (calibration scenes) add up with affine_moments_add.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    n, H, d = x.shape
+    if per_head:
+        xs = [x[:, h] for h in range(H)]
+        ys = [y[:, h] for h in range(H)]
+    else:
+        xs = [x.reshape(n * H, d)]
+        ys = [y.reshape(n * H, d)]
+    return {
+        "n": np.array([float(xi.shape[0]) for xi in xs]),
+        "sx": np.stack([xi.sum(0) for xi in xs]),
+        "sy": np.stack([yi.sum(0) for yi in ys]),
+        "sxx": np.stack([xi.T @ xi for xi in xs]),
+        "sxy": np.stack([xi.T @ yi for xi, yi in zip(xs, ys)]),
+    }
+
+
+def affine_moments_add(m1: dict, m2: dict) -> dict:
+    """Moments of the union of two sample sets."""
+    return {k: m1[k] + m2[k] for k in m1}
+
+
+def affine_solve(m: dict, lam: float):
+    """A [G, d, d] and b [G, d] of the centred ridge fit from raw moments (READING R21)."""
+    out_a, out_b = [], []
+    for gi in range(m["n"].shape[0]):
+        n = m["n"][gi]
+        mu_x = m["sx"][gi] / n
+        mu_y = m["sy"][gi] / n
+        cxx = m["sxx"][gi] / n - np.outer(mu_x, mu_x)
+        cxy = m["sxy"][gi] / n - np.outer(mu_x, mu_y)
+        a_t = np.linalg.solve(cxx + lam * np.eye(cxx.shape[0]), cxy)
+        A = a_t.T
+        out_a.append(A)
+        out_b.append(mu_y - A @ mu_x)
+    return np.stack(out_a), np.stack(out_b)
+
+
+def affine_fit(x, y, lam: float, per_head: bool = False):
+    """Centred affine correction fitted to samples x -> y (READINGS R20, R21)."""
+    return affine_solve(affine_moments(x, y, per_head), lam)

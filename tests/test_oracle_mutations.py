@@ -13,6 +13,7 @@ import types
 import pytest
 
 import oracle.zebra_oracle as zo
+from tests import test_oracle_affine as affine_pins
 from tests import test_oracle_pins as pins
 
 SRC = open(zo.__file__).read()
@@ -29,6 +30,7 @@ def _mutant(old: str, new: str) -> types.ModuleType:
 
 def _fails(pin_calls, mod, monkeypatch):
     monkeypatch.setattr(pins, "oracle", mod)
+    monkeypatch.setattr(affine_pins, "oracle", mod)
     for call in pin_calls:
         try:
             call()
@@ -92,6 +94,17 @@ MUTATIONS = [
     ("tile column index uses grid rows", "(row // g.tile) * g.tile_cols + (col // g.tile)",
      "(row // g.tile) * g.tile_rows + (col // g.tile)",
      [pins.test_tile_index_is_row_major_and_views_do_not_mix]),
+    ("affine covariance not centred", 'cxx = m["sxx"][gi] / n - np.outer(mu_x, mu_x)', 'cxx = m["sxx"][gi] / n',
+     [affine_pins.test_noise_free_recovery_per_head]),
+    ("affine A transposed", "A = a_t.T", "A = a_t",
+     [affine_pins.test_noise_free_recovery_per_head]),
+    ("affine bias ignores mean of x", "out_b.append(mu_y - A @ mu_x)", "out_b.append(mu_y)",
+     [affine_pins.test_noise_free_recovery_per_head]),
+    ("affine ridge term dropped", "cxx + lam * np.eye(cxx.shape[0])", "cxx",
+     [lambda: affine_pins.test_ridge_normal_equations_two_pass(0.05)]),
+    ("affine pooled fit uses one head", "xs = [x.reshape(n * H, d)]\n        ys = [y.reshape(n * H, d)]",
+     "xs = [x[:, 0]]\n        ys = [y[:, 0]]",
+     [affine_pins.test_pooled_equals_lstsq_on_augmented_system]),
 ]
 
 
@@ -105,6 +118,7 @@ def test_unmutated_copy_passes_the_same_pins(monkeypatch):
     mod = _mutant("NEAR_TIE_REL_GAP = 1e-5", "NEAR_TIE_REL_GAP = 1e-5")
     calls = [c for m in MUTATIONS for c in m[3]]
     monkeypatch.setattr(pins, "oracle", mod)
+    monkeypatch.setattr(affine_pins, "oracle", mod)
     for c in calls:
         c()
     assert os.path.exists(zo.__file__)
