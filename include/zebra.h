@@ -29,8 +29,9 @@
  *    as void*; NULL = legacy default stream) and returns without synchronising.
  *  - Errors: argument errors return a nonzero status before anything is enqueued;
  *    zebra_last_error() then describes the failure (thread-local). Launch errors
- *    return ZEBRA_ERR_CUDA. Device-side failures (a bounded wait that ran out)
- *    set a sticky device status word, read by zebra_sync_status().
+ *    return ZEBRA_ERR_CUDA. Device-side failures (a bounded wait that ran out,
+ *    a failed numerical check) set a sticky device status word, read by
+ *    zebra_sync_status().
  *  - Inputs are never modified. Outputs are written completely.
  */
 #ifndef ZEBRA_H
@@ -56,6 +57,8 @@ extern "C" {
 #define ZEBRA_ERR_WORKSPACE 3     /* workspace smaller than zebra_workspace_bytes() */
 #define ZEBRA_ERR_CUDA 4          /* a CUDA runtime or cuBLASLt call failed */
 #define ZEBRA_ERR_TIMEOUT 5       /* a device-side bounded wait gave up (sticky) */
+#define ZEBRA_ERR_NUMERIC 6       /* a device-side numerical check failed (sticky): the affine
+                                     fit's system was not positive definite */
 
 /* Element types of Q/K/V/out. bf16 is the production type; fp32 is accepted
  * by the stage entry points for small, CPU-checkable runs. */
@@ -92,6 +95,7 @@ typedef struct zebra_layout {
 #define ZEBRA_OP_HYBRID_LINEAR 3
 #define ZEBRA_OP_HYBRID_SPARSE 4
 #define ZEBRA_OP_HYBRID_DENSE 5
+#define ZEBRA_OP_AFFINE 6         /* zebra_affine_moments */
 
 /* Number of kept key tiles per query tile for sparsity y in [0,1):
  * k = clamp(ceil((1-y)*T - 1e-6), 1, T) — the selector "retains a key-tile
@@ -207,12 +211,57 @@ ZEBRA_API size_t zebra_workspace_bytes(const zebra_geom* g, int op, zebra_dtype 
 /* Description of the last error of the calling thread ("" if none). */
 ZEBRA_API const char* zebra_last_error(void);
 
-/* Synchronises `stream`, then reads and clears the device status word of the
- * current device. Returns ZEBRA_OK, ZEBRA_ERR_TIMEOUT or ZEBRA_ERR_CUDA. */
+/* Synchronises `stream`, then reads and clears the device status words of the
+ * current device. Returns ZEBRA_OK, ZEBRA_ERR_TIMEOUT, ZEBRA_ERR_NUMERIC or
+ * ZEBRA_ERR_CUDA. */
 ZEBRA_API int zebra_sync_status(void* stream);
 
 /* Number of kernels this library has launched in this process (all devices). */
 ZEBRA_API uint64_t zebra_launch_count(void);
+
+/* ---------------------------------------------------------------------------
+ * Closed-form centred affine fit of the linear stage's output correction.
+ *
+ * Section "A closed-form fit avoids retraining from scratch": teacher (dense
+ * softmax) outputs and converted linear outputs are accumulated across scenes,
+ * tokens, heads and views, and a centred affine correction is fitted by a
+ * regularised least-squares solve in float64. One sample is the pair (x, y) of
+ * 64-vectors at one (token, head): x the linear stage's output before the
+ * correction (zebra_linear_attn with A = b = NULL), y the teacher's output.
+ * Samples of all heads are pooled into one fit (per_head = 0), or each head is
+ * fitted on its own (per_head = 1).
+ *
+ * `moments` (device, float64, caller-owned) holds, per group (1 group pooled,
+ * H groups per head), ZEBRA_AFFINE_GROUP_DOUBLES values in this order: the
+ * sample count, sum x [64], sum y [64], sum x x^T [64 x 64, row-major],
+ * sum x y^T [64 x 64, row-major; entry (i, j) = sum x_i y_j]. Zero it before
+ * the first call of a fit; each zebra_affine_moments call (one scene) adds its
+ * samples. The additions are deterministic (fixed order).
+ * ------------------------------------------------------------------------- */
+#define ZEBRA_AFFINE_GROUP_DOUBLES 8321
+
+/* Adds the moments of the samples x, y ([N, H, 64] of dtype dt, both with
+ * `layout`, NULL = contiguous) to `moments`.
+ *   workspace  device scratch of zebra_workspace_bytes(g, ZEBRA_OP_AFFINE, ..)
+ *              bytes (per-CTA partial moments)
+ * Errors: ZEBRA_ERR_INVALID_ARG (null or misaligned pointers, bad strides),
+ * ZEBRA_ERR_WORKSPACE, ZEBRA_ERR_CUDA. */
+ZEBRA_API int zebra_affine_moments(const zebra_geom* g, zebra_dtype dt, const void* x, const void* y,
+                                   const zebra_layout* layout, int per_head, double* moments, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* Solves the centred ridge fit of every group of `moments`:
+ *   mu_x = sum x / n, mu_y = sum y / n,
+ *   C_xx = sum x x^T / n - mu_x mu_x^T,  C_xy = sum x y^T / n - mu_x mu_y^T,
+ *   A^T = (C_xx + lam I)^-1 C_xy (Cholesky, float64),  b = mu_y - A mu_x,
+ * and writes A [H, 64, 64] and b [H, 64] as float32, the layout
+ * zebra_linear_attn takes (the same A, b for every head when pooled).
+ * lam >= 0 (the page gives no value). If C_xx + lam I is not positive definite
+ * or a group holds no sample, that group's A and b are NaN and
+ * zebra_sync_status() returns ZEBRA_ERR_NUMERIC.
+ * Errors: ZEBRA_ERR_INVALID_ARG (null pointers, lam < 0 or not finite). */
+ZEBRA_API int zebra_affine_solve(const zebra_geom* g, const double* moments, int per_head, double lam, float* A,
+                                 float* b, void* stream);
 
 /* Optional per-kernel timing. zebra_profile_enable(1) clears the record and
  * from then on brackets every kernel this library launches (or, for the sparse

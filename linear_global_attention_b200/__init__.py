@@ -16,20 +16,23 @@ __all__ = [
     "zebra_keep_count", "zebra_tile_pool", "zebra_tile_select", "zebra_sparse_attn",
     "zebra_linear_attn", "zebra_hybrid_layer", "zebra_workspace_bytes", "zebra_last_error",
     "zebra_sync_status", "zebra_launch_count", "zebra_version", "workspace", "zebra_profile_enable",
-    "zebra_profile_report", "zebra_linear_attn_noalloc",
+    "zebra_profile_report", "zebra_linear_attn_noalloc", "zebra_affine_moments", "zebra_affine_solve",
+    "affine_moments_buffer",
     "ZEBRA_OK", "ZEBRA_ERR_INVALID_ARG", "ZEBRA_ERR_UNSUPPORTED", "ZEBRA_ERR_WORKSPACE", "ZEBRA_ERR_CUDA",
-    "ZEBRA_ERR_TIMEOUT", "ZEBRA_F32", "ZEBRA_BF16", "ZEBRA_LAYER_LINEAR", "ZEBRA_LAYER_SPARSE",
+    "ZEBRA_ERR_TIMEOUT", "ZEBRA_ERR_NUMERIC", "ZEBRA_AFFINE_GROUP_DOUBLES", "ZEBRA_F32", "ZEBRA_BF16", "ZEBRA_LAYER_LINEAR", "ZEBRA_LAYER_SPARSE",
     "ZEBRA_LAYER_DENSE", "ZEBRA_OP_SELECT", "ZEBRA_OP_SPARSE", "ZEBRA_OP_LINEAR", "ZEBRA_OP_HYBRID_LINEAR",
-    "ZEBRA_OP_HYBRID_SPARSE", "ZEBRA_OP_HYBRID_DENSE",
+    "ZEBRA_OP_HYBRID_SPARSE", "ZEBRA_OP_HYBRID_DENSE", "ZEBRA_OP_AFFINE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzebra.so")
 
-ZEBRA_OK, ZEBRA_ERR_INVALID_ARG, ZEBRA_ERR_UNSUPPORTED, ZEBRA_ERR_WORKSPACE, ZEBRA_ERR_CUDA, ZEBRA_ERR_TIMEOUT = range(6)
+(ZEBRA_OK, ZEBRA_ERR_INVALID_ARG, ZEBRA_ERR_UNSUPPORTED, ZEBRA_ERR_WORKSPACE, ZEBRA_ERR_CUDA, ZEBRA_ERR_TIMEOUT,
+ ZEBRA_ERR_NUMERIC) = range(7)
 ZEBRA_F32, ZEBRA_BF16 = 0, 1
 ZEBRA_LAYER_LINEAR, ZEBRA_LAYER_SPARSE, ZEBRA_LAYER_DENSE = 0, 1, 2
 (ZEBRA_OP_SELECT, ZEBRA_OP_SPARSE, ZEBRA_OP_LINEAR, ZEBRA_OP_HYBRID_LINEAR, ZEBRA_OP_HYBRID_SPARSE,
- ZEBRA_OP_HYBRID_DENSE) = range(6)
+ ZEBRA_OP_HYBRID_DENSE, ZEBRA_OP_AFFINE) = range(7)
+ZEBRA_AFFINE_GROUP_DOUBLES = 8321
 
 
 class Geom(ctypes.Structure):
@@ -99,6 +102,9 @@ def lib() -> ctypes.CDLL:
             "zebra_version": (ctypes.c_char_p, []),
             "zebra_linear_attn_noalloc": (ctypes.c_int, [_G, ctypes.c_int, _P, _P, _P, _L, _P, _P, ctypes.c_float,
                                                          ctypes.c_float, _P, _P]),
+            "zebra_affine_moments": (ctypes.c_int, [_G, ctypes.c_int, _P, _P, _L, ctypes.c_int, _P, _P,
+                                                    ctypes.c_size_t, _P]),
+            "zebra_affine_solve": (ctypes.c_int, [_G, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P]),
             "zebra_profile_enable": (ctypes.c_int, [ctypes.c_int]),
             "zebra_profile_report": (ctypes.c_longlong, [ctypes.c_char_p, ctypes.c_size_t]),
         }
@@ -211,6 +217,27 @@ def zebra_linear_attn_noalloc(g: Geom, q, k, v, A, b, out, rope_base=100.0, eps=
     lay = _layout(q, k, v)
     _check(lib().zebra_linear_attn_noalloc(ctypes.byref(g), _dtype(q), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(lay),
                                            _ptr(A), _ptr(b), rope_base, eps, _ptr(out), _stream(stream)))
+
+
+def affine_moments_buffer(g: Geom, per_head: bool = False, device="cuda"):
+    """Zeroed float64 moments of one affine fit (1 group pooled, H groups per head)."""
+    import torch
+    groups = g.heads if per_head else 1
+    return torch.zeros(groups * ZEBRA_AFFINE_GROUP_DOUBLES, dtype=torch.float64, device=device)
+
+
+def zebra_affine_moments(g: Geom, x, y, moments, ws, per_head: bool = False, stream=None):
+    """Adds the moments of samples x (linear output) -> y (teacher output), both [N, H, 64], to `moments`."""
+    lay = _layout(x, y)
+    _check(lib().zebra_affine_moments(ctypes.byref(g), _dtype(x), _ptr(x), _ptr(y), ctypes.byref(lay),
+                                      1 if per_head else 0, _ptr(moments), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def zebra_affine_solve(g: Geom, moments, lam: float, A, b, per_head: bool = False, stream=None):
+    """A [H, 64, 64], b [H, 64] (float32) of the centred ridge fit of `moments`."""
+    _check(lib().zebra_affine_solve(ctypes.byref(g), _ptr(moments), 1 if per_head else 0, float(lam), _ptr(A),
+                                    _ptr(b), _stream(stream)))
 
 
 def zebra_hybrid_layer(g: Geom, kind: int, x, w_qkv, w_o, A, b, y, x_out, ws, rope_base=100.0, eps=1e-6,

@@ -402,6 +402,9 @@ size_t zebra_workspace_bytes(const zebra_geom* g, int op, zebra_dtype dt, double
       carve_linear(G, c, w);
       break;
     }
+    case ZEBRA_OP_AFFINE:
+      c.take<double>((size_t)G.H * affine_chunks(G) * AF_STRIDE);
+      break;
     case ZEBRA_OP_HYBRID_LINEAR:
     case ZEBRA_OP_HYBRID_SPARSE:
     case ZEBRA_OP_HYBRID_DENSE: {
@@ -522,6 +525,51 @@ int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const 
   return run_linear<float>(G, q, k, v, ts, hs, A, b, rope_base, eps, out, w, st);
 }
 
+int zebra_affine_moments(const zebra_geom* g, zebra_dtype dt, const void* x, const void* y,
+                         const zebra_layout* layout, int per_head, double* moments, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  ZTRY(check_geom(g));
+  ZTRY(check_dtype(dt));
+  long long ts, hs;
+  ZTRY(check_layout(g, dt, layout, &ts, &hs));
+  if (per_head != 0 && per_head != 1) return fail(ZEBRA_ERR_INVALID_ARG, "per_head must be 0 or 1");
+  if (!moments || (reinterpret_cast<uintptr_t>(moments) & 7))
+    return fail(ZEBRA_ERR_INVALID_ARG, "moments must be non-null and 8-byte aligned");
+  const Geo G = make_geo(*g);
+  if (G.N == 0) return ZEBRA_OK;
+  ZTRY(check_ptr16(x, "x"));
+  ZTRY(check_ptr16(y, "y"));
+  AffineArgs a{};
+  a.g = G;
+  a.x = x;
+  a.y = y;
+  a.ts = ts;
+  a.hs = hs;
+  a.per_head = per_head;
+  a.chunks = affine_chunks(G);
+  a.chunk_tokens = (int)((G.N + a.chunks - 1) / a.chunks);
+  a.moments = moments;
+  Carver c(workspace);
+  a.part = c.take<double>((size_t)G.H * a.chunks * AF_STRIDE);
+  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == ZEBRA_BF16 ? launch_affine_moments<__nv_bfloat16>(a, st) : launch_affine_moments<float>(a, st);
+}
+
+int zebra_affine_solve(const zebra_geom* g, const double* moments, int per_head, double lam, float* A, float* b,
+                       void* stream) {
+  ZTRY(check_geom(g));
+  if (per_head != 0 && per_head != 1) return fail(ZEBRA_ERR_INVALID_ARG, "per_head must be 0 or 1");
+  if (!(lam >= 0.0) || !std::isfinite(lam)) return fail(ZEBRA_ERR_INVALID_ARG, "lam must be finite and >= 0");
+  if (!moments || (reinterpret_cast<uintptr_t>(moments) & 7))
+    return fail(ZEBRA_ERR_INVALID_ARG, "moments must be non-null and 8-byte aligned");
+  if (!A || !b || (reinterpret_cast<uintptr_t>(A) & 3) || (reinterpret_cast<uintptr_t>(b) & 3))
+    return fail(ZEBRA_ERR_INVALID_ARG, "A and b must be non-null and 4-byte aligned");
+  ZTRY(check_device());
+  return launch_affine_solve(moments, per_head, g->heads, lam, A, b, static_cast<cudaStream_t>(stream));
+}
+
 int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void* w_qkv, const void* w_o,
                        const float* A, const float* b, double y, float rope_base, float eps, void* x_out,
                        void* workspace, size_t ws_bytes, void* stream) {
@@ -626,6 +674,9 @@ int zebra_sync_status(void* stream) {
   int st = 0;
   if (read_and_clear_status(&st) != ZEBRA_OK) return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
   if (st) return fail(ZEBRA_ERR_TIMEOUT, "a device-side wait gave up (kernel aborted; outputs are invalid)");
+  if (read_and_clear_affine_status(&st) != ZEBRA_OK)
+    return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
+  if (st) return fail(ZEBRA_ERR_NUMERIC, "an affine fit met a system that is not positive definite (A, b are NaN)");
   return ZEBRA_OK;
 }
 

@@ -88,4 +88,24 @@ struct LinearArgs {
 template <typename T> int launch_linear(const LinearArgs& a, cudaStream_t st);
 int linear_chunks(const Geo& g, int* chunk_tokens);
 
+// ---- closed-form affine fit ----
+constexpr int AF_D = 64;
+// one group's float64 moments: count, sum x, sum y, sum x x^T, sum x y^T
+constexpr int AF_N = 0, AF_SX = 1, AF_SY = AF_SX + AF_D, AF_SXX = AF_SY + AF_D, AF_SXY = AF_SXX + AF_D * AF_D;
+constexpr int AF_STRIDE = AF_SXY + AF_D * AF_D;   // 8321
+struct AffineArgs {
+  Geo g;
+  const void* x; const void* y;     // [N, H, d] samples (linear output, teacher output)
+  long long ts, hs;
+  int chunks, chunk_tokens;         // token chunks per head
+  int per_head;
+  double* part;                     // [H, chunks, AF_STRIDE] partial moments
+  double* moments;                  // [groups, AF_STRIDE], accumulated into
+};
+int affine_chunks(const Geo& g);
+template <typename T> int launch_affine_moments(const AffineArgs& a, cudaStream_t st);
+int launch_affine_solve(const double* moments, int per_head, int heads, double lam, float* A, float* b,
+                        cudaStream_t st);
+int read_and_clear_affine_status(int* out);
+
 }  // namespace zebra

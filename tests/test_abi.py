@@ -65,7 +65,7 @@ def _g(**kw):
 
 def test_workspace_bytes(L):
     g = _g()
-    for op in range(6):
+    for op in range(7):
         assert zb.zebra_workspace_bytes(g, op, zb.ZEBRA_BF16, 0.6) > 0
     bad = _g(head_dim=32)
     with pytest.raises(zb.ZebraError):
@@ -148,3 +148,28 @@ def test_no_gpu_gives_a_cuda_error_not_a_crash(L):
         pytest.skip("a GPU is present")
     assert _sparse(L, _g()) == zb.ZEBRA_ERR_CUDA
     assert "CUDA" in zb.zebra_last_error() or "device" in zb.zebra_last_error()
+
+
+def test_affine_argument_errors(L):
+    p = ctypes.c_void_p(4096)
+    g = _g()
+    big = 1 << 40
+
+    def moments(ptr=p, per_head=0, nbytes=big, xptr=p, layout=None, dtype=zb.ZEBRA_BF16):
+        return L.zebra_affine_moments(ctypes.byref(g), dtype, xptr, p, layout, per_head, ptr, p, nbytes, None)
+
+    assert moments(ptr=None) == zb.ZEBRA_ERR_INVALID_ARG                      # moments null
+    assert moments(ptr=ctypes.c_void_p(4100)) == zb.ZEBRA_ERR_INVALID_ARG     # moments misaligned
+    assert moments(per_head=2) == zb.ZEBRA_ERR_INVALID_ARG
+    assert moments(xptr=ctypes.c_void_p(4104)) == zb.ZEBRA_ERR_INVALID_ARG    # x misaligned
+    assert moments(dtype=5) == zb.ZEBRA_ERR_INVALID_ARG
+    assert moments(layout=ctypes.byref(zb.Layout(130, 64))) == zb.ZEBRA_ERR_INVALID_ARG
+    assert moments(nbytes=64) == zb.ZEBRA_ERR_WORKSPACE
+    e = _g(views=0)
+    assert L.zebra_affine_moments(ctypes.byref(e), zb.ZEBRA_BF16, None, None, None, 0, p, None, 0,
+                                  None) == zb.ZEBRA_OK                        # empty: nothing to add
+    for lam in (-1.0, float("nan"), float("inf")):
+        assert L.zebra_affine_solve(ctypes.byref(g), p, 0, lam, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_solve(ctypes.byref(g), None, 0, 0.1, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_solve(ctypes.byref(g), p, 0, 0.1, None, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_solve(ctypes.byref(g), p, 3, 0.1, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
