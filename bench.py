@@ -90,6 +90,37 @@ def sparse_traffic_per_launch(items_per_launch: float):
     return round(t["bytes_per_item"] * items_per_launch)
 
 
+def stage_rates(kern: dict, g, hbm_gbs: float) -> dict:
+    """Rates of the smaller sparse-stage kernels per sparse layer, from their event times.
+
+    kern: {name: (records, total_ms)} of the profile report; g: the layer
+    geometry (bf16). pool_pack: algorithmic bytes = patch rows of Q, K, V read
+    once; packed [H, T, 64, 64] tiles, fp32 means and landmark rows written.
+    tile_scores: 2 * 64 FLOPs per (query tile, key tile) score (fp32 ALU).
+    tile_select: the T x T fp32 scores read once per head.
+    """
+    layers = kern.get("pool_pack", (0, 0.0))[0]
+    if not layers:
+        return {}
+    H, T = g.heads, g.n_tiles
+    t_pad = (T + 63) // 64 * 64
+    patches = g.views * g.grid_h * g.grid_w
+    out = {}
+    ms = kern["pool_pack"][1] / layers
+    nbytes = 3 * patches * H * 128 + 3 * H * T * 64 * 128 + 3 * H * T * 64 * 4 + 2 * H * t_pad * 128
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["pool_pack"] = {"ms_per_layer": round(ms, 3), "bytes_per_layer": nbytes, "gbs": round(gbs, 1),
+                        "frac_hbm": round(gbs / hbm_gbs, 4)}
+    if "tile_scores" in kern:
+        ms = kern["tile_scores"][1] / layers
+        out["tile_scores"] = {"ms_per_layer": round(ms, 3),
+                              "fp32_tflops": round(2 * 64 * T * T * H / (ms / 1e3) / 1e12, 2)}
+    if "tile_select" in kern:
+        ms = kern["tile_select"][1] / layers
+        out["tile_select"] = {"ms_per_layer": round(ms, 3), "score_gbs": round(4 * T * T * H / (ms / 1e3) / 1e9, 1)}
+    return out
+
+
 def dist_setup():
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -321,6 +352,7 @@ def run_zebra(args):
         "layer_ms": {k: round(statistics.mean(v), 3) for k, v in per_layer.items() if v},
         "linear_stage_hbm": {"gbs": round(lin_gbs, 1), "peak_gbs": pk["hbm_gbs"],
                              "frac": round(lin_gbs / pk["hbm_gbs"], 4), "compulsory_bytes": lin_bytes},
+        "sparse_prep": stage_rates(kern, g, pk["hbm_gbs"]),
         "kernels": stages,
         "dominant_kernel": dom[0],
         "input_gen_s": round(gen_s, 1),
