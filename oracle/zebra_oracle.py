@@ -12,6 +12,7 @@ below by section title:
   [LC]  "Linear-centered stages plus tile-sparse stages"
   [CF]  "A closed-form fit avoids retraining from scratch"
   [SP]  "Speedup scales with the number of input views"
+  [SC]  "Sensitive stages also concentrate their attention"
 The Chinese page's section on linear and tile-sparse layers adds that each
 *complete* tile holds 64 tokens, i.e. edge tiles may be partial.
 
@@ -55,6 +56,10 @@ Readings of points the page leaves open (each marked READING below):
      covariances C_xx = mean((x-mu_x)(x-mu_x)^T), C_xy = mean((x-mu_x)(y-mu_y)^T)
      over the n accumulated samples, A^T = (C_xx + lam I)^-1 C_xy and
      b = mu_y - A mu_x; lam >= 0 is a parameter (the page gives no value).
+  R22 attention concentration [SC]: the coverage of a stage is the dense
+     softmax probability mass (scale 1/sqrt(d), all N keys) that a patch query
+     puts on the tokens of its query tile's selected key tiles, averaged over
+     queries (and heads); the mass on special-token keys is reported apart.
 """
 from __future__ import annotations
 
@@ -477,3 +482,46 @@ def affine_solve(m: dict, lam: float):
 def affine_fit(x, y, lam: float, per_head: bool = False):
     """Centred affine correction fitted to samples x -> y (READINGS R20, R21)."""
     return affine_solve(affine_moments(x, y, per_head), lam)
+
+
+# ----------------------------------------------------------------------------
+# attention concentration: dense mass covered by the selected tiles [SC]
+# ----------------------------------------------------------------------------
+def coverage(q, k, g: Geom, keep: int, query_tiles=None, heads=None):
+    """Dense softmax mass of patch queries on their selected key tiles (READING R22).
+
+    For every query row of the query tiles `query_tiles` (default: all) and
+    head in `heads` (default: all): p = softmax(q . K^T / sqrt(d)) over all N
+    keys; `selected` = the sum of p over the tokens of the key tiles the
+    selector keeps for the row's tile (select_tiles, `keep` tiles); `special`
+    = the sum of p over the special-token keys. Returns (rows [R] token
+    indices, selected [R, nh], special [R, nh]) as float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    N, H, d = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    tiles = np.arange(g.n_tiles) if query_tiles is None else np.asarray(query_tiles, dtype=np.int64)
+    order, starts, counts = tile_members(g)
+    tid = tile_of_token(g)
+    rows = np.concatenate([order[starts[t]:starts[t] + counts[t]] for t in tiles]) if len(tiles) else np.zeros(0, np.int64)
+    row_tile = tid[rows]
+    spec = special_tokens(g)
+    sel_mass = np.zeros((len(rows), len(heads)))
+    spec_mass = np.zeros((len(rows), len(heads)))
+    scale = 1.0 / math.sqrt(d)
+    for a, h in enumerate(heads):
+        qm = tile_means(q[:, h], g, (order, starts, counts))
+        km = tile_means(k[:, h], g, (order, starts, counts))
+        sel, _ = select_tiles(qm, km, keep, rows=tiles)
+        logits = (q[rows, h] @ k[:, h].T) * scale
+        logits -= logits.max(axis=1, keepdims=True)
+        p = np.exp(logits)
+        p /= p.sum(axis=1, keepdims=True)
+        pos = {int(t): i for i, t in enumerate(tiles)}
+        for r in range(len(rows)):
+            kept = np.flatnonzero(sel[pos[int(row_tile[r])]])
+            toks = np.concatenate([order[starts[u]:starts[u] + counts[u]] for u in kept]) if len(kept) else []
+            sel_mass[r, a] = p[r, toks].sum()
+            spec_mass[r, a] = p[r, spec].sum()
+    return rows, sel_mass, spec_mass

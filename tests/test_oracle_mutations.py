@@ -14,6 +14,7 @@ import pytest
 
 import oracle.zebra_oracle as zo
 from tests import test_oracle_affine as affine_pins
+from tests import test_oracle_coverage as coverage_pins
 from tests import test_oracle_pins as pins
 
 SRC = open(zo.__file__).read()
@@ -31,6 +32,7 @@ def _mutant(old: str, new: str) -> types.ModuleType:
 def _fails(pin_calls, mod, monkeypatch):
     monkeypatch.setattr(pins, "oracle", mod)
     monkeypatch.setattr(affine_pins, "oracle", mod)
+    monkeypatch.setattr(coverage_pins, "oracle", mod)
     for call in pin_calls:
         try:
             call()
@@ -105,6 +107,13 @@ MUTATIONS = [
     ("affine pooled fit uses one head", "xs = [x.reshape(n * H, d)]\n        ys = [y.reshape(n * H, d)]",
      "xs = [x[:, 0]]\n        ys = [y[:, 0]]",
      [affine_pins.test_pooled_equals_lstsq_on_augmented_system]),
+    ("coverage without the softmax scale", "logits = (q[rows, h] @ k[:, h].T) * scale",
+     "logits = (q[rows, h] @ k[:, h].T)", [coverage_pins.test_brute_force_rows]),
+    ("coverage sums the unselected tiles", "kept = np.flatnonzero(sel[pos[int(row_tile[r])]])",
+     "kept = np.flatnonzero(~sel[pos[int(row_tile[r])]])", [coverage_pins.test_all_tiles_kept_covers_all_patch_mass]),
+    ("coverage counts special keys as selected", "sel_mass[r, a] = p[r, toks].sum()",
+     "sel_mass[r, a] = p[r, toks].sum() + p[r, spec].sum()",
+     [coverage_pins.test_all_tiles_kept_covers_all_patch_mass]),
 ]
 
 
@@ -119,6 +128,7 @@ def test_unmutated_copy_passes_the_same_pins(monkeypatch):
     calls = [c for m in MUTATIONS for c in m[3]]
     monkeypatch.setattr(pins, "oracle", mod)
     monkeypatch.setattr(affine_pins, "oracle", mod)
+    monkeypatch.setattr(coverage_pins, "oracle", mod)
     for c in calls:
         c()
     assert os.path.exists(zo.__file__)
