@@ -173,3 +173,16 @@ def test_affine_argument_errors(L):
     assert L.zebra_affine_solve(ctypes.byref(g), None, 0, 0.1, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
     assert L.zebra_affine_solve(ctypes.byref(g), p, 0, 0.1, None, p, None) == zb.ZEBRA_ERR_INVALID_ARG
     assert L.zebra_affine_solve(ctypes.byref(g), p, 3, 0.1, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+
+
+def test_microbenchmark_compiles(tmp_path):
+    # the tcgen05 issue-cost microbenchmark behind profiles/mma_issue_b200.md stays buildable
+    import shutil
+    import subprocess
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    src = os.path.join(ROOT, "linear_global_attention_b200", "microbench", "mma_issue.cu")
+    r = subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-o",
+                        str(tmp_path / "mma_issue"), src], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
