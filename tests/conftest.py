@@ -16,3 +16,21 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def root():
     return ROOT
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Parity errors of every GPU-vs-oracle comparison that ran (worst per label)."""
+    mod = sys.modules.get("tests.parity_helpers")
+    rec = getattr(mod, "RECORD", None) if mod else None
+    if not rec:
+        return
+    worst = {}
+    for what, dtype, max_abs, rel in rec:
+        key = (what, dtype)
+        a, r = worst.get(key, (0.0, 0.0))
+        worst[key] = (max(a, max_abs), max(r, rel))
+    tr = terminalreporter
+    tr.section("parity against the oracle (worst per comparison)")
+    tr.write_line(f"{'comparison':60s} {'dtype':5s} {'max_abs':>10s} {'rel_l2':>10s}")
+    for (what, dtype), (a, r) in sorted(worst.items()):
+        tr.write_line(f"{what[:60]:60s} {dtype:5s} {a:10.3e} {r:10.3e}")

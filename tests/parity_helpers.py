@@ -52,9 +52,15 @@ def errors(got: np.ndarray, want: np.ndarray):
     return max_abs, rel
 
 
+# (label, dtype, max_abs, rel_l2) of every comparison in this session, printed by
+# the terminal-summary hook in conftest.py
+RECORD = []
+
+
 def assert_close(got, want, dtype: str, what: str = ""):
     max_abs, rel = errors(got, want)
     ta, tr = TOL[dtype]
+    RECORD.append((what, dtype, float(max_abs), float(rel)))
     assert max_abs <= ta and rel <= tr, f"{what}: max_abs {max_abs:.3e} (tol {ta}), rel_l2 {rel:.3e} (tol {tr})"
     return max_abs, rel
 
