@@ -327,7 +327,10 @@ def run_zebra(args):
                 "algorithmic_flops_per_launch": sparse_flops / sparse_launches,
                 "avg_launch_ms": sparse_ms / sparse_launches,
                 "launches_per_call": sparse_launches / max(sparse_calls, 1),
-                "work_items_per_launch": round(items_per_launch, 1)}
+                "work_items_per_launch": round(items_per_launch, 1),
+                # a 64-row query tile gives M = 64 MMAs, which use half of the tensor datapath
+                # (linear_global_attention_b200/microbench/mma_issue.cu): context, not the peak
+                "frac_of_m64_ceiling": round(achieved / (pk["bf16_sustained"] / 2), 4)}
     # linear stage: compulsory HBM bytes (Q, K, V read once, O written once, bf16)
     lin_bytes = 8 * N * H * 64
     lin_ms = sum(kern.get(n, (0, 0.0))[1] for n in ("linear_state", "linear_reduce", "linear_apply"))
