@@ -60,6 +60,11 @@ Readings of points the page leaves open (each marked READING below):
      softmax probability mass (scale 1/sqrt(d), all N keys) that a patch query
      puts on the tokens of its query tile's selected key tiles, averaged over
      queries (and heads); the mass on special-token keys is reported apart.
+  R23 layer allocation [LC]: the single-stage linear-conversion error of a
+     stage is the mean, over its fit samples, of |A x + b - y|^2 (the
+     converted output after its fitted correction against the teacher); for a
+     requested linear fraction x of L stages, the round(x * L) stages with the
+     smallest error (ties: lower stage index) become linear, the rest sparse.
 """
 from __future__ import annotations
 
@@ -455,6 +460,7 @@ def affine_moments(x, y, per_head: bool = False) -> dict:
         "sy": np.stack([yi.sum(0) for yi in ys]),
         "sxx": np.stack([xi.T @ xi for xi in xs]),
         "sxy": np.stack([xi.T @ yi for xi, yi in zip(xs, ys)]),
+        "syy": np.array([float((yi * yi).sum()) for yi in ys]),
     }
 
 
@@ -525,3 +531,34 @@ def coverage(q, k, g: Geom, keep: int, query_tiles=None, heads=None):
             sel_mass[r, a] = p[r, toks].sum()
             spec_mass[r, a] = p[r, spec].sum()
     return rows, sel_mass, spec_mass
+
+
+# ----------------------------------------------------------------------------
+# layer allocation by single-stage linear-conversion error [LC]
+# ----------------------------------------------------------------------------
+def affine_residual(m: dict, A, b) -> np.ndarray:
+    """Mean |A x + b - y|^2 over each group's samples, from its raw moments (READING R23).
+
+    Expands sum |A x + b - y|^2 = tr(A Sxx A^T) + 2 b.(A sx) - 2 tr(A Sxy)
+    + n |b|^2 - 2 b.sy + sum |y|^2 and divides by n.
+    """
+    out = []
+    for gi in range(m["n"].shape[0]):
+        n = m["n"][gi]
+        Ag = np.asarray(A[gi], np.float64)
+        bg = np.asarray(b[gi], np.float64)
+        total = (np.trace(Ag @ m["sxx"][gi] @ Ag.T) + 2.0 * bg @ (Ag @ m["sx"][gi])
+                 - 2.0 * np.trace(Ag @ m["sxy"][gi]) + n * (bg @ bg) - 2.0 * bg @ m["sy"][gi] + m["syy"][gi])
+        out.append(total / n)
+    return np.array(out)
+
+
+def allocate_layers(errors, linear_fraction: float) -> np.ndarray:
+    """True for the stages that become linear (READING R23)."""
+    errors = np.asarray(errors, dtype=np.float64)
+    L = errors.shape[0]
+    count = int(np.floor(linear_fraction * L + 0.5))
+    order = np.argsort(errors, kind="stable")   # ties keep the lower index first
+    linear = np.zeros(L, dtype=bool)
+    linear[order[:count]] = True
+    return linear

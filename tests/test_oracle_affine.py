@@ -102,3 +102,33 @@ def test_fit_reduces_error_of_linear_stage_against_dense():
     A, b = oracle.affine_fit(x, y, 0.0, per_head=True)
     corrected = np.einsum("nhj,hij->nhi", x, A) + b
     assert np.mean((corrected - y) ** 2) < np.mean((x - y) ** 2)
+
+
+def test_residual_from_moments_equals_direct_error():
+    # the conversion error computed from raw moments equals the mean squared
+    # error of the corrected samples
+    X, Y, _, _ = _data(8, noise=0.4)
+    m = oracle.affine_moments(X, Y, per_head=True)
+    A, b = oracle.affine_solve(m, 0.05)
+    err = oracle.affine_residual(m, A, b)
+    for h in range(X.shape[1]):
+        direct = np.mean(np.sum((X[:, h] @ A[h].T + b[h] - Y[:, h]) ** 2, axis=1))
+        assert abs(err[h] - direct) < 1e-9 * max(1.0, direct)
+    # an exact fit leaves no error
+    X0, Y0, _, _ = _data(9)
+    m0 = oracle.affine_moments(X0, Y0, per_head=True)
+    A0, b0 = oracle.affine_solve(m0, 0.0)
+    assert (np.abs(oracle.affine_residual(m0, A0, b0)) < 1e-8).all()
+
+
+def test_allocation_takes_the_lowest_errors():
+    errors = [0.5, 0.1, 0.3, 0.1, 0.9, 0.2]
+    # round(0.5 * 6) = 3 stages: the two 0.1 (lower index first) and 0.2
+    assert oracle.allocate_layers(errors, 0.5).tolist() == [False, True, False, True, False, True]
+    assert not oracle.allocate_layers(errors, 0.0).any()
+    assert oracle.allocate_layers(errors, 1.0).all()
+    # 0.7 x 24 = 16.8 -> 17 linear stages; with increasing errors they are the first 17
+    lin = oracle.allocate_layers(np.arange(24.0), 0.7)
+    assert lin.sum() == 17 and lin[:17].all()
+    # ties: the lower stage index wins the last place
+    assert oracle.allocate_layers([1.0, 1.0, 1.0], 1 / 3).tolist() == [True, False, False]

@@ -114,6 +114,12 @@ MUTATIONS = [
     ("coverage counts special keys as selected", "sel_mass[r, a] = p[r, toks].sum()",
      "sel_mass[r, a] = p[r, toks].sum() + p[r, spec].sum()",
      [coverage_pins.test_all_tiles_kept_covers_all_patch_mass]),
+    ("allocation takes the largest errors", 'order = np.argsort(errors, kind="stable")',
+     'order = np.argsort(-errors, kind="stable")', [affine_pins.test_allocation_takes_the_lowest_errors]),
+    ("allocation count truncated", "count = int(np.floor(linear_fraction * L + 0.5))",
+     "count = int(linear_fraction * L)", [affine_pins.test_allocation_takes_the_lowest_errors]),
+    ("residual drops the cross term", "- 2.0 * np.trace(Ag @ m[\"sxy\"][gi])", "",
+     [affine_pins.test_residual_from_moments_equals_direct_error]),
 ]
 
 
