@@ -489,8 +489,8 @@ int zebra_sparse_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const 
   ZTRY(check_ptr16(v, "v"));
   ZTRY(check_ptr16(out, "out"));
   if (!mask && G.T > SELECT_MAX_T) return fail(ZEBRA_ERR_UNSUPPORTED, "selection supports at most 49152 tiles");
-  if ((long long)G.T * G.H > 0x7fffffffLL)
-    return fail(ZEBRA_ERR_UNSUPPORTED, "tiles x heads must stay below 2^31 (32-bit work-item index)");
+  if ((long long)G.T * G.H * 64 > 0x7fffffffLL)
+    return fail(ZEBRA_ERR_UNSUPPORTED, "tiles x heads x 64 must stay below 2^31 (32-bit TMA row coordinates)");
   Carver c(workspace);
   SparseWs w;
   carve_sparse(G, dt, c, w);
@@ -588,8 +588,8 @@ int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void*
   ZTRY(check_ptr16(x_out, "x_out"));
   if (kind != ZEBRA_LAYER_LINEAR && G.T > SELECT_MAX_T)
     return fail(ZEBRA_ERR_UNSUPPORTED, "selection supports at most 49152 tiles");
-  if (kind != ZEBRA_LAYER_LINEAR && (long long)G.T * G.H > 0x7fffffffLL)
-    return fail(ZEBRA_ERR_UNSUPPORTED, "tiles x heads must stay below 2^31 (32-bit work-item index)");
+  if (kind != ZEBRA_LAYER_LINEAR && (long long)G.T * G.H * 64 > 0x7fffffffLL)
+    return fail(ZEBRA_ERR_UNSUPPORTED, "tiles x heads x 64 must stay below 2^31 (32-bit TMA row coordinates)");
   Carver c(workspace);
   HybridWs w;
   carve_hybrid(G, kind, c, w);

@@ -100,8 +100,8 @@ def test_sparse_argument_errors(L):
     assert "strides" in zb.zebra_last_error()
     # more tiles than the selector handles
     assert _sparse(L, _g(views=2000, grid_h=64, grid_w=64)) == zb.ZEBRA_ERR_UNSUPPORTED
-    # 49,152 tiles x 43,700 heads: more work items than a 32-bit index holds
-    assert _sparse(L, _g(views=768, grid_h=64, grid_w=64, heads=43700, n_special=0)) == zb.ZEBRA_ERR_UNSUPPORTED
+    # 49,152 tiles x 700 heads x 64 rows: beyond 32-bit TMA row coordinates
+    assert _sparse(L, _g(views=768, grid_h=64, grid_w=64, heads=700, n_special=0)) == zb.ZEBRA_ERR_UNSUPPORTED
     assert "2^31" in zb.zebra_last_error()
 
 
