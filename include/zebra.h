@@ -146,7 +146,11 @@ ZEBRA_API int zebra_tile_select(const zebra_geom* g, const float* q_mean, const 
  *   y         sparsity in [0,1); y = 0 keeps every tile (dense attention)
  *   mask      [H, T, W] selection from zebra_tile_select, or NULL to select here
  *   out       [N, H, d] of type dt, contiguous
- *   workspace zebra_workspace_bytes(g, ZEBRA_OP_SPARSE, dt, y) bytes */
+ *   workspace zebra_workspace_bytes(g, ZEBRA_OP_SPARSE, dt, y) bytes
+ * In bf16 the patch rows go out as ceil(T*H / (4 * SMs)) kernel launches of
+ * one resident wave each, all on `stream` (each becomes a node when the call
+ * is captured into a CUDA graph). Requires T*H*64 < 2^31 (ZEBRA_ERR_UNSUPPORTED
+ * otherwise) and, without a mask, T <= 49152. */
 ZEBRA_API int zebra_sparse_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k, const void* v,
                       const zebra_layout* layout, double y, const uint32_t* mask, void* out,
                       void* workspace, size_t ws_bytes, void* stream);
