@@ -67,7 +67,7 @@ def peaks():
 # ---------------------------------------------------------------------------
 # DRAM traffic of the sparse attention kernel, from an ncu capture of
 # dram__bytes_read.sum + dram__bytes_write.sum over every launch of one call
-# (profiles/attn_tc_dram_v1024_h1.md): bytes per (head, query tile) work item.
+# at 1,024 views x 1 head: bytes per (head, query tile) work item.
 # Valid only for the kernel sources it was taken on; otherwise traffic is null.
 SPARSE_TRAFFIC = {"bytes_per_item": 1660215, "sources_sha1": "cb380bcb8ca331aa170f31c9948d0d842fab10b2"}
 SPARSE_SOURCES = ("linear_global_attention_b200/csrc/attn_tc.cuh", "linear_global_attention_b200/csrc/attn.cu")
@@ -329,7 +329,7 @@ def run_zebra(args):
                 "launches_per_call": sparse_launches / max(sparse_calls, 1),
                 "work_items_per_launch": round(items_per_launch, 1),
                 # a 64-row query tile gives M = 64 MMAs, which use half of the tensor datapath
-                # (linear_global_attention_b200/microbench/mma_issue.cu): context, not the peak
+                # (measured issue rate of M = 64 tcgen05.mma on this part): context, not the peak
                 "frac_of_m64_ceiling": round(achieved / (pk["bf16_sustained"] / 2), 4)}
     # linear stage: compulsory HBM bytes (Q, K, V read once, O written once, bf16)
     lin_bytes = 8 * N * H * 64
