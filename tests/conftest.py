@@ -22,6 +22,18 @@ def pytest_terminal_summary(terminalreporter):
     """Parity errors of every GPU-vs-oracle comparison that ran (worst per label)."""
     mod = sys.modules.get("tests.parity_helpers")
     rec = getattr(mod, "RECORD", None) if mod else None
+    near = getattr(mod, "NEAR_TIES", None) if mod else None
+    if near:
+        tot = {}
+        for what, rows, n in near:
+            a, b = tot.get(what, (0, 0))
+            tot[what] = (a + rows, b + n)
+        tr = terminalreporter
+        tr.section("selection near-ties (oracle relative score gap < 1e-5; left out of element-wise checks)")
+        tr.write_line(f"{'selection comparison':60s} {'rows':>8s} {'near-tie':>9s}")
+        for what, (rows, n) in sorted(tot.items()):
+            tr.write_line(f"{what[:60]:60s} {rows:8d} {n:9d}")
+        tr.write_line(f"{'total':60s} {sum(r for r, _ in tot.values()):8d} {sum(n for _, n in tot.values()):9d}")
     if not rec:
         return
     worst = {}

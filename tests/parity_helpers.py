@@ -55,6 +55,13 @@ def errors(got: np.ndarray, want: np.ndarray):
 # (label, dtype, max_abs, rel_l2) of every comparison in this session, printed by
 # the terminal-summary hook in conftest.py
 RECORD = []
+# (label, query-tile rows compared, rows with an oracle near-tie) of every
+# selection comparison, printed by the same hook
+NEAR_TIES = []
+
+
+def record_near_ties(what: str, rows: int, near: int):
+    NEAR_TIES.append((what, int(rows), int(near)))
 
 
 def assert_close(got, want, dtype: str, what: str = ""):
@@ -91,9 +98,9 @@ def run_select(g: oracle.Geom, q, k, y: float, dtype: str):
     return unpack_mask(mask, T), nt.cpu().numpy().astype(bool), keep, mask
 
 
-def check_selection(g: oracle.Geom, q, k, keep: int, gpu_sel: np.ndarray, heads=None, rows=None):
+def check_selection(g: oracle.Geom, q, k, keep: int, gpu_sel: np.ndarray, heads=None, rows=None, what=None):
     """Bit-exact selection outside oracle near-ties; valid top-k inside them.
-    Returns {h: near-tie rows (oracle)}."""
+    Returns {h: near-tie rows (oracle)}; the near-tie count is recorded."""
     near = {}
     heads = range(g.heads) if heads is None else heads
     members = oracle.tile_members(g)
@@ -104,6 +111,7 @@ def check_selection(g: oracle.Geom, q, k, keep: int, gpu_sel: np.ndarray, heads=
         sel, gap = oracle.select_tiles(qm, km, keep, rows=r)
         nt = gap < oracle.NEAR_TIE_REL_GAP
         near[h] = r[nt]
+        record_near_ties(what or f"{g} keep={keep} head {h}", len(r), int(nt.sum()))
         gs = gpu_sel[h][r]
         assert (gs.sum(1) == keep).all(), "GPU keeps a different number of tiles"
         bad = np.nonzero((gs != sel).any(1) & ~nt)[0]

@@ -64,6 +64,7 @@ def test_sparse_stage_full_size_sampled(qkv, dev_qkv):
     tid = oracle.tile_of_token(G)
     for h in HEADS:
         near_tiles = tiles[gaps[h] < oracle.NEAR_TIE_REL_GAP]
+        ph.record_near_ties(f"full-size sparse head {h}", len(tiles), len(near_tiles))
         ok = ~np.isin(tid[rows], near_tiles)
         ph.assert_close(got[ok, h], want[ok, h], "bf16", f"full-size sparse head {h}")
     # selections of the sampled query tiles are bit-exact outside near-ties
