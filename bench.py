@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--views", type=int, default=None, help="override the view count (quick runs only)")
     p.add_argument("--no-dense", action="store_true", help="skip the dense softmax baseline")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    p.add_argument("--no-scaling", action="store_true",
+                   help="skip the view-scaling workloads and the other operating points")
     p.add_argument("--json-extra", default=None, help="also write the full result dict to this file")
     return p.parse_args()
 
@@ -361,8 +363,38 @@ def run_zebra(args):
         "input_gen_s": round(gen_s, 1),
     }
 
+    # the other operating points of the page (xL/yS), from measured per-layer
+    # times: one extra C4 sparse layer at y = 0.6 is timed here
+    if rank == 0 and not args.no_scaling:
+        first_sparse = kinds.index("sparse")
+        f = lambda: zb.zebra_hybrid_layer(g, zb.ZEBRA_LAYER_SPARSE, x0, wq[first_sparse], wo[first_sparse], None,
+                                          None, 0.6, xa, ws)
+        sp06_ms, sp06_all = timed_ms(f, 2, warmup=0)
+        t_lin = statistics.mean(per_layer["linear"])
+        t_sp08 = statistics.mean(per_layer["sparse"])
+        layer_ms = {"0.8": t_sp08, "0.6": sp06_ms}
+        ops = {}
+        for name, lin_frac, yy in (("0.5L/0.6S", 0.5, "0.6"), ("0.5L/0.8S", 0.5, "0.8"), ("0.7L/0.6S", 0.7, "0.6"),
+                                   ("0.7L/0.8S", 0.7, "0.8")):
+            n_lin = int(math.floor(lin_frac * L + 0.5))
+            st_ms = ms_step if name == "0.7L/0.8S" else n_lin * t_lin + (L - n_lin) * layer_ms[yy]
+            ops[name] = {"linear_layers": n_lin, "sparse_layers": L - n_lin, "stack_ms": round(st_ms, 1),
+                         "tokens_per_s_per_layer": round(ws_n * N * L / (st_ms / 1e3), 1),
+                         "source": "measured step" if name == "0.7L/0.8S" else "sum of measured per-layer times"}
+        result["operating_points"] = {"sparse_layer_ms_y0.6": round(sp06_ms, 1),
+                                      "sparse_layer_ms_y0.6_reps": [round(x, 1) for x in sp06_all],
+                                      "sparse_layer_ms_y0.8": round(t_sp08, 1), "linear_layer_ms": round(t_lin, 2),
+                                      "points": ops}
     if not args.no_dense and rank == 0:
         result["dense_baseline"] = dense_baseline(g, N, H, D, kern, ms_step, L)
+        if "operating_points" in result:
+            for v in result["operating_points"]["points"].values():
+                v["speedup_vs_dense_stack"] = round(result["dense_baseline"]["stack_ms"] / v["stack_ms"], 3)
+    if rank == 0 and not args.no_scaling:
+        del ws
+        import torch
+        torch.cuda.empty_cache()
+        result["view_scaling"] = view_scaling(pk)
     if not args.no_cpu and rank == 0:
         result["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
     if ws_n > 1:
@@ -372,29 +404,120 @@ def run_zebra(args):
     return result, rank
 
 
+def timed_ms(fn, reps: int, warmup: int = 1):
+    """Median device time (CUDA events on the current stream) of `reps` calls of fn after `warmup` calls."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return statistics.median(out), out
+
+
+def sdpa_ms(q, k, v, reps: int = 3):
+    """Median time of torch SDPA (bf16, flash/cuDNN) over [1, H, N, 64] tensors."""
+    import torch
+    f = lambda: torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    torch.nn.functional.scaled_dot_product_attention(q[:, :, :65536], k[:, :, :65536], v[:, :, :65536])
+    return timed_ms(f, reps, warmup=0)
+
+
+def view_scaling(pk, reps: int = 10):
+    """The view-scaling workloads at 1 GPU (section "Speedup scales with the number of
+    input views"), each timed as whole stage calls (pooling/packing, selection,
+    attention, special rows; or the three linear kernels) with CUDA events:
+      sparse_v32       32 views x (32x32 + 5), 16 heads, y = 0.8, latent recipe;
+      linear_v128      128 views x (37x37 + 5), 16 heads, the full linear stage;
+      sidebyside_v512  512 views x (37x37 + 5), 16 heads, y = 0.6 and y = 0.8,
+                       latent recipe, against torch SDPA on identical inputs.
+    Median of `reps` calls (3 for the 512-view calls and SDPA)."""
+    import torch
+
+    import linear_global_attention_b200 as zb
+    import synth
+
+    def inputs(name):
+        w = synth.WORKLOADS[name]
+        g = zb.geom(w.views, w.grid_h, w.grid_w, w.heads)
+        q, k, v = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in synth.qkv(w))
+        desc = (f"{name}: {w.views} views x ({w.grid_h}x{w.grid_w} patches + 5 special) = {g.n_tokens:,} tokens, "
+                f"{w.heads} heads x 64, bf16, {w.recipe} recipe, seed {w.seed}")
+        return w, g, q, k, v, desc
+
+    def sparse(g, q, k, v, y, n):
+        ws = zb.workspace(g, zb.ZEBRA_OP_SPARSE, zb.ZEBRA_BF16, y)
+        o = torch.empty_like(q)
+        f = lambda: zb.zebra_sparse_attn(g, q, k, v, y, o, ws)
+        f()
+        zb.zebra_profile_enable(True)
+        ms, all_ms = timed_ms(f, n, warmup=0)
+        rep = zb.zebra_profile_report()
+        zb.zebra_profile_enable(False)
+        calls, att_ms = rep["kernels"]["attn_sparse_rows"]
+        tfl = 256 * rep["logits"]["sparse_rows"] / (att_ms / 1e3) / 1e12
+        del ws, o
+        return {"keep": zb.zebra_keep_count(y, g.n_tiles), "ms": round(ms, 3), "ms_reps": [round(x, 3) for x in all_ms],
+                "tokens_per_s": round(g.n_tokens / (ms / 1e3), 1), "attn_kernel_ms": round(att_ms / calls, 3),
+                "attn_kernel_tflops": round(tfl, 1), "attn_frac_of_sustained_bf16": round(tfl / pk["bf16_sustained"], 4)}
+
+    out = {}
+    w, g, q, k, v, desc = inputs("sparse_v32")
+    out["sparse_v32"] = {"workload": desc, "y=0.8": sparse(g, q, k, v, 0.8, reps)}
+    del q, k, v
+    w, g, q, k, v, desc = inputs("linear_v128")
+    A, b = (torch.from_numpy(x).cuda() for x in synth.affine(w.heads, w.seed))
+    ws = zb.workspace(g, zb.ZEBRA_OP_LINEAR)
+    o = torch.empty_like(q)
+    ms, all_ms = timed_ms(lambda: zb.zebra_linear_attn(g, q, k, v, A, b, o, ws), 2 * reps, warmup=3)
+    nbytes = 8 * g.n_tokens * g.heads * 64
+    out["linear_v128"] = {"workload": desc, "ms": round(ms, 4), "tokens_per_s": round(g.n_tokens / (ms / 1e3), 1),
+                          "compulsory_bytes": nbytes, "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
+                          "frac_of_measured_hbm": round(nbytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 4)}
+    del q, k, v, ws, o
+    w, g, q, k, v, desc = inputs("sidebyside_v512")
+    res = {"workload": desc}
+    for y in (0.6, 0.8):
+        res[f"y={y}"] = sparse(g, q, k, v, y, 3)
+    qt, kt, vt = (x.permute(1, 0, 2).unsqueeze(0).contiguous() for x in (q, k, v))   # [1, H, N, 64]
+    del q, k, v
+    med, all_ms = sdpa_ms(qt, kt, vt, reps=3)
+    N, H = g.n_tokens, g.heads
+    res["sdpa"] = {"ms": round(med, 1), "ms_reps": [round(x, 1) for x in all_ms],
+                   "tflops": round(4 * 64 * N * N * H / (med / 1e3) / 1e12, 1)}
+    for y in (0.6, 0.8):
+        res[f"y={y}"]["speedup_vs_sdpa"] = round(med / res[f"y={y}"]["ms"], 3)
+    out["sidebyside_v512"] = res
+    del qt, kt, vt
+    torch.cuda.empty_cache()
+    return out
+
+
 def dense_baseline(g, N, H, D, kern, ms_step, L):
     """Same-GPU dense softmax layer on identical shapes: torch SDPA (flash/cuDNN,
-    bf16) over [1, 16, N, 64] plus this run's projection GEMM time per layer."""
+    bf16) over [1, 16, N, 64] (median of 3 calls) plus this run's projection
+    GEMM time per layer."""
     import torch
     gen = torch.Generator(device="cuda").manual_seed(0)
     q = torch.randn((1, H, N, 64), device="cuda", dtype=torch.bfloat16, generator=gen)
     k = torch.randn_like(q)
     v = torch.randn_like(q)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.nn.functional.scaled_dot_product_attention(q[:, :, :65536], k[:, :, :65536], v[:, :, :65536])
-    torch.cuda.synchronize()
-    e0.record()
-    o = torch.nn.functional.scaled_dot_product_attention(q, k, v)
-    e1.record()
-    torch.cuda.synchronize()
-    sdpa_ms = e0.elapsed_time(e1)
-    del q, k, v, o
+    sdpa_ms_med, sdpa_all = sdpa_ms(q, k, v, reps=3)
+    sdpa_ms_ = sdpa_ms_med
+    del q, k, v
     gemm_n, gemm_ms = kern.get("cublasLt_gemm", (0, 0.0))
     gemm_per_layer = gemm_ms / max(gemm_n, 1) * 2
-    layer_ms = sdpa_ms + gemm_per_layer
+    layer_ms = sdpa_ms_ + gemm_per_layer
     flops = 4 * 64 * N * N * H
     return {"impl": "torch.nn.functional.scaled_dot_product_attention (bf16) + the stack's projection GEMMs",
-            "sdpa_ms": round(sdpa_ms, 1), "sdpa_tflops": round(flops / (sdpa_ms / 1e3) / 1e12, 1),
+            "sdpa_ms": round(sdpa_ms_, 1), "sdpa_ms_reps": [round(x, 1) for x in sdpa_all],
+            "sdpa_tflops": round(flops / (sdpa_ms_ / 1e3) / 1e12, 1),
             "layer_ms": round(layer_ms, 1), "stack_ms": round(layer_ms * L, 1),
             "tokens_per_s_per_layer": round(N / (layer_ms / 1e3), 1),
             "hybrid_speedup": round(layer_ms * L / ms_step, 3)}

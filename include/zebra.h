@@ -171,7 +171,7 @@ ZEBRA_API int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void*
                       const zebra_layout* layout, const float* A, const float* b, float rope_base,
                       float eps, void* out, void* workspace, size_t ws_bytes, void* stream);
 
-/* The linear stage of zebra_linear_attn (same arguments, same result) for
+/* The linear stage of zebra_linear_attn (same arguments and checks) for
  * callers that cannot allocate device memory: code whose device memory is
  * owned by another framework's allocator or a fixed reservation (so a
  * cudaMalloc of a workspace would fail or fragment it), latency-critical paths
@@ -181,12 +181,18 @@ ZEBRA_API int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void*
  * Scratch: a built-in device array of 16 MiB (every GPU that loads the
  * library holds it until the process exits); no cudaMalloc, cudaFree or
  * allocating library routine is called. Geometries whose per-head state and
- * per-chunk partials do not fit in it return ZEBRA_ERR_UNSUPPORTED (at 16
- * heads any token count fits). The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) and caches it; make that first call
- * before any stream capture. Every call uses the same array, so calls that
- * overlap on the GPU (e.g. on two streams) race; serialise them. Nothing in
- * the array has to start at zero: each call overwrites what it reads. */
+ * one chunk's partials do not fit in it return ZEBRA_ERR_UNSUPPORTED (at 16
+ * heads any token count fits). The token chunks are those of
+ * zebra_linear_attn while their partials fit (at 16 heads: up to 124,928
+ * tokens), and then the result is bit-identical to it; beyond that the chunks
+ * grow to fit, and the result differs from zebra_linear_attn only by the order
+ * of the fp32 sums. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture. cudaDeviceReset invalidates the cached address: do not
+ * call this entry point after a reset. Every call uses the same array, so
+ * calls that overlap on the GPU (e.g. on two streams) race; serialise them.
+ * Nothing in the array has to start at zero: each call overwrites what it
+ * reads. */
 ZEBRA_API int zebra_linear_attn_noalloc(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k,
                                         const void* v, const zebra_layout* layout, const float* A, const float* b,
                                         float rope_base, float eps, void* out, void* stream);
@@ -220,6 +226,20 @@ ZEBRA_API const char* zebra_last_error(void);
  * ZEBRA_ERR_CUDA. */
 ZEBRA_API int zebra_sync_status(void* stream);
 
+/* Test hook of the error path (no counterpart in the paper; for tests of the
+ * library only). On the current device it sets the limit of every bounded
+ * wait of the bf16 sparse attention kernel to `wait_ns` nanoseconds (0 = the
+ * default of 2 s) and, when `block` >= 0, makes that kernel's copy producer
+ * stop before the block of index `block` of each query tile's block stream,
+ * so that the tensor-core warp's wait for that block's keys runs out: the
+ * kernel then records ZEBRA_ERR_TIMEOUT in the sticky status word, lets its
+ * copies and MMAs in flight land (each wait bounded again), frees its tensor
+ * memory and exits, leaving the outputs of the affected rows undefined.
+ * zebra_sync_status() reports the timeout. zebra_debug_inject(-1, 0) restores
+ * normal operation. Every wait stays bounded, so no setting can hang the GPU.
+ * Returns ZEBRA_OK, ZEBRA_ERR_CUDA or ZEBRA_ERR_UNSUPPORTED (no sm_100 device). */
+ZEBRA_API int zebra_debug_inject(int32_t block, uint64_t wait_ns);
+
 /* Number of kernels this library has launched in this process (all devices). */
 ZEBRA_API uint64_t zebra_launch_count(void);
 
@@ -238,11 +258,11 @@ ZEBRA_API uint64_t zebra_launch_count(void);
  * `moments` (device, float64, caller-owned) holds, per group (1 group pooled,
  * H groups per head), ZEBRA_AFFINE_GROUP_DOUBLES values in this order: the
  * sample count, sum x [64], sum y [64], sum x x^T [64 x 64, row-major],
- * sum x y^T [64 x 64, row-major; entry (i, j) = sum x_i y_j]. Zero it before
- * the first call of a fit; each zebra_affine_moments call (one scene) adds its
- * samples. The additions are deterministic (fixed order).
+ * sum x y^T [64 x 64, row-major; entry (i, j) = sum x_i y_j], sum |y|^2 [1].
+ * Zero it before the first call of a fit; each zebra_affine_moments call (one
+ * scene) adds its samples. The additions are deterministic (fixed order).
  * ------------------------------------------------------------------------- */
-#define ZEBRA_AFFINE_GROUP_DOUBLES 8321
+#define ZEBRA_AFFINE_GROUP_DOUBLES 8322
 
 /* Adds the moments of the samples x, y ([N, H, 64] of dtype dt, both with
  * `layout`, NULL = contiguous) to `moments`.
@@ -266,6 +286,59 @@ ZEBRA_API int zebra_affine_moments(const zebra_geom* g, zebra_dtype dt, const vo
  * Errors: ZEBRA_ERR_INVALID_ARG (null pointers, lam < 0 or not finite). */
 ZEBRA_API int zebra_affine_solve(const zebra_geom* g, const double* moments, int per_head, double lam, float* A,
                                  float* b, void* stream);
+
+/* Attention-concentration diagnostic (section "Sensitive stages also
+ * concentrate their attention": the stages that resist linear conversion are
+ * the ones whose attention mass is concentrated). For every row of the sampled
+ * patch query tiles and every head, dense softmax attention over all N keys
+ * (scale 1/sqrt(d)) is evaluated, and its mass is split into
+ *   selected_mass  the sum of the probabilities of the tokens of the key tiles
+ *                  that `mask` keeps for the row's tile (what the sparse
+ *                  stage keeps exact), and
+ *   special_mass   the sum over the special-token keys.
+ *   q, k          [N, H, d] bf16, strided by `layout` (NULL = contiguous);
+ *                 ZEBRA_ERR_UNSUPPORTED for other types
+ *   mask          [H, T, W] selection (zebra_tile_select)
+ *   query_tiles   HOST [n_query_tiles] int32 tile indices in [0, T),
+ *                 1 <= n_query_tiles <= 1024
+ *   selected_mass, special_mass  out [n_query_tiles, H, 64] fp32: entry
+ *                 (i, h, a) for row a (row-major inside the tile) of tile
+ *                 query_tiles[i]; rows a >= n_t of a partial tile are 0
+ *   workspace     zebra_coverage_workspace_bytes(g, n_query_tiles) bytes
+ * Deterministic (fixed-order combines). */
+ZEBRA_API int zebra_coverage(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k,
+                             const zebra_layout* layout, const uint32_t* mask, const int32_t* query_tiles,
+                             int32_t n_query_tiles, float* selected_mass, float* special_mass, void* workspace,
+                             size_t ws_bytes, void* stream);
+/* Workspace bytes of zebra_coverage (0 and an error message for invalid
+ * arguments). Host only. */
+ZEBRA_API size_t zebra_coverage_workspace_bytes(const zebra_geom* g, int32_t n_query_tiles);
+
+/* Single-stage linear-conversion error (section "Linear-centered stages plus
+ * tile-sparse stages": stages are ranked by the error of converting them
+ * alone to linear attention). For every group of `moments` (accumulated by
+ * zebra_affine_moments; 1 group pooled, H per head) writes
+ *   err[g] = mean over the group's samples of |A x + b - y|^2
+ *          = (tr(A Sxx A^T) + 2 b.(A sx) - 2 tr(A Sxy) + n|b|^2 - 2 b.sy + sum|y|^2) / n
+ * in float64, with A, b the correction of zebra_affine_solve's layout
+ * ([H, 64, 64] and [H, 64] fp32; a pooled group uses head 0's). An empty group
+ * gives NaN. err: device, float64, one value per group.
+ * Errors: ZEBRA_ERR_INVALID_ARG (null or misaligned pointers). */
+ZEBRA_API int zebra_affine_residual(const zebra_geom* g, const double* moments, int per_head, const float* A,
+                                    const float* b, double* err, void* stream);
+
+/* Layer allocation for a linear fraction x (section "Linear-centered stages
+ * plus tile-sparse stages": the xL/yS setting converts the fraction x of
+ * stages with the lowest single-stage linear-conversion error to linear
+ * attention and the rest to tile-sparse attention). Host only, no CUDA call.
+ *   errors     HOST [n_layers] float64 (e.g. from zebra_affine_residual)
+ *   is_linear  HOST out [n_layers] int32: 1 = linear, 0 = sparse
+ * The count is floor(x * n_layers + 1/2); layers are ranked by error with
+ * ties (and NaN errors, which rank last) in index order. Returns the count,
+ * or -1 for n_layers < 0, x outside [0, 1] or a null pointer with
+ * n_layers > 0. */
+ZEBRA_API int32_t zebra_allocate_layers(const double* errors, int32_t n_layers, double linear_fraction,
+                                        int32_t* is_linear);
 
 /* Optional per-kernel timing. zebra_profile_enable(1) clears the record and
  * from then on brackets every kernel this library launches (or, for the sparse

@@ -17,7 +17,8 @@ __all__ = [
     "zebra_linear_attn", "zebra_hybrid_layer", "zebra_workspace_bytes", "zebra_last_error",
     "zebra_sync_status", "zebra_launch_count", "zebra_version", "workspace", "zebra_profile_enable",
     "zebra_profile_report", "zebra_linear_attn_noalloc", "zebra_affine_moments", "zebra_affine_solve",
-    "affine_moments_buffer",
+    "affine_moments_buffer", "zebra_debug_inject", "zebra_affine_residual", "zebra_allocate_layers",
+    "zebra_coverage", "zebra_coverage_workspace_bytes",
     "ZEBRA_OK", "ZEBRA_ERR_INVALID_ARG", "ZEBRA_ERR_UNSUPPORTED", "ZEBRA_ERR_WORKSPACE", "ZEBRA_ERR_CUDA",
     "ZEBRA_ERR_TIMEOUT", "ZEBRA_ERR_NUMERIC", "ZEBRA_AFFINE_GROUP_DOUBLES", "ZEBRA_F32", "ZEBRA_BF16", "ZEBRA_LAYER_LINEAR", "ZEBRA_LAYER_SPARSE",
     "ZEBRA_LAYER_DENSE", "ZEBRA_OP_SELECT", "ZEBRA_OP_SPARSE", "ZEBRA_OP_LINEAR", "ZEBRA_OP_HYBRID_LINEAR",
@@ -32,7 +33,7 @@ ZEBRA_F32, ZEBRA_BF16 = 0, 1
 ZEBRA_LAYER_LINEAR, ZEBRA_LAYER_SPARSE, ZEBRA_LAYER_DENSE = 0, 1, 2
 (ZEBRA_OP_SELECT, ZEBRA_OP_SPARSE, ZEBRA_OP_LINEAR, ZEBRA_OP_HYBRID_LINEAR, ZEBRA_OP_HYBRID_SPARSE,
  ZEBRA_OP_HYBRID_DENSE, ZEBRA_OP_AFFINE) = range(7)
-ZEBRA_AFFINE_GROUP_DOUBLES = 8321
+ZEBRA_AFFINE_GROUP_DOUBLES = 8322
 
 
 class Geom(ctypes.Structure):
@@ -105,7 +106,13 @@ def lib() -> ctypes.CDLL:
             "zebra_affine_moments": (ctypes.c_int, [_G, ctypes.c_int, _P, _P, _L, ctypes.c_int, _P, _P,
                                                     ctypes.c_size_t, _P]),
             "zebra_affine_solve": (ctypes.c_int, [_G, _P, ctypes.c_int, ctypes.c_double, _P, _P, _P]),
+            "zebra_affine_residual": (ctypes.c_int, [_G, _P, ctypes.c_int, _P, _P, _P, _P]),
+            "zebra_coverage": (ctypes.c_int, [_G, ctypes.c_int, _P, _P, _L, _P, _P, ctypes.c_int32, _P, _P, _P,
+                                              ctypes.c_size_t, _P]),
+            "zebra_coverage_workspace_bytes": (ctypes.c_size_t, [_G, ctypes.c_int32]),
+            "zebra_allocate_layers": (ctypes.c_int32, [_P, ctypes.c_int32, ctypes.c_double, _P]),
             "zebra_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+            "zebra_debug_inject": (ctypes.c_int, [ctypes.c_int32, ctypes.c_uint64]),
             "zebra_profile_report": (ctypes.c_longlong, [ctypes.c_char_p, ctypes.c_size_t]),
         }
         for name, (res, args) in sig.items():
@@ -184,6 +191,11 @@ def zebra_sync_status(stream=None) -> int:
     return int(lib().zebra_sync_status(_stream(stream)))
 
 
+def zebra_debug_inject(block: int, wait_ns: int = 0):
+    """Error-path test hook of the sparse kernel (see include/zebra.h); (-1, 0) turns it off."""
+    _check(lib().zebra_debug_inject(int(block), int(wait_ns)))
+
+
 def zebra_tile_pool(g: Geom, x, x_mean, x_packed=None, tile_counts=None, stream=None):
     lay = _layout(x)
     _check(lib().zebra_tile_pool(ctypes.byref(g), _dtype(x), _ptr(x), ctypes.byref(lay), _ptr(x_mean),
@@ -238,6 +250,42 @@ def zebra_affine_solve(g: Geom, moments, lam: float, A, b, per_head: bool = Fals
     """A [H, 64, 64], b [H, 64] (float32) of the centred ridge fit of `moments`."""
     _check(lib().zebra_affine_solve(ctypes.byref(g), _ptr(moments), 1 if per_head else 0, float(lam), _ptr(A),
                                     _ptr(b), _stream(stream)))
+
+
+def zebra_affine_residual(g: Geom, moments, A, b, err, per_head: bool = False, stream=None):
+    """err (float64, one per group): mean |A x + b - y|^2 of each group's samples, from `moments`."""
+    _check(lib().zebra_affine_residual(ctypes.byref(g), _ptr(moments), 1 if per_head else 0, _ptr(A), _ptr(b),
+                                       _ptr(err), _stream(stream)))
+
+
+def zebra_coverage_workspace_bytes(g: Geom, n_query_tiles: int) -> int:
+    n = lib().zebra_coverage_workspace_bytes(ctypes.byref(g), int(n_query_tiles))
+    if n == 0:
+        raise ZebraError(ZEBRA_ERR_INVALID_ARG, zebra_last_error())
+    return int(n)
+
+
+def zebra_coverage(g: Geom, q, k, mask, query_tiles, selected_mass, special_mass, ws, stream=None):
+    """Dense softmax mass of the sampled tiles' rows on their selected key tiles and on the special keys.
+    query_tiles: host sequence of tile indices; outputs [n, H, 64] float32."""
+    import numpy as np
+    lay = _layout(q, k)
+    t = np.ascontiguousarray(np.asarray(query_tiles, dtype=np.int32))
+    _check(lib().zebra_coverage(ctypes.byref(g), _dtype(q), _ptr(q), _ptr(k), ctypes.byref(lay), _ptr(mask),
+                                t.ctypes.data_as(ctypes.c_void_p), len(t), _ptr(selected_mass), _ptr(special_mass),
+                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def zebra_allocate_layers(errors, linear_fraction: float):
+    """Host call: 0/1 int32 array, 1 for the round(x * L) layers of lowest error (ties in index order)."""
+    import numpy as np
+    e = np.ascontiguousarray(np.asarray(errors, dtype=np.float64))
+    out = np.zeros(len(e), dtype=np.int32)
+    n = lib().zebra_allocate_layers(e.ctypes.data_as(ctypes.c_void_p), len(e), float(linear_fraction),
+                                    out.ctypes.data_as(ctypes.c_void_p))
+    if n < 0:
+        raise ZebraError(ZEBRA_ERR_INVALID_ARG, "bad arguments to zebra_allocate_layers")
+    return out
 
 
 def zebra_hybrid_layer(g: Geom, kind: int, x, w_qkv, w_o, A, b, y, x_out, ws, rope_base=100.0, eps=1e-6,

@@ -9,7 +9,7 @@
 // Samples are pairs (x, y) of 64-vectors: x the linear stage's output before
 // the correction, y the teacher's output, one pair per (token, head) of every
 // call. Raw moments accumulate in float64 (count, sum x, sum y, sum x x^T,
-// sum x y^T), per head or pooled over heads; the solve forms the centred
+// sum x y^T, sum |y|^2), per head or pooled over heads; the solve forms the centred
 // covariances C_xx = E[x x^T] - mu_x mu_x^T, C_xy = E[x y^T] - mu_x mu_y^T and
 // returns A^T = (C_xx + lam I)^-1 C_xy, b = mu_y - A mu_x.
 //
@@ -22,6 +22,11 @@
 //   affine_solve_kernel    CTA = group: Cholesky factorisation of
 //                          C_xx + lam I, forward and back substitution for the
 //                          64 columns of A^T, all in fp64; fp32 A, b out.
+//   affine_residual_kernel CTA = group: the mean |A x + b - y|^2 over the
+//                          group's samples from its raw moments (the
+//                          single-stage conversion error that ranks stages in
+//                          section "Linear-centered stages plus tile-sparse
+//                          stages").
 #include <math.h>
 
 #include "common.cuh"
@@ -107,10 +112,23 @@ __global__ void __launch_bounds__(256) affine_moments_kernel(const __grid_consta
         }
       if (tid < 64) s1 += xs[tk][tid];
       else if (tid < 128) s1 += ys[tk][tid - 64];
+      else if (tid < 192) s1 = fma(ys[tk][tid - 128], ys[tk][tid - 128], s1);
     }
   }
+  // sum |y|^2: threads 128-191 hold one channel each; two warp sums, then one add
+  __shared__ double syy_w[2];
+  if (tid >= 128 && tid < 192) {
+    double v = s1;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) syy_w[(tid - 128) >> 5] = v;
+  }
+  __syncthreads();
   double* part = a.part + ((size_t)h * a.chunks + c) * AF_STRIDE;
-  if (tid == 0) part[AF_N] = (double)(n1 > n0 ? n1 - n0 : 0);
+  if (tid == 0) {
+    part[AF_N] = (double)(n1 > n0 ? n1 - n0 : 0);
+    part[AF_SYY] = syy_w[0] + syy_w[1];
+  }
   if (tid < 64) part[AF_SX + tid] = s1;
   else if (tid < 128) part[AF_SY + tid - 64] = s1;
 #pragma unroll
@@ -212,6 +230,57 @@ __global__ void __launch_bounds__(256) affine_solve_kernel(const double* __restr
     const float v = bad ? __int_as_float(0x7fc00000) : (float)acc;
     for (int h = h0; h < h1; ++h) b[(size_t)h * AF_D + tid] = v;
   }
+}
+
+// Mean |A x + b - y|^2 of group g's samples from its raw moments:
+//   sum |A x + b - y|^2 = tr(A Sxx A^T) + 2 b.(A sx) - 2 tr(A Sxy) + n |b|^2
+//                         - 2 b.sy + sum |y|^2,
+// divided by n (NaN for an empty group). A, b of the group: head g's when per
+// head, head 0's when pooled. Fixed-order reductions (deterministic).
+__global__ void __launch_bounds__(256) affine_residual_kernel(const double* __restrict__ moments, int per_head,
+                                                              const float* __restrict__ A,
+                                                              const float* __restrict__ b, double* __restrict__ err) {
+  __shared__ double As[AF_D][AF_D + 1];
+  __shared__ double bs[AF_D];
+  __shared__ double part[256];
+  const int tid = threadIdx.x, gidx = blockIdx.x;
+  const double* m = moments + (size_t)gidx * AF_STRIDE;
+  const int h = per_head ? gidx : 0;
+  for (int e = tid; e < AF_D * AF_D; e += 256) As[e / AF_D][e % AF_D] = (double)A[(size_t)h * AF_D * AF_D + e];
+  if (tid < AF_D) bs[tid] = (double)b[(size_t)h * AF_D + tid];
+  __syncthreads();
+  // thread (i = tid / 4, quarter = tid % 4) covers row i of A, columns q = quarter, quarter + 4, ...
+  const int i = tid >> 2, qq = tid & 3;
+  double acc = 0.0;
+  for (int q = qq; q < AF_D; q += 4) {
+    double u = 0.0;   // (A Sxx)[i][q]
+    for (int p = 0; p < AF_D; ++p) u = fma(As[i][p], m[AF_SXX + p * AF_D + q], u);
+    acc = fma(u, As[i][q], acc);                              // tr(A Sxx A^T)
+    acc = fma(-2.0 * As[i][q], m[AF_SXY + q * AF_D + i], acc); // -2 tr(A Sxy)
+    acc = fma(2.0 * bs[i] * As[i][q], m[AF_SX + q], acc);      // 2 b.(A sx)
+  }
+  if (qq == 0) acc += m[AF_N] * bs[i] * bs[i] - 2.0 * bs[i] * m[AF_SY + i];
+  part[tid] = acc;
+  __syncthreads();
+  for (int w = 128; w >= 1; w >>= 1) {
+    if (tid < w) part[tid] += part[tid + w];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const double n = m[AF_N];
+    err[gidx] = n > 0.0 ? (part[0] + m[AF_SYY]) / n : __longlong_as_double(0x7ff8000000000000LL);
+  }
+}
+
+int launch_affine_residual(const double* moments, int per_head, int heads, const float* A, const float* b,
+                           double* err, cudaStream_t st) {
+  const int groups = per_head ? heads : 1;
+  {
+    ProfScope prof("affine_residual", st);
+    affine_residual_kernel<<<groups, 256, 0, st>>>(moments, per_head, A, b, err);
+  }
+  count_launch();
+  return check_launch("affine_residual_kernel");
 }
 
 // chunks per head for the moments pass: about four CTAs per SM overall

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <map>
@@ -80,7 +81,7 @@ static int fail(int code, const std::string& msg) {
   return code;
 }
 
-static int check_geom(const zebra_geom* g) {
+int check_geom(const zebra_geom* g) {
   if (!g) return fail(ZEBRA_ERR_INVALID_ARG, "geometry pointer is null");
   if (g->head_dim != 64) return fail(ZEBRA_ERR_UNSUPPORTED, "head_dim must be 64");
   if (g->tile != 8) return fail(ZEBRA_ERR_UNSUPPORTED, "tile must be 8");
@@ -101,14 +102,14 @@ static int check_y(double y) {
   return ZEBRA_OK;
 }
 
-static int check_dtype(zebra_dtype dt) {
+int check_dtype(zebra_dtype dt) {
   if (dt != ZEBRA_F32 && dt != ZEBRA_BF16) return fail(ZEBRA_ERR_INVALID_ARG, "unknown dtype");
   return ZEBRA_OK;
 }
 
 static size_t esize(zebra_dtype dt) { return dt == ZEBRA_BF16 ? 2 : 4; }
 
-static int check_layout(const zebra_geom* g, zebra_dtype dt, const zebra_layout* lay, long long* ts, long long* hs) {
+int check_layout(const zebra_geom* g, zebra_dtype dt, const zebra_layout* lay, long long* ts, long long* hs) {
   const long long H = g->heads;
   *ts = lay ? lay->tok_stride : H * 64;
   *hs = lay ? lay->head_stride : 64;
@@ -118,14 +119,14 @@ static int check_layout(const zebra_geom* g, zebra_dtype dt, const zebra_layout*
   return ZEBRA_OK;
 }
 
-static int check_ptr16(const void* p, const char* name) {
+int check_ptr16(const void* p, const char* name) {
   if (!p) return fail(ZEBRA_ERR_INVALID_ARG, std::string(name) + " is null");
   if (reinterpret_cast<uintptr_t>(p) & 15) return fail(ZEBRA_ERR_INVALID_ARG, std::string(name) + " must be 16-byte aligned");
   return ZEBRA_OK;
 }
 
 // current device must be an sm_100 part
-static int check_device() {
+int check_device() {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -193,10 +194,12 @@ static void carve_sparse(const Geo& G, zebra_dtype dt, Carver& c, SparseWs& w) {
   w.vm = c.take<float>(means);
   w.mask = c.take<uint32_t>((size_t)G.H * G.T * G.W);
   carve_select(G, c, w.sel);
+  // key splits of the special-token rows: about 8 resident waves of work
+  // items (148 SMs x 4 CTAs each) over all query blocks and heads
   const int nqb = G.NSp / 64;
   long long splits = 1;
   if (nqb > 0) {
-    splits = (1184 + (long long)nqb * G.H - 1) / ((long long)nqb * G.H);
+    splits = (4736 + (long long)nqb * G.H - 1) / ((long long)nqb * G.H);
     if (splits > 64) splits = 64;
     if (splits > G.T) splits = G.T > 0 ? G.T : 1;
     if (splits < 1) splits = 1;
@@ -572,6 +575,86 @@ int zebra_affine_solve(const zebra_geom* g, const double* moments, int per_head,
   return launch_affine_solve(moments, per_head, g->heads, lam, A, b, static_cast<cudaStream_t>(stream));
 }
 
+size_t zebra_coverage_workspace_bytes(const zebra_geom* g, int32_t n_query_tiles) {
+  if (check_geom(g)) return 0;
+  if (n_query_tiles < 1 || n_query_tiles > COV_MAX_TILES) {
+    set_error("n_query_tiles must lie in [1, 1024]");
+    return 0;
+  }
+  const Geo G = make_geo(*g);
+  if (G.T == 0) return 256;
+  return align256((size_t)n_query_tiles * G.H * coverage_splits(G, n_query_tiles) * 64 * sizeof(float4));
+}
+
+int zebra_coverage(const zebra_geom* g, zebra_dtype dt, const void* q, const void* k, const zebra_layout* layout,
+                   const uint32_t* mask, const int32_t* query_tiles, int32_t n_query_tiles, float* selected_mass,
+                   float* special_mass, void* workspace, size_t ws_bytes, void* stream) {
+  ZTRY(check_geom(g));
+  ZTRY(check_dtype(dt));
+  if (dt != ZEBRA_BF16) return fail(ZEBRA_ERR_UNSUPPORTED, "the coverage diagnostic takes bf16 Q and K");
+  long long ts, hs;
+  ZTRY(check_layout(g, dt, layout, &ts, &hs));
+  const Geo G = make_geo(*g);
+  if (n_query_tiles < 1 || n_query_tiles > COV_MAX_TILES)
+    return fail(ZEBRA_ERR_INVALID_ARG, "n_query_tiles must lie in [1, 1024]");
+  if (!query_tiles) return fail(ZEBRA_ERR_INVALID_ARG, "query_tiles is null");
+  for (int32_t i = 0; i < n_query_tiles; ++i)
+    if (query_tiles[i] < 0 || query_tiles[i] >= G.T)
+      return fail(ZEBRA_ERR_INVALID_ARG, "query tile index outside [0, T)");
+  ZTRY(check_ptr16(q, "q"));
+  ZTRY(check_ptr16(k, "k"));
+  if (!mask) return fail(ZEBRA_ERR_INVALID_ARG, "mask is null");
+  if (!selected_mass || !special_mass) return fail(ZEBRA_ERR_INVALID_ARG, "output pointers are null");
+  CoverageArgs a{};
+  a.g = G;
+  a.q = q;
+  a.k = k;
+  a.ts = ts;
+  a.hs = hs;
+  a.mask = mask;
+  a.n = n_query_tiles;
+  a.splits = coverage_splits(G, n_query_tiles);
+  const size_t need = (size_t)a.n * G.H * a.splits * 64 * sizeof(float4);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15))
+    return fail(ZEBRA_ERR_WORKSPACE, "workspace too small (zebra_coverage_workspace_bytes) or misaligned");
+  a.part = static_cast<float4*>(workspace);
+  a.sel = selected_mass;
+  a.spec = special_mass;
+  for (int32_t i = 0; i < n_query_tiles; ++i) a.tiles[i] = query_tiles[i];
+  ZTRY(check_device());
+  return launch_coverage(a, static_cast<cudaStream_t>(stream));
+}
+
+int zebra_affine_residual(const zebra_geom* g, const double* moments, int per_head, const float* A, const float* b,
+                          double* err, void* stream) {
+  ZTRY(check_geom(g));
+  if (per_head != 0 && per_head != 1) return fail(ZEBRA_ERR_INVALID_ARG, "per_head must be 0 or 1");
+  if (!moments || (reinterpret_cast<uintptr_t>(moments) & 7) || !err || (reinterpret_cast<uintptr_t>(err) & 7))
+    return fail(ZEBRA_ERR_INVALID_ARG, "moments and err must be non-null and 8-byte aligned");
+  if (!A || !b || (reinterpret_cast<uintptr_t>(A) & 3) || (reinterpret_cast<uintptr_t>(b) & 3))
+    return fail(ZEBRA_ERR_INVALID_ARG, "A and b must be non-null and 4-byte aligned");
+  ZTRY(check_device());
+  return launch_affine_residual(moments, per_head, g->heads, A, b, err, static_cast<cudaStream_t>(stream));
+}
+
+int32_t zebra_allocate_layers(const double* errors, int32_t n_layers, double linear_fraction, int32_t* is_linear) {
+  if (n_layers < 0 || !(linear_fraction >= 0.0 && linear_fraction <= 1.0)) return -1;
+  if (n_layers > 0 && (!errors || !is_linear)) return -1;
+  const int32_t count = (int32_t)floor(linear_fraction * (double)n_layers + 0.5);
+  std::vector<int32_t> order((size_t)n_layers);
+  for (int32_t i = 0; i < n_layers; ++i) order[(size_t)i] = i;
+  // ascending error, NaN last, equal errors in index order
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t c) {
+    const double ea = errors[a], ec = errors[c];
+    if (std::isnan(ea)) return false;
+    if (std::isnan(ec)) return true;
+    return ea < ec;
+  });
+  for (int32_t i = 0; i < n_layers; ++i) is_linear[i] = 0;
+  for (int32_t r = 0; r < count; ++r) is_linear[order[(size_t)r]] = 1;
+  return count;
+}
+
 int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void* w_qkv, const void* w_o,
                        const float* A, const float* b, double y, float rope_base, float eps, void* x_out,
                        void* workspace, size_t ws_bytes, void* stream) {
@@ -670,6 +753,13 @@ long long zebra_profile_report(char* buf, size_t len) {
     buf[n] = 0;
   }
   return (long long)out.size();
+}
+
+int zebra_debug_inject(int32_t block, uint64_t wait_ns) {
+  ZTRY(check_device());
+  if (set_debug_inject(block, (unsigned long long)wait_ns) != ZEBRA_OK)
+    return fail(ZEBRA_ERR_CUDA, "setting the test hook failed");
+  return ZEBRA_OK;
 }
 
 int zebra_sync_status(void* stream) {

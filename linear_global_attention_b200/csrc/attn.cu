@@ -22,9 +22,8 @@
 //
 // Special-token query rows attend all N keys: split-KV over key-tile ranges,
 // partial (max, sum, unnormalised output) per split, then a combine kernel. In
-// bf16 they run on mma.sync m16n8k16 with fp32 accumulation, 4 warps x 16
-// query rows, K/V blocks double-buffered in shared memory by cp.async with an
-// XOR swizzle on 16-byte chunks so ldmatrix reads are conflict-free.
+// bf16 they run on the tcgen05 kernel (attn_tc.cuh, mode 1); in fp32 on one
+// thread per row.
 #include <math.h>
 
 #include "common.cuh"
@@ -201,7 +200,7 @@ __device__ __forceinline__ void block_src(const AttnArgs& a, int h, int kind, in
 }
 
 // ---------------------------------------------------------------------------
-// bf16 mma.sync path
+// mma.sync helpers (the attention-concentration diagnostic)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -228,219 +227,197 @@ __device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// round a pair to bf16 in place and return it packed: the softmax sum then uses
-// exactly the weights that enter the PV product
-__device__ __forceinline__ uint32_t pack_round(float& lo, float& hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  const float2 f = __bfloat1622float2(v);
-  lo = f.x;
-  hi = f.y;
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // byte offset of (row, 16-byte chunk) in a swizzled 64x64 bf16 tile
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-struct MmaSmem {
-  __nv_bfloat16 q[64 * 64];
-  __nv_bfloat16 k[2][64 * 64];
-  __nv_bfloat16 v[2][64 * 64];
-  float bias[2][64];
-};
-
-// Dense rows of the special-token queries (mma.sync, bf16): CTA = one block of
-// 64 special queries x one head x one key split (blockIdx.z of a.splits); the
-// key range is the split's share of the patch tiles, plus every special key in
-// split 0. Writes unnormalised partial O, row maximum and row sum for
-// special_combine_kernel. (MODE 1 is the only mode: the sparse patch rows run
-// on the tcgen05 kernel.)
-template <int MODE>
-__global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
-  static_assert(MODE == 1, "dense special-token rows only");
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  MmaSmem& sm = *reinterpret_cast<MmaSmem*>(smem_raw);
+// ---------------------------------------------------------------------------
+// attention-concentration diagnostic (page section "Sensitive stages also
+// concentrate their attention"): for each row of a sampled patch query tile,
+// the dense softmax mass (scale 1/sqrt(d), all N keys) that falls on the
+// tokens of the tile's selected key tiles and on the special-token keys.
+// CTA = (sampled tile, head, key split), 4 warps x 16 query rows, mma.sync
+// QK^T over 64-key blocks read straight from the strided K; per row a running
+// maximum and three sums (all keys, selected tiles, special keys) in the same
+// units; coverage_combine_kernel merges the splits in a fixed order.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) coverage_kernel(const __grid_constant__ CoverageArgs a) {
+  __shared__ __align__(128) __nv_bfloat16 qs[64 * 64];
+  __shared__ __align__(128) __nv_bfloat16 ks[2][64 * 64];
+  __shared__ float bias[2][64];
+  __shared__ int kind_sh[2];   // 0 unselected tile, 1 selected tile, 2 special block
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const int t = blockIdx.x;  // special query block
-
-  // query rows -> shared (swizzled)
-  const __nv_bfloat16* qsrc = static_cast<const __nv_bfloat16*>(a.Qs) + ((size_t)h * g.NSp + (size_t)t * 64) * D;
-  for (int i = tid; i < 512; i += 128) {
-    const int r = i >> 3, c = i & 7;
-    cp_async16(smem_u32(sm.q) + swz(r, c), qsrc + r * D + c * 8);
+  const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
+  const int t = a.tiles[i];
+  const uint32_t* mrow = a.mask + ((size_t)h * g.T + t) * g.W;
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q) + (long long)h * a.hs;
+  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
+  const TileShape qt = tile_shape(g, t);
+  const int n_t = qt.rows * qt.cols;
+  for (int e = tid; e < 512; e += 128) {
+    const int r = e >> 3, c = e & 7;
+    if (r < n_t) cp_async16(smem_u32(qs) + swz(r, c), Q + tile_token(g, qt, r) * a.ts + c * 8);
+    else store16_zero(reinterpret_cast<char*>(qs) + swz(r, c));
   }
   cp_async_commit();
-
-  BlockIter it{};
-  it.phase = 0;
-  const int sp = blockIdx.z;
-  it.w = (int)((long long)g.T * sp / a.splits);
-  it.t_end = (int)((long long)g.T * (sp + 1) / a.splits);
-  const bool with_special = sp == 0;
-
-  auto issue = [&](int kind, int id, int buf) {
-    const __nv_bfloat16 *ks, *vs;
-    block_src<__nv_bfloat16>(a, h, kind, id, ks, vs);
-    for (int i = tid; i < 512; i += 128) {
-      const int r = i >> 3, c = i & 7;
-      cp_async16(smem_u32(sm.k[buf]) + swz(r, c), ks + r * D + c * 8);
-      cp_async16(smem_u32(sm.v[buf]) + swz(r, c), vs + r * D + c * 8);
+  const int u0 = (int)((long long)g.T * sp / a.splits), u1 = (int)((long long)g.T * (sp + 1) / a.splits);
+  const int nspec = sp == 0 ? g.NSp / 64 : 0;
+  const int nblk = (u1 - u0) + nspec;
+  // block b: key tile u0 + b, then the special blocks
+  auto issue = [&](int b, int buf) {
+    if (b < u1 - u0) {
+      const int u = u0 + b;
+      const TileShape ks_ = tile_shape(g, u);
+      const int n_u = ks_.rows * ks_.cols;
+      for (int e = tid; e < 512; e += 128) {
+        const int r = e >> 3, c = e & 7;
+        if (r < n_u) cp_async16(smem_u32(ks[buf]) + swz(r, c), K + tile_token(g, ks_, r) * a.ts + c * 8);
+        else store16_zero(reinterpret_cast<char*>(ks[buf]) + swz(r, c));
+      }
+      if (tid < 64) bias[buf][tid] = tid < n_u ? 0.f : -INFINITY;
+      if (tid == 0) kind_sh[buf] = (int)((__ldg(mrow + (u >> 5)) >> (u & 31)) & 1u);
+    } else {
+      const int sb = b - (u1 - u0);
+      for (int e = tid; e < 512; e += 128) {
+        const int r = e >> 3, c = e & 7, si = sb * 64 + r;
+        if (si < g.NS) cp_async16(smem_u32(ks[buf]) + swz(r, c), K + special_token(g, si) * a.ts + c * 8);
+        else store16_zero(reinterpret_cast<char*>(ks[buf]) + swz(r, c));
+      }
+      if (tid < 64) bias[buf][tid] = sb * 64 + tid < g.NS ? 0.f : -INFINITY;
+      if (tid == 0) kind_sh[buf] = 2;
     }
-    if (tid < 64) sm.bias[buf][tid] = block_bias(a, nullptr, t, kind, id, tid);   // kinds 0 and 2 only
   };
-
-  int kind = 0, id = 0, nv = 0;
-  long long keys = 0;  // visible keys per query row, summed over blocks
-  bool have = next_block_dense(it, g, with_special, kind, id, nv);
-  if (have) {
-    issue(kind, id, 0);
-    keys += nv;
-  }
+  if (nblk > 0) issue(0, 0);
   cp_async_commit();
-
-  const float sc = LOG2E * 0.125f;  // log2(e) / sqrt(64)
-  float o[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  uint32_t qf[4][4];
-  bool qloaded = false;
+  const float sc = LOG2E * 0.125f;
   const int g4 = lane >> 2, q4 = lane & 3;
-
-  int buf = 0;
-  while (have) {
-    int nkind = 0, nid = 0, nnv = 0;
-    const bool nhave = next_block_dense(it, g, with_special, nkind, nid, nnv);
-    if (nhave) {
-      issue(nkind, nid, buf ^ 1);
-      keys += nnv;
-    }
+  float m[2] = {-INFINITY, -INFINITY}, z[2] = {0.f, 0.f}, ssel[2] = {0.f, 0.f}, sspec[2] = {0.f, 0.f};
+  uint32_t qf[4][4];
+  for (int b = 0; b < nblk; ++b) {
+    const int buf = b & 1;
+    if (b + 1 < nblk) issue(b + 1, buf ^ 1);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
-    if (!qloaded) {
+    if (b == 0) {
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
+      for (int kk = 0; kk < 4; ++kk) {
         const int mi = lane >> 3, ri = lane & 7;
-        const int row = warp * 16 + (mi & 1) * 8 + ri;
-        ldsm_x4(smem_u32(sm.q) + swz(row, 2 * ks + (mi >> 1)), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+        ldsm_x4(smem_u32(qs) + swz(warp * 16 + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1)), qf[kk][0], qf[kk][1],
+                qf[kk][2], qf[kk][3]);
       }
-      qloaded = true;
     }
-    // S = Q K^T
-    float s[8][4];
+    float sv[8][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-    const uint32_t kb = smem_u32(sm.k[buf]);
+    for (int j = 0; j < 8; ++j) sv[j][0] = sv[j][1] = sv[j][2] = sv[j][3] = 0.f;
+    const uint32_t kb = smem_u32(ks[buf]);
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
+    for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         const int mi = lane >> 3, ri = lane & 7;
-        const int row = np * 16 + (mi >> 1) * 8 + ri;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + swz(row, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-        mma_bf16(s[2 * np], qf[ks], b0, b1);
-        mma_bf16(s[2 * np + 1], qf[ks], b2, b3);
+        ldsm_x4(kb + swz(np * 16 + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+        mma_bf16(sv[2 * np], qf[kk], b0, b1);
+        mma_bf16(sv[2 * np + 1], qf[kk], b2, b3);
       }
     }
-    // online softmax (rows g4 and g4 + 8 of this warp)
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float b0v = sm.bias[buf][8 * j + 2 * q4], b1v = sm.bias[buf][8 * j + 2 * q4 + 1];
-      s[j][0] = fmaf(s[j][0], sc, b0v);
-      s[j][1] = fmaf(s[j][1], sc, b1v);
-      s[j][2] = fmaf(s[j][2], sc, b0v);
-      s[j][3] = fmaf(s[j][3], sc, b1v);
-      mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
-      mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-    const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float al0 = fast_exp2(m0 - base0), al1 = fast_exp2(m1 - base1);
-    m0 = mn0;
-    m1 = mn1;
-    float rs0 = 0.f, rs1 = 0.f;
-    uint32_t pk[8][2];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      s[j][0] = fast_exp2(s[j][0] - base0);
-      s[j][1] = fast_exp2(s[j][1] - base0);
-      s[j][2] = fast_exp2(s[j][2] - base1);
-      s[j][3] = fast_exp2(s[j][3] - base1);
-      pk[j][0] = pack_round(s[j][0], s[j][1]);
-      pk[j][1] = pack_round(s[j][2], s[j][3]);
-      rs0 += s[j][0] + s[j][1];
-      rs1 += s[j][2] + s[j][3];
-    }
-    l0 = l0 * al0 + rs0;
-    l1 = l1 * al1 + rs1;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      o[j][0] *= al0; o[j][1] *= al0;
-      o[j][2] *= al1; o[j][3] *= al1;
-    }
-    // O += P V
-    const uint32_t vb = smem_u32(sm.v[buf]);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pa[4];
-      pa[0] = pk[2 * kk][0];
-      pa[1] = pk[2 * kk][1];
-      pa[2] = pk[2 * kk + 1][0];
-      pa[3] = pk[2 * kk + 1][1];
-#pragma unroll
-      for (int dp = 0; dp < 4; ++dp) {
-        const int mi = lane >> 3, ri = lane & 7;
-        const int row = kk * 16 + (mi & 1) * 8 + ri;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + swz(row, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-        mma_bf16(o[2 * dp], pa, b0, b1);
-        mma_bf16(o[2 * dp + 1], pa, b2, b3);
-      }
-    }
-    __syncthreads();
-    buf ^= 1;
-    have = nhave;
-    kind = nkind;
-    id = nid;
-  }
-  cp_async_wait<0>();
-  if (!qloaded) __syncthreads();
-  if (tid == 0) {
-    const long long rows = min(64, g.NS - t * 64);
-    atomicAdd(&g_logits[1], (unsigned long long)(rows * keys));
-  }
-
-  const int r0 = warp * 16 + g4, r1 = r0 + 8;
-  {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const int kind = kind_sh[buf];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      const int r = half ? r1 : r0;
-      const int qi = t * 64 + r;  // special query index
-      const size_t row = ((size_t)sp * g.H + h) * g.NSp + qi;
-      float* po = a.part_o + row * D;
+      float mx = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int c = 8 * j + 2 * q4;
-        *reinterpret_cast<float2*>(po + c) = make_float2(o[j][half * 2], o[j][half * 2 + 1]);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float& x = sv[j][2 * half + e];
+          x = fmaf(x, sc, bias[buf][8 * j + 2 * q4 + e]);
+          mx = fmaxf(mx, x);
+        }
       }
-      if (q4 == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(half ? m1 : m0, half ? l1 : l0);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mn = fmaxf(m[half], mx);
+      const float base = mn == -INFINITY ? 0.f : mn;
+      const float al = exp2f(m[half] - base);
+      float ps = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ps += exp2f(sv[j][2 * half] - base) + exp2f(sv[j][2 * half + 1] - base);
+      m[half] = mn;
+      z[half] = z[half] * al + ps;
+      ssel[half] = ssel[half] * al + (kind == 1 ? ps : 0.f);
+      sspec[half] = sspec[half] * al + (kind == 2 ? ps : 0.f);
+    }
+    __syncthreads();   // the buffer is reloaded by the next issue
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      z[half] += __shfl_xor_sync(0xffffffffu, z[half], o);
+      ssel[half] += __shfl_xor_sync(0xffffffffu, ssel[half], o);
+      sspec[half] += __shfl_xor_sync(0xffffffffu, sspec[half], o);
+    }
+    if (q4 == 0) {
+      const int r = warp * 16 + g4 + 8 * half;
+      a.part[(((size_t)i * g.H + h) * a.splits + sp) * 64 + r] = make_float4(m[half], z[half], ssel[half], sspec[half]);
     }
   }
+}
+
+// merge the splits of every (sampled tile, head, row): fixed order
+__global__ void coverage_combine_kernel(const __grid_constant__ CoverageArgs a) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)a.n * a.g.H * 64) return;
+  const int r = (int)(e & 63);
+  const long long ih = e >> 6;   // i * H + h
+  const int i = (int)(ih / a.g.H);
+  const TileShape qt = tile_shape(a.g, a.tiles[i]);
+  if (r >= qt.rows * qt.cols) {
+    a.sel[e] = 0.f;
+    a.spec[e] = 0.f;
+    return;
+  }
+  const float4* p = a.part + ih * a.splits * 64 + r;
+  float mstar = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) mstar = fmaxf(mstar, p[s * 64].x);
+  float z = 0.f, ss = 0.f, sp = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const float4 v = p[s * 64];
+    if (v.x == -INFINITY) continue;
+    const float w = exp2f(v.x - mstar);
+    z += w * v.y;
+    ss += w * v.z;
+    sp += w * v.w;
+  }
+  a.sel[e] = ss / z;
+  a.spec[e] = sp / z;
+}
+
+int coverage_splits(const Geo& g, int n) {
+  long long s = (4LL * 148 + (long long)n * g.H - 1) / ((long long)n * g.H);
+  if (s > 64) s = 64;
+  if (s > g.T) s = g.T;
+  return (int)(s < 1 ? 1 : s);
+}
+
+int launch_coverage(const CoverageArgs& a, cudaStream_t st) {
+  {
+    ProfScope prof("coverage", st);
+    coverage_kernel<<<dim3(a.n, a.g.H, a.splits), 128, 0, st>>>(a);
+  }
+  count_launch();
+  if (int rc = check_launch("coverage_kernel")) return rc;
+  const long long threads = (long long)a.n * a.g.H * 64;
+  {
+    ProfScope prof("coverage_combine", st);
+    coverage_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(a);
+  }
+  count_launch();
+  return check_launch("coverage_combine_kernel");
 }
 
 // ---------------------------------------------------------------------------
@@ -600,20 +577,17 @@ int launch_sparse_attn<float>(const AttnArgs& a, cudaStream_t st) {
 template <typename T>
 int launch_special_rows(const AttnArgs& a, cudaStream_t st) {
   if (a.g.NS == 0) return ZEBRA_OK;
-  dim3 grid(a.g.NSp / 64, a.g.H, a.splits);
-  {
-  ProfScope prof("attn_special_rows", st);
   if (sizeof(T) == 2) {
-    const size_t smem = sizeof(MmaSmem);
-    cudaFuncSetAttribute(attn_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_mma_kernel<1><<<grid, 128, smem, st>>>(a);
+    if (int rc = launch_special_rows_tc(a, st)) return rc;
   } else {
-    attn_simt_kernel<1><<<grid, 64, 0, st>>>(a);
+    dim3 grid(a.g.NSp / 64, a.g.H, a.splits);
+    {
+      ProfScope prof("attn_special_rows_f32", st);
+      attn_simt_kernel<1><<<grid, 64, 0, st>>>(a);
+    }
+    count_launch();
+    if (int rc = check_launch("attn_simt_kernel<special rows>")) return rc;
   }
-  }
-  count_launch();
-  int rc = check_launch("attn_kernel<special rows>");
-  if (rc) return rc;
   const long long threads = (long long)a.g.NS * a.g.H * 32;
   ProfScope prof("special_combine", st);
   special_combine_kernel<T><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(a);

@@ -48,6 +48,20 @@
 namespace zebra {
 
 __device__ int g_status;   // sticky device status word (0 = ok)
+// Error-path test hook (zebra_debug_inject): the limit of every bounded wait of
+// the sparse kernel, and the block before which its producer stops issuing
+// copies (-1 = never), so that a consumer's wait runs out.
+__device__ unsigned long long g_wait_ns = 2000000000ull;
+__device__ int g_inject_block = -1;
+
+int set_debug_inject(int block, unsigned long long wait_ns) {
+  const int b = block < 0 ? -1 : block;
+  const unsigned long long w = wait_ns ? wait_ns : 2000000000ull;
+  if (cudaMemcpyToSymbol(g_inject_block, &b, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_wait_ns, &w, sizeof(w)) != cudaSuccess)
+    return ZEBRA_ERR_CUDA;
+  return ZEBRA_OK;
+}
 
 int read_and_clear_status(int* out) {
   int v = 0;
@@ -78,11 +92,24 @@ constexpr int NSBUF = ZEBRA_TC_NSBUF;     // TMEM score buffers (QK^T lookahead)
 #endif
 constexpr int PBUF = ZEBRA_TC_PBUF;       // shared-memory P buffers (softmax lead over PV)
 constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
+#ifndef ZEBRA_TC_RSUM_MMA
+#define ZEBRA_TC_RSUM_MMA 0
+#endif
+// 1: row sums as P x ones MMAs (N = 16) on the tensor cores; 0: in the softmax
+// warps' registers (fp32 sums of the exponentials)
+constexpr bool RSUM_MMA = ZEBRA_TC_RSUM_MMA != 0;
+#ifndef ZEBRA_TC_EMU
+#define ZEBRA_TC_EMU 0
+#endif
+// of the 8 column groups a softmax thread holds per block, how many take
+// their exponentials from the FMA-pipe polynomial (exp2_poly2) instead of the
+// MUFU ex2 unit
+constexpr int EMU = ZEBRA_TC_EMU;
+static_assert(EMU >= 0 && EMU <= 8, "EMU counts column groups");
 constexpr int THREADS = 192;
 constexpr uint32_t COL_O = 64 * NSBUF;   // O after the score buffers
 constexpr uint32_t TMEM_COLS = COL_O + 64 <= 128 ? 128 : 256;
 constexpr uint32_t LANE_L = 16u << 16;   // TMEM lane offset of the row-sum accumulator L
-constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
 static_assert(NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
 
@@ -91,7 +118,7 @@ struct __align__(1024) Smem {
   __nv_bfloat16 k[STAGES][64 * 64];
   __nv_bfloat16 v[STAGES][64 * 64];
   __nv_bfloat16 p[PBUF][64 * 64];
-  __nv_bfloat16 ones[16 * 64];  // B operand of the row-sum MMA (N = 16, K = 64), all 1.0
+  __nv_bfloat16 ones[RSUM_MMA ? 16 * 64 : 8];  // B operand of the row-sum MMA (N = 16, K = 64), all 1.0
   float bias[STAGES][64];       // logit bias row of the block in each stage (log2 units)
   int all_zero[STAGES];         // 1 when every bias of the stage is 0 (a complete kept tile)
   uint64_t q_full;
@@ -119,9 +146,9 @@ static_assert(SMEM_BYTES * CTAS_PER_SM <= SMEM_CAP, "shared memory layout");
 static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "TMEM columns");
 
 struct alignas(64) Params {
-  CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs;
+  CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs, tqs;
   AttnArgs a;
-  int item0;   // first work item (h * T + t) of this launch; CTA b takes item0 + b
+  int item0;   // first work item of this launch; CTA b takes item0 + b
 };
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -182,11 +209,29 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, volati
   }
 }
 
-// Wait for the phase of `parity` to complete; true when it did.
+// Wait for the phase of `parity` to complete; true when it did. `limit_ns` is
+// the kernel's wait limit (g_wait_ns, read once at kernel start).
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          unsigned long long limit_ns = WAIT_NS) {
+                                          unsigned long long limit_ns) {
   if (mbar_try(b, parity)) return true;
   return mbar_wait_slow(b, parity, abort_flag, limit_ns);
+}
+
+// Drain wait after an abort: waits for the phase whatever the abort flag says
+// (copies or MMAs still in flight must land before the CTA frees its shared
+// memory and TMEM), and gives up after `limit_ns`.
+__device__ __noinline__ bool mbar_drain(uint64_t* b, uint32_t parity, unsigned long long limit_ns) {
+  const unsigned long long t0 = gtime();
+  while (!mbar_try(b, parity))
+    if (gtime() - t0 > limit_ns) return false;
+  return true;
+}
+__device__ __noinline__ bool mbar_drain_warp(uint64_t* b, uint32_t parity, unsigned long long limit_ns) {
+  const unsigned long long t0 = gtime();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
+    if (__any_sync(0xffffffffu, gtime() - t0 > limit_ns)) return false;
+  }
 }
 
 // Whole-warp form (all 32 lanes call it): the result is the same in every lane,
@@ -208,7 +253,7 @@ __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* b, uint32_t parity, v
   }
 }
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                               unsigned long long limit_ns = WAIT_NS) {
+                                               unsigned long long limit_ns) {
   if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
   return mbar_wait_warp_slow(b, parity, abort_flag, limit_ns);
 }
@@ -297,6 +342,23 @@ __device__ __forceinline__ void mma_pv_elect(uint32_t d_o, uint32_t d_l, uint64_
       "r"(saddr(bar0)), "r"(saddr(bar1))
       : "memory");
 }
+// O += P V alone (row sums kept in the softmax warps' registers), then commits
+// to `bar0` and `bar1`.
+__device__ __forceinline__ void mma_pv_only_elect(uint32_t d_o, uint64_t p, uint64_t v, uint32_t id_pv, uint32_t acc,
+                                                  uint64_t* bar0, uint64_t* bar1) {
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, %10, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n}\n"
+      ::"r"(d_o), "l"(p), "l"(p + 2), "l"(p + 4), "l"(p + 6), "l"(v), "l"(v + 128), "l"(v + 256), "l"(v + 384),
+      "r"(id_pv), "r"(acc), "r"(saddr(bar0)), "r"(saddr(bar1))
+      : "memory");
+}
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;
   asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
@@ -371,6 +433,29 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// 2^x for a pair (x <= 8) on the FMA pipe: clamp to >= -126, x = j + f with
+// j = round-to-nearest(x) (adding 1.5 * 2^23 leaves j in the low mantissa
+// bits), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial minimax in relative
+// error on that interval (coefficients from linear_global_attention_b200/
+// exp2_fit.py, max relative error 7.5e-5); 2^j enters by an integer add to the
+// exponent field.
+constexpr float EXP2_C0 = 0.9999280571937561f, EXP2_C1 = 0.6932608485221863f, EXP2_C2 = 0.24261115491390228f,
+                EXP2_C3 = 0.05517221987247467f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 one = make_float2(1.f, 1.f), mone = make_float2(-1.f, -1.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f), nmagic = make_float2(-12582912.f, -12582912.f);
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = ffma2(x, one, magic);      // 1.5 * 2^23 + j
+  const float2 j = ffma2(t, one, nmagic);     // j (exact)
+  const float2 f = ffma2(j, mone, x);         // x - j (exact)
+  float2 p = ffma2(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  p = ffma2(p, f, make_float2(EXP2_C1, EXP2_C1));
+  p = ffma2(p, f, make_float2(EXP2_C0, EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // maximum of one row's 16 values in the 16x256b fragment (sv[4j + O], sv[4j + O + 1], j < 8),
 // as a tree of 3-input maxima
 template <int O>
@@ -396,6 +481,13 @@ __device__ __forceinline__ int block_row(const Geo& g, int h, int kind, int id) 
   return h * g.NSp + id * 64;
 }
 
+// MODE 0: patch query rows of the tile-sparse stage; work item h * T + t.
+// MODE 1: dense special-token query rows: work item (h * splits + sp) * NQB + qb
+// is query block qb (64 special queries, packed) of head h against key split
+// sp (the key tiles [T sp / splits, T (sp + 1) / splits), plus every special
+// key in split 0); it writes the split's unnormalised output, row maximum and
+// row sum for special_combine_kernel.
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -403,9 +495,22 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   const Geo& g = a.g;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = P.item0 + (int)blockIdx.x;
-  const int h = item / g.T, t = item - h * g.T;
-  const uint32_t* mrow = a.mask + ((size_t)h * g.T + t) * g.W;
+  int h, t = 0, qb = 0, sp = 0, u0 = 0, u1 = 0;
+  if constexpr (MODE == 0) {
+    h = item / g.T;
+    t = item - h * g.T;
+  } else {
+    const int nqb = g.NSp / 64;
+    qb = item % nqb;
+    const int hsp = item / nqb;
+    sp = hsp % a.splits;
+    h = hsp / a.splits;
+    u0 = (int)((long long)g.T * sp / a.splits);
+    u1 = (int)((long long)g.T * (sp + 1) / a.splits);
+  }
+  const uint32_t* mrow = MODE == 0 ? a.mask + ((size_t)h * g.T + t) * g.W : nullptr;
   volatile int* abort_flag = &sm.abort;
+  const unsigned long long wl = *(volatile unsigned long long*)&g_wait_ns;   // limit of every wait
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
@@ -429,20 +534,25 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the all-ones operand of the row-sum MMA (read by the tensor cores: async proxy)
-  for (int i = tid; i < 16 * 64 / 2; i += THREADS) reinterpret_cast<uint32_t*>(sm.ones)[i] = 0x3F803F80u;
+  if (RSUM_MMA)
+    for (int i = tid; i < 16 * 64 / 2; i += THREADS) reinterpret_cast<uint32_t*>(sm.ones)[i] = 0x3F803F80u;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
-    // pre-pass, lane-parallel: the number of blocks the walk below will
-    // produce (kept tiles, landmark blocks with a visible landmark, special
-    // blocks)
-    int n = 0;
-    for (int w = lane; w < g.W; w += 32) n += __popc(mask_word(mrow, w, g.T));
-    for (int lb = lane; lb < g.Tpad / 64; lb += 32) {
-      int nvis;
-      n += lmk_visible(mrow, g, t, lb, nvis) != 0u ? 1 : 0;
+    if constexpr (MODE == 0) {
+      // pre-pass, lane-parallel: the number of blocks the walk below will
+      // produce (kept tiles, landmark blocks with a visible landmark, special
+      // blocks)
+      int n = 0;
+      for (int w = lane; w < g.W; w += 32) n += __popc(mask_word(mrow, w, g.T));
+      for (int lb = lane; lb < g.Tpad / 64; lb += 32) {
+        int nvis;
+        n += lmk_visible(mrow, g, t, lb, nvis) != 0u ? 1 : 0;
+      }
+      n = __reduce_add_sync(0xffffffffu, n);
+      if (lane == 0) sm.nblocks = n + g.NSp / 64;
+    } else {
+      if (lane == 0) sm.nblocks = (u1 - u0) + (sp == 0 ? g.NSp / 64 : 0);
     }
-    n = __reduce_add_sync(0xffffffffu, n);
-    if (lane == 0) sm.nblocks = n + g.NSp / 64;
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sm.tmem_base)),
                  "r"(TMEM_COLS));
@@ -454,29 +564,42 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   const uint32_t tmem = sm.tmem_base;
   const int nb = sm.nblocks;
 
-  const bool own_kept = (__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u;
+  // MODE 0: the query tile's shape and whether it keeps its own tile;
+  // MODE 1: n_t = the valid special queries of the block
+  const bool own_kept = MODE == 0 ? ((__ldg(mrow + (t >> 5)) >> (t & 31)) & 1u) != 0 : true;
   const TileShape ts = tile_shape(g, t);
-  const int n_t = ts.rows * ts.cols;
+  const int n_t = MODE == 0 ? ts.rows * ts.cols : min(64, g.NS - qb * 64);
 
   if (warp == 0) {
     // ---------------- producer (whole warp; one elected lane issues) ----------------
-    int issued = 0;
-    tma_load_2d_elect(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+    int issued = 0, nk = 0;   // blocks whose V (and K) copies were issued; K copies issued
+    const int inject = *(volatile int*)&g_inject_block;   // error-path test hook (-1: off)
     BlockIter it{};
-    iter_init(it, mrow, g);
+    if constexpr (MODE == 0) {
+      tma_load_2d_elect(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
+      iter_init(it, mrow, g);
+    } else {
+      tma_load_2d_elect(sm.q, &P.tqs, 0, h * g.NSp + qb * 64, &sm.q_full);
+      it.w = u0;
+      it.t_end = u1;
+    }
     int kind, id, nv;
     long long keys = 0;   // visible keys per query row (for the logit counter)
     bool ok = true;
-    while (ok && next_block_sparse(it, g, mrow, t, true, kind, id, nv)) {
+    while (ok && (MODE == 0 ? next_block_sparse(it, g, mrow, t, true, kind, id, nv)
+                            : next_block_dense(it, g, sp == 0, kind, id, nv))) {
+      // test hook: stop before this block, so the MMA warp's wait for its K tile runs out
+      if (issued == inject) break;
       keys += nv;
       const int s = issued % STAGES;
       const uint32_t par = ((issued / STAGES) - 1) & 1;
       const int row = block_row(g, h, kind, id);
-      if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag);
+      if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag, wl);
       if (!ok) break;
       tma_load_2d_elect(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
+      ++nk;
       // the V tile and the bias row of this stage are free once PV of block issued - STAGES is done
-      if (issued >= STAGES) ok = mbar_wait_warp(&sm.v_empty[s], par, abort_flag);
+      if (issued >= STAGES) ok = mbar_wait_warp(&sm.v_empty[s], par, abort_flag, wl);
       if (!ok) break;
       tma_load_2d_elect(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
       // bias row: two columns per lane
@@ -500,36 +623,38 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     }
     if (lane == 0 && ok && issued == nb) {
       const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);   // the own-tile extras of the epilogue
-      atomicAdd(&g_logits[0], (unsigned long long)((long long)n_t * (keys + extra)));
+      atomicAdd(&g_logits[MODE], (unsigned long long)((long long)n_t * (keys + extra)));
     }
-    if (lane == 0 && *abort_flag) {
-      // let the copies already in flight land before the CTA goes away
-      mbar_wait(&sm.q_full, 0, abort_flag, DRAIN_NS);
-      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i) {
-        mbar_wait(&sm.k_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
-        mbar_wait(&sm.v_full[i % STAGES], (i / STAGES) & 1, abort_flag, DRAIN_NS);
-      }
+    if (lane == 0 && (issued < nb || *abort_flag)) {
+      // stopped early: let the copies already in flight land before the CTA
+      // frees its shared memory (the last STAGES copies into each ring are the
+      // only ones whose landing nobody may have waited for)
+      mbar_drain(&sm.q_full, 0, DRAIN_NS);
+      for (int i = nk > STAGES ? nk - STAGES : 0; i < nk; ++i)
+        mbar_drain(&sm.k_full[i % STAGES], (i / STAGES) & 1, DRAIN_NS);
+      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+        mbar_drain(&sm.v_full[i % STAGES], (i / STAGES) & 1, DRAIN_NS);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
     const uint32_t id_qk = idesc(false), id_pv = idesc(true), id_sum = idesc(false, 16);
     const uint64_t dq = desc_k(saddr(sm.q));
     const uint64_t d1 = desc_k(saddr(sm.ones));
-    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
+    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag, wl);
     int qk = 0;
     for (int j = 0; ok && j < nb; ++j) {
       // S = Q K^T up to NSBUF blocks ahead of this PV (a score buffer is
       // reusable as soon as the softmax has loaded it)
       while (qk < nb && qk <= j + NSBUF) {
         const int s = qk % STAGES, b = qk % NSBUF;
-        ok = mbar_wait_warp(&sm.k_full[s], (qk / STAGES) & 1, abort_flag);
-        if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag);
+        ok = mbar_wait_warp(&sm.k_full[s], (qk / STAGES) & 1, abort_flag, wl);
+        if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag, wl);
         if (!ok) break;
         fence_after();
         mma_qk_elect(tmem + 64u * b, dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
         // forward the stage's bias row to the softmax through s_full: this
         // warp acquires it here and releases it with one arrival
-        ok = mbar_wait_warp(&sm.b_full[s], (qk / STAGES) & 1, abort_flag);
+        ok = mbar_wait_warp(&sm.b_full[s], (qk / STAGES) & 1, abort_flag, wl);
         if (!ok) break;
         if (lane == 0) mbar_arrive(&sm.s_full[b]);
         __syncwarp();
@@ -538,17 +663,21 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (!ok) break;
       // O += P V and L += P ones of block j
       const int s = j % STAGES, pb = j % PBUF;
-      ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag);
-      if (ok) ok = mbar_wait_warp(&sm.p_full[pb], (j / PBUF) & 1, abort_flag);
+      ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag, wl);
+      if (ok) ok = mbar_wait_warp(&sm.p_full[pb], (j / PBUF) & 1, abort_flag, wl);
       if (!ok) break;
       fence_after();
-      mma_pv_elect(tmem + COL_O, tmem + LANE_L + COL_O, desc_k(saddr(sm.p[pb])), desc_mn(saddr(sm.v[s])), d1, id_pv,
-                   id_sum, j > 0 ? 1u : 0u, &sm.v_empty[s], &sm.pv_done[pb]);
+      if (RSUM_MMA)
+        mma_pv_elect(tmem + COL_O, tmem + LANE_L + COL_O, desc_k(saddr(sm.p[pb])), desc_mn(saddr(sm.v[s])), d1,
+                     id_pv, id_sum, j > 0 ? 1u : 0u, &sm.v_empty[s], &sm.pv_done[pb]);
+      else
+        mma_pv_only_elect(tmem + COL_O, desc_k(saddr(sm.p[pb])), desc_mn(saddr(sm.v[s])), id_pv, j > 0 ? 1u : 0u,
+                          &sm.v_empty[s], &sm.pv_done[pb]);
     }
     // drain: every MMA this warp issued completes before TMEM is freed
     if (elect_one()) mma_commit(&sm.drain);
     __syncwarp();
-    mbar_wait_warp(&sm.drain, 0, abort_flag, *abort_flag ? DRAIN_NS : WAIT_NS);
+    mbar_drain_warp(&sm.drain, 0, *abort_flag ? DRAIN_NS : wl);
   } else {
     // ---------------- softmax warpgroup ----------------
     const int rb = warp & 3;                  // TMEM lane quarter this warp may access
@@ -558,6 +687,10 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     const float2 sc2 = make_float2(sc, sc);
     const float NEG = -INFINITY;
     float m0 = NEG, m1 = NEG;
+    // this thread's share of the row sums (its 16 columns of rows r0 and r1),
+    // in the units of the running maxima m0, m1 (register row sums only)
+    float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+    const float2 one2 = make_float2(1.f, 1.f);
     const int r0 = 16 * rb + g4, r1 = r0 + 8;  // query rows of this thread
     // stmatrix row address in P buffer 0: matrix mi = lane >> 3 of store jj
     // covers rows 16 rb + 8 (mi & 1) .. + 7 and 16-byte chunk 2 jj + (mi >> 1),
@@ -572,7 +705,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int s = i % STAGES, b = i % NSBUF, pb = i % PBUF;
-      if (!mbar_wait_warp(&sm.s_full[b], (i / NSBUF) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&sm.s_full[b], (i / NSBUF) & 1, abort_flag, wl)) { ok = false; break; }
       fence_after();
       float sv[32];
       tmem_ld64(tmem + lane_off + 64u * b, sv);
@@ -615,18 +748,36 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       const float ka = nobias ? sc : 1.f;
       const float2 ka2 = make_float2(ka, ka);
       const float2 nb0 = make_float2(-base0, -base0), nb1 = make_float2(-base1, -base1);
+      if (!RSUM_MMA) {
+        ls0.x *= al0;
+        ls0.y *= al0;
+        ls1.x *= al1;
+        ls1.y *= al1;
+      }
       uint32_t pk[8][2];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float2 e0 = ffma2(make_float2(sv[4 * j + 0], sv[4 * j + 1]), ka2, nb0);
         const float2 e1 = ffma2(make_float2(sv[4 * j + 2], sv[4 * j + 3]), ka2, nb1);
-        pk[j][0] = pack_bf16(fast_exp2(e0.x), fast_exp2(e0.y));
-        pk[j][1] = pack_bf16(fast_exp2(e1.x), fast_exp2(e1.y));
+        float2 p0, p1;
+        if (j >= 8 - EMU) {
+          p0 = exp2_poly2(e0);
+          p1 = exp2_poly2(e1);
+        } else {
+          p0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
+          p1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
+        }
+        if (!RSUM_MMA) {
+          ls0 = ffma2(p0, one2, ls0);
+          ls1 = ffma2(p1, one2, ls1);
+        }
+        pk[j][0] = pack_bf16(p0.x, p0.y);
+        pk[j][1] = pack_bf16(p1.x, p1.y);
       }
       m0 = mn0;
       m1 = mn1;
       // P buffer pb is free once PV of block i-PBUF has completed
-      if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
+      if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag, wl)) { ok = false; break; }
       const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
@@ -636,7 +787,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       // rescale O and L (TMEM) when any row of this warp moved its maximum
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
-        if (!mbar_wait_warp(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag, wl)) { ok = false; break; }
         fence_after();
         float o[32];
         tmem_ld64(tmem + lane_off + COL_O, o);
@@ -648,35 +799,59 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           o[4 * j + 3] *= al1;
         }
         tmem_st64(tmem + lane_off + COL_O, o);
-        float lv[4];
-        tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
-        lv[0] *= al0;
-        lv[1] *= al0;
-        lv[2] *= al1;
-        lv[3] *= al1;
-        tmem_st8(tmem + lane_off + LANE_L + COL_O, lv);
+        if (RSUM_MMA) {
+          float lv[4];
+          tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
+          lv[0] *= al0;
+          lv[1] *= al0;
+          lv[2] *= al1;
+          lv[3] *= al1;
+          tmem_st8(tmem + lane_off + LANE_L + COL_O, lv);
+        }
       }
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
     // ---------------- epilogue ----------------
-    if (ok && nb >= 1 && !mbar_wait_warp(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag)) ok = false;
+    if (ok && nb >= 1 && !mbar_wait_warp(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag, wl)) ok = false;
     if (ok) {
       fence_after();
       float o[32];
       float l0 = 0.f, l1 = 0.f;   // row sums (every column of L holds the row's sum)
       if (nb >= 1) {
         tmem_ld64(tmem + lane_off + COL_O, o);
-        float lv[4];
-        tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
-        l0 = lv[0];
-        l1 = lv[2];
+        if (RSUM_MMA) {
+          float lv[4];
+          tmem_ld8(tmem + lane_off + LANE_L + COL_O, lv);
+          l0 = lv[0];
+          l1 = lv[2];
+        } else {
+          // the four threads of a quad hold the 64 columns of rows r0 and r1
+          l0 = ls0.x + ls0.y;
+          l1 = ls1.x + ls1.y;
+          l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+          l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        }
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
       }
-      if (!own_kept) {
+      if constexpr (MODE == 1) {
+        // split partials: unnormalised output, row maximum (log2 units) and row sum
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = half ? r1 : r0;
+          const size_t row = ((size_t)sp * g.H + h) * g.NSp + (size_t)qb * 64 + r;
+          float* po = a.part_o + row * D;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float2*>(po + 8 * j + 2 * q4) = make_float2(o[4 * j + half * 2], o[4 * j + half * 2 + 1]);
+          if (q4 == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(half ? m1 : m0, half ? l1 : l0);
+        }
+      } else if (!own_kept) {
         // exact self key + landmark of the other n_t - 1 tokens of the own tile
         const size_t tb = ((size_t)h * g.T + t) * TOK * D;
         const __nv_bfloat16* Qp = static_cast<const __nv_bfloat16*>(a.Qp) + tb;
@@ -729,7 +904,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       }
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2 && MODE == 0; ++half) {
         const int r = half ? r1 : r0;
         if (r >= n_t) continue;
         const float il = 1.0f / (half ? l1 : l0);
@@ -781,31 +956,35 @@ static bool make_map(CUtensorMap* m, const void* base, unsigned long long rows) 
   return r == CUDA_SUCCESS;
 }
 
-int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) {
+// Launches the tcgen05 kernel for every work item of `mode` (0: patch rows of
+// the sparse stage, one per (head, query tile); 1: special-token rows, one per
+// (head, key split, query block)).
+static int launch_tc(const AttnArgs& a, int mode, cudaStream_t st) {
   const Geo& g = a.g;
-  if (g.T == 0) return ZEBRA_OK;
+  const long long items = mode == 0 ? (long long)g.T * g.H : (long long)(g.NSp / 64) * g.H * a.splits;
+  if (items == 0 || g.T == 0) return ZEBRA_OK;
   tc::Params p;
   p.a = a;
   const unsigned long long tile_rows = (unsigned long long)g.H * g.T * 64;
+  const unsigned long long spec_rows = (unsigned long long)g.H * g.NSp;
   bool ok = make_map(&p.tq, a.Qp, tile_rows) && make_map(&p.tk, a.Kp, tile_rows) && make_map(&p.tv, a.Vp, tile_rows) &&
             make_map(&p.tkl, a.Kl, (unsigned long long)g.H * g.Tpad) &&
-            make_map(&p.tvl, a.Vl, (unsigned long long)g.H * g.Tpad) &&
-            make_map(&p.tks, a.Ks, (unsigned long long)g.H * g.NSp) &&
-            make_map(&p.tvs, a.Vs, (unsigned long long)g.H * g.NSp);
+            make_map(&p.tvl, a.Vl, (unsigned long long)g.H * g.Tpad) && make_map(&p.tks, a.Ks, spec_rows) &&
+            make_map(&p.tvs, a.Vs, spec_rows) && make_map(&p.tqs, a.Qs, spec_rows);
   if (!ok) {
     set_error("cuTensorMapEncodeTiled failed");
     return ZEBRA_ERR_CUDA;
   }
-  cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
-  // Work items (h, t) go out in launches of one resident wave each. All CTAs
-  // of a launch start together and walk their kept tiles in ascending order at
+  auto kern = mode == 0 ? tc::attn_tc_kernel<0> : tc::attn_tc_kernel<1>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
+  // Work items go out in launches of one resident wave each. All CTAs of a
+  // launch start together and walk their key blocks in ascending order at
   // about the same rate, so at any moment they read K/V tiles from a narrow
   // window of tile indices that stays in L2. In one launch of all items the
   // CTAs of later waves start whenever a slot frees up, their positions spread
-  // over the whole key range, and most K/V reads go to DRAM (at 1,024 views x
-  // 16 heads: 25% slower, the extra DRAM power pulling the clock down under
-  // the board's power limit).
-  const long long items = (long long)g.T * g.H;
+  // over the whole key range, and most K/V reads go to DRAM (sparse rows at
+  // 1,024 views x 16 heads: 25% slower, the extra DRAM power pulling the clock
+  // down under the board's power limit).
   long long wave = items;
   {
     // the kernel is built for CTAS_PER_SM resident CTAs per SM (registers,
@@ -816,16 +995,19 @@ int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) {
       wave = (long long)tc::CTAS_PER_SM * sms;
     cudaGetLastError();
   }
-  ProfScope prof("attn_sparse_rows", st);
+  ProfScope prof(mode == 0 ? "attn_sparse_rows" : "attn_special_rows", st);
   prof.set_launches((int)((items + wave - 1) / wave));
   for (long long base = 0; base < items; base += wave) {
     p.item0 = (int)base;
     const unsigned n = (unsigned)(items - base < wave ? items - base : wave);
-    tc::attn_tc_kernel<<<n, tc::THREADS, tc::SMEM_BYTES, st>>>(p);
+    kern<<<n, tc::THREADS, tc::SMEM_BYTES, st>>>(p);
     count_launch();
-    if (int rc = check_launch("attn_tc_kernel")) return rc;
+    if (int rc = check_launch(mode == 0 ? "attn_tc_kernel<patch rows>" : "attn_tc_kernel<special rows>")) return rc;
   }
   return ZEBRA_OK;
 }
+
+int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st) { return launch_tc(a, 0, st); }
+int launch_special_rows_tc(const AttnArgs& a, cudaStream_t st) { return launch_tc(a, 1, st); }
 
 }  // namespace zebra

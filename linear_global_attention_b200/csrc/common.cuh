@@ -160,6 +160,16 @@ void set_error(const std::string& msg);
 void count_launch(int n = 1);
 int check_launch(const char* what);   // ZEBRA_OK or ZEBRA_ERR_CUDA (sets the message)
 
+// Argument checks shared by the entry points (each returns a ZEBRA_* status and
+// sets the message): geometry limits, element type, strides of a [N, H, d]
+// input (NULL layout = contiguous; fills *ts, *hs), a non-null 16-byte aligned
+// device pointer, and an sm_100 current device.
+int check_geom(const zebra_geom* g);
+int check_dtype(zebra_dtype dt);
+int check_layout(const zebra_geom* g, zebra_dtype dt, const zebra_layout* lay, long long* ts, long long* hs);
+int check_ptr16(const void* p, const char* name);
+int check_device();
+
 // Optional per-kernel timing: while profiling is on (zebra_profile_enable), a
 // ProfScope records a CUDA event on `st` when it is made and another when it
 // goes out of scope, around one kernel launch (or set_launches(n) launches).

@@ -67,9 +67,27 @@ struct AttnArgs {
 };
 template <typename T> int launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
 int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st);
+int launch_special_rows_tc(const AttnArgs& a, cudaStream_t st);
 // sticky device status word of the kernels with bounded waits (per device)
 int read_and_clear_status(int* out);
+// error-path test hook of the tcgen05 sparse kernel (current device)
+int set_debug_inject(int block, unsigned long long wait_ns);
 template <typename T> int launch_special_rows(const AttnArgs& a, cudaStream_t st);
+
+// ---- attention-concentration diagnostic ----
+constexpr int COV_MAX_TILES = 1024;   // sampled query tiles per call (passed as kernel parameters)
+struct CoverageArgs {
+  Geo g;
+  const void* q; const void* k;       // [N, H, d] bf16, strided
+  long long ts, hs;
+  const uint32_t* mask;               // [H, T, W] selection
+  int n, splits;
+  float4* part;                       // [n, H, splits, 64]: (max, total, selected, special), log2 units
+  float* sel; float* spec;            // [n, H, 64]
+  int32_t tiles[COV_MAX_TILES];
+};
+int coverage_splits(const Geo& g, int n);
+int launch_coverage(const CoverageArgs& a, cudaStream_t st);
 
 // ---- linear stage ----
 struct LinearArgs {
@@ -90,9 +108,10 @@ int linear_chunks(const Geo& g, int* chunk_tokens);
 
 // ---- closed-form affine fit ----
 constexpr int AF_D = 64;
-// one group's float64 moments: count, sum x, sum y, sum x x^T, sum x y^T
+// one group's float64 moments: count, sum x, sum y, sum x x^T, sum x y^T, sum |y|^2
 constexpr int AF_N = 0, AF_SX = 1, AF_SY = AF_SX + AF_D, AF_SXX = AF_SY + AF_D, AF_SXY = AF_SXX + AF_D * AF_D;
-constexpr int AF_STRIDE = AF_SXY + AF_D * AF_D;   // 8321
+constexpr int AF_SYY = AF_SXY + AF_D * AF_D;
+constexpr int AF_STRIDE = AF_SYY + 1;   // 8322
 struct AffineArgs {
   Geo g;
   const void* x; const void* y;     // [N, H, d] samples (linear output, teacher output)
@@ -107,5 +126,7 @@ template <typename T> int launch_affine_moments(const AffineArgs& a, cudaStream_
 int launch_affine_solve(const double* moments, int per_head, int heads, double lam, float* A, float* b,
                         cudaStream_t st);
 int read_and_clear_affine_status(int* out);
+int launch_affine_residual(const double* moments, int per_head, int heads, const float* A, const float* b,
+                           double* err, cudaStream_t st);
 
 }  // namespace zebra

@@ -178,14 +178,70 @@ def test_affine_argument_errors(L):
     assert L.zebra_affine_solve(ctypes.byref(g), p, 3, 0.1, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
 
 
-def test_microbenchmark_compiles(tmp_path):
-    # the tcgen05 issue-cost microbenchmark behind profiles/mma_issue_b200.md stays buildable
-    import shutil
-    import subprocess
-    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
-    if not os.path.exists(nvcc):
-        pytest.skip("nvcc not available")
-    src = os.path.join(ROOT, "linear_global_attention_b200", "microbench", "mma_issue.cu")
-    r = subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-o",
-                        str(tmp_path / "mma_issue"), src], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr
+def _hybrid(L, g, kind, y=0.8, ptr=4096):
+    p = ctypes.c_void_p(ptr)
+    return L.zebra_hybrid_layer(ctypes.byref(g), kind, p, p, p, None, None, y, 100.0, 1e-6, p, p, 1 << 40, None)
+
+
+@pytest.mark.parametrize("kind", [zb.ZEBRA_LAYER_SPARSE, zb.ZEBRA_LAYER_DENSE])
+def test_hybrid_layer_rejects_32bit_tma_overflow(L, kind):
+    # 49,152 tiles x 700 heads x 64 rows: beyond 32-bit TMA row coordinates, refused before any launch
+    assert _hybrid(L, _g(views=768, grid_h=64, grid_w=64, heads=700, n_special=0), kind) == zb.ZEBRA_ERR_UNSUPPORTED
+    assert "2^31" in zb.zebra_last_error()
+
+
+def test_hybrid_layer_argument_errors(L):
+    assert _hybrid(L, _g(), 7) == zb.ZEBRA_ERR_INVALID_ARG                       # unknown kind
+    assert _hybrid(L, _g(), zb.ZEBRA_LAYER_SPARSE, y=1.0) == zb.ZEBRA_ERR_INVALID_ARG
+    assert _hybrid(L, _g(), zb.ZEBRA_LAYER_LINEAR, ptr=4100) == zb.ZEBRA_ERR_INVALID_ARG
+    # more tiles than the selector handles
+    assert _hybrid(L, _g(views=2000, grid_h=64, grid_w=64), zb.ZEBRA_LAYER_SPARSE) == zb.ZEBRA_ERR_UNSUPPORTED
+
+
+def test_noalloc_shares_the_argument_checks(L):
+    p = ctypes.c_void_p(4096)
+
+    def call(g, layout=None, ptr=p):
+        return L.zebra_linear_attn_noalloc(ctypes.byref(g), zb.ZEBRA_BF16, ptr, ptr, ptr, layout, None, None,
+                                           100.0, 1e-6, ptr, None)
+
+    # the same statuses as zebra_linear_attn for the same bad inputs
+    for g, code in ((_g(head_dim=32), zb.ZEBRA_ERR_UNSUPPORTED), (_g(grid_h=5000), zb.ZEBRA_ERR_UNSUPPORTED),
+                    (_g(heads=0), zb.ZEBRA_ERR_INVALID_ARG), (_g(views=1 << 30, grid_h=64, grid_w=64),
+                                                              zb.ZEBRA_ERR_UNSUPPORTED)):
+        assert call(g) == code
+        assert L.zebra_linear_attn(ctypes.byref(g), zb.ZEBRA_BF16, p, p, p, None, None, None, 100.0, 1e-6, p, p,
+                                   1 << 40, None) == code
+    assert call(_g(), layout=ctypes.byref(zb.Layout(130, 64))) == zb.ZEBRA_ERR_INVALID_ARG
+    assert call(_g(), ptr=ctypes.c_void_p(4100)) == zb.ZEBRA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.3, 0.5, 0.7, 1.0])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_allocate_layers_matches_oracle(L, frac, seed):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    err = rng.integers(0, 6, 24).astype(np.float64)      # many ties
+    err[rng.integers(0, 24, 2)] = np.nan                   # NaN ranks last
+    got = zb.zebra_allocate_layers(err, frac).astype(bool)
+    assert (got == oracle.allocate_layers(err, frac)).all()
+    assert got.sum() == int(np.floor(frac * 24 + 0.5))
+
+
+def test_allocate_layers_rejects_bad_arguments(L):
+    import numpy as np
+    assert L.zebra_allocate_layers(None, 3, 0.5, None) == -1
+    e = np.zeros(3)
+    out = np.zeros(3, np.int32)
+    assert L.zebra_allocate_layers(e.ctypes.data_as(ctypes.c_void_p), 3, 1.5,
+                                   out.ctypes.data_as(ctypes.c_void_p)) == -1
+    assert L.zebra_allocate_layers(None, 0, 0.5, None) == 0
+
+
+def test_affine_residual_argument_errors(L):
+    p = ctypes.c_void_p(4096)
+    g = _g()
+    assert L.zebra_affine_residual(ctypes.byref(g), None, 0, p, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_residual(ctypes.byref(g), p, 2, p, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_residual(ctypes.byref(g), p, 0, p, p, ctypes.c_void_p(4100), None) == zb.ZEBRA_ERR_INVALID_ARG
+    assert L.zebra_affine_residual(ctypes.byref(g), p, 0, None, p, p, None) == zb.ZEBRA_ERR_INVALID_ARG

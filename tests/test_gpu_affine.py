@@ -1,5 +1,7 @@
 """GPU parity of the closed-form centred affine fit (zebra_affine_moments,
-zebra_affine_solve) with the oracle's affine_moments / affine_solve.
+zebra_affine_solve), the single-stage conversion error (zebra_affine_residual)
+and the layer allocation (zebra_allocate_layers) with the oracle's
+affine_moments / affine_solve / affine_residual / allocate_layers.
 
 Page "How Hybrid Attention Lets Feed-Forward 3D Models Scale to Many Views",
 section "A closed-form fit avoids retraining from scratch". Moments are float64
@@ -20,14 +22,15 @@ from tests import parity_helpers as ph
 pytestmark = pytest.mark.gpu
 
 D = 64
-KEYS = ("n", "sx", "sy", "sxx", "sxy")
+KEYS = ("n", "sx", "sy", "sxx", "sxy", "syy")
 
 
 def _split(buf, groups):
     m = buf.cpu().numpy().reshape(groups, zb.ZEBRA_AFFINE_GROUP_DOUBLES)
     return {"n": m[:, 0], "sx": m[:, 1:1 + D], "sy": m[:, 1 + D:1 + 2 * D],
             "sxx": m[:, 1 + 2 * D:1 + 2 * D + D * D].reshape(groups, D, D),
-            "sxy": m[:, 1 + 2 * D + D * D:].reshape(groups, D, D)}
+            "sxy": m[:, 1 + 2 * D + D * D:1 + 2 * D + 2 * D * D].reshape(groups, D, D),
+            "syy": m[:, 1 + 2 * D + 2 * D * D]}
 
 
 def _moments(g, x_d, y_d, per_head, m=None):
@@ -164,3 +167,56 @@ def test_fit_of_the_gpu_linear_stage_to_dense_attention():
     torch.cuda.synchronize()
     want = np.einsum("nhj,hij->nhi", xh, A) + b
     np.testing.assert_allclose(ph.host(out), want, atol=1e-4 * scale, rtol=1e-4)
+
+
+def test_conversion_errors_and_allocation_match_oracle():
+    """Section "Linear-centered stages plus tile-sparse stages": stages are ranked
+    by the error of converting each alone to linear attention, and the fraction x
+    with the lowest errors becomes linear. Six synthetic stages of the tiny
+    geometry (Q, K sharpened by a different factor each, so the linear stage
+    misses the dense teacher by different amounts): x = the GPU linear stage
+    without a correction, y = the dense teacher (the sparse entry point at
+    y = 0), one pooled fit per stage. The GPU's errors (from its moments and
+    its fitted A, b) match the oracle's affine_residual of the same samples and
+    the same A, b, and the allocations for x = 0.5 and 0.7 match
+    oracle.allocate_layers on the oracle's errors."""
+    g = Geom(4, 16, 16, 2)
+    zg = ph.zgeom(g)
+    r = np.random.default_rng(36)
+    ws_lin = zb.workspace(zg, zb.ZEBRA_OP_LINEAR, zb.ZEBRA_F32)
+    ws_sp = zb.workspace(zg, zb.ZEBRA_OP_SPARSE, zb.ZEBRA_F32, 0.0)
+    err_gpu, err_want = [], []
+    for stage in range(6):
+        sharp = 0.4 + 0.35 * stage
+        q, k, v = (r.standard_normal((g.n_tokens, g.heads, D)).astype(np.float32) for _ in range(3))
+        q *= np.float32(sharp)
+        k *= np.float32(sharp)
+        qd, kd, vd = (ph.dev(t, "f32") for t in (q, k, v))
+        x_d = torch.empty_like(qd)
+        y_d = torch.empty_like(qd)
+        zb.zebra_linear_attn(zg, qd, kd, vd, None, None, x_d, ws_lin)
+        zb.zebra_sparse_attn(zg, qd, kd, vd, 0.0, y_d, ws_sp)           # y = 0: dense softmax teacher
+        m = _moments(g, x_d, y_d, False)
+        xh, yh = ph.host(x_d), ph.host(y_d)
+        mw = oracle.affine_moments(xh, yh)
+        lam = 1e-2 * float(np.trace(mw["sxx"][0] / mw["n"][0] - np.outer(mw["sx"][0], mw["sx"][0]) / mw["n"][0] ** 2)) / D
+        A, b = _solve(g, m, lam, False)
+        At = torch.from_numpy(A.astype(np.float32)).cuda()
+        bt = torch.from_numpy(b.astype(np.float32)).cuda()
+        e = torch.empty(1, dtype=torch.float64, device="cuda")
+        zb.zebra_affine_residual(zg, m, At, bt, e)
+        torch.cuda.synchronize()
+        assert zb.zebra_sync_status() == zb.ZEBRA_OK
+        got = _split(m, 1)
+        np.testing.assert_allclose(got["syy"], mw["syy"], rtol=1e-11)
+        want = oracle.affine_residual(mw, A[:1], b[:1])
+        # the error also equals the direct mean squared error of the corrected samples
+        direct = np.mean(np.sum((np.einsum("nhj,ij->nhi", xh, A[0]) + b[0] - yh) ** 2, axis=-1))
+        np.testing.assert_allclose(want[0], direct, rtol=1e-9)
+        err_gpu.append(float(e.cpu()[0]))
+        err_want.append(float(want[0]))
+    np.testing.assert_allclose(err_gpu, err_want, rtol=1e-8)
+    assert len(set(np.round(err_want, 6))) == 6          # the stages really differ
+    for frac in (0.5, 0.7):
+        got = zb.zebra_allocate_layers(err_gpu, frac).astype(bool)
+        assert (got == oracle.allocate_layers(err_want, frac)).all()

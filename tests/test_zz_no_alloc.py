@@ -3,10 +3,13 @@ callers that cannot allocate device memory (its scratch is a built-in device
 array instead of a caller workspace).
 
 Two calls in a row on different inputs are compared with zebra_linear_attn,
-the workspace-based entry point, within the bf16 tolerance of the parity
-tests. The second call checks that nothing left in the shared scratch array by
-the first call leaks into its result. The file name makes pytest collect it
-last; it also passes alone in a fresh process.
+the workspace-based entry point. Below the size at which the chunk partials
+fill the built-in array the two entry points sum in the same order, so the
+outputs must be bit-identical; above it (128 views) the chunks grow and the
+outputs must agree within the bf16 tolerance of the parity tests. The second
+call of each pair checks that nothing left in the shared scratch array by the
+first call leaks into its result. The file name makes pytest collect it last;
+it also passes alone in a fresh process.
 """
 import ctypes
 
@@ -21,18 +24,19 @@ from tests import parity_helpers as ph
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(seed):
-    w = synth.custom(6, 37, 37, 16, seed=seed, recipe="iid", dtype="bf16")
+def _inputs(seed, views):
+    w = synth.custom(views, 37, 37, 16, seed=seed, recipe="iid", dtype="bf16")
     q, k, v = synth.qkv(w)
     A, b = synth.affine(16, seed)
     return w, q, k, v, A, b
 
 
-@pytest.mark.parametrize("dtype", ["bf16"])
-def test_noalloc_matches_workspace_entry_point_twice(dtype):
+@pytest.mark.parametrize("views,exact", [(6, True), (128, False)], ids=["same_chunks", "grown_chunks"])
+def test_noalloc_matches_workspace_entry_point_twice(views, exact):
+    dtype = "bf16"
     results = []
     for seed in (31, 32):                       # two calls in a row, different inputs
-        w, q, k, v, A, b = _inputs(seed)
+        w, q, k, v, A, b = _inputs(seed, views)
         g = zb.geom(w.views, w.grid_h, w.grid_w, w.heads)
         qd, kd, vd = ph.dev(q, dtype), ph.dev(k, dtype), ph.dev(v, dtype)
         At, bt = torch.from_numpy(A).cuda(), torch.from_numpy(b).cuda()
@@ -45,7 +49,9 @@ def test_noalloc_matches_workspace_entry_point_twice(dtype):
         assert zb.zebra_sync_status() == zb.ZEBRA_OK
         got, want = ph.host(out), ph.host(ref)
         assert np.isfinite(got).all()
-        ph.assert_close(got, want, dtype, f"noalloc vs workspace entry point, seed {seed}")
+        ph.assert_close(got, want, dtype, f"noalloc vs workspace entry point, {views} views, seed {seed}")
+        if exact:
+            assert torch.equal(out, ref), "same chunks must give bit-identical outputs"
         results.append(got)
     assert not np.array_equal(results[0], results[1])
 
