@@ -281,6 +281,317 @@ __global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_const
 }
 
 // --------------------------------------------------------------------------
+// 1'/3'. state and apply (bf16), four threads per token
+// --------------------------------------------------------------------------
+// 256 threads, 64 tokens per step. Thread (tok = tid / 4, part = tid % 4) owns
+// 16 channels of its token that form 8 whole rotation pairs: half = part / 2
+// (channels 0-31 turn by patch row, 32-63 by column), sub = part % 2 (pairs
+// j = 8 sub .. 8 sub + 7 of the half): the "a" channels 32 half + 8 sub .. + 7
+// and their partners 16 further. The four threads of a token combine the RMS
+// norm, the maximum and the sum with two shuffles each. 8 warps split the
+// 64 x 72 contraction: rows 16 (warp % 4) .. + 15, columns 0-31 plus the
+// z column (warp / 4 = 0) or columns 32-63 (warp / 4 = 1).
+constexpr int LQ_THREADS = 256;
+
+__device__ __forceinline__ void fetch_rows_q4(uint32_t tile, const __nv_bfloat16* base, long long nb, long long n1,
+                                              long long ts, int tok, int half, int sub) {
+  const long long n = nb + tok;
+  const bool ok = n < n1;
+  const __nv_bfloat16* p = base + (ok ? n : 0) * ts + 32 * half + 8 * sub;
+  const int ca = 4 * half + sub;   // 16-byte chunk of the "a" channels; the partners are 2 chunks on
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, ca)), "l"(p),
+               "r"(ok ? 16 : 0));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, ca + 2)), "l"(p + 16),
+               "r"(ok ? 16 : 0));
+}
+
+// f(x) on this thread's 16 channels (xa: the "a" channels, xb: their partners)
+__device__ __forceinline__ void features_q4(float* xa, float* xb, int half, int sub, bool special, int row, int col,
+                                            const float2* __restrict__ tab, float eps) {
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(xa[e], xa[e], fmaf(xb[e], xb[e], ss));
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float sc = rsqrtf(ss * (1.0f / D) + eps);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    xa[e] *= sc;
+    xb[e] *= sc;
+  }
+  if (!special) {
+    const float2* t = tab + (half ? col : row) * 16 + 8 * sub;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 cs = __ldg(t + e);
+      const float a = xa[e], b = xb[e];
+      xa[e] = a * cs.x - b * cs.y;
+      xb[e] = b * cs.x + a * cs.y;
+    }
+  }
+  float mx = fmaxf(xa[0], xb[0]);
+#pragma unroll
+  for (int e = 1; e < 8; ++e) mx = fmaxf(mx, fmaxf(xa[e], xb[e]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float off = -mx * LOG2E;
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    xa[e] = fast_exp2(fmaf(xa[e], LOG2E, off));
+    xb[e] = fast_exp2(fmaf(xb[e], LOG2E, off));
+    sum += xa[e] + xb[e];
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const float inv = 1.0f / sum;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    xa[e] *= inv;
+    xb[e] *= inv;
+  }
+}
+
+__device__ __forceinline__ void read_q4(const unsigned char* tile, int tok, int half, int sub, float* xa, float* xb) {
+  const int ca = 4 * half + sub;
+  const uint4 wa = *reinterpret_cast<const uint4*>(tile + lswz(tok, ca));
+  const uint4 wb = *reinterpret_cast<const uint4*>(tile + lswz(tok, ca + 2));
+  const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&wa);
+  const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&wb);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 fa = __bfloat1622float2(ha[e]), fb = __bfloat1622float2(hb[e]);
+    xa[2 * e] = fa.x;
+    xa[2 * e + 1] = fa.y;
+    xb[2 * e] = fb.x;
+    xb[2 * e + 1] = fb.y;
+  }
+}
+
+__device__ __forceinline__ void store_q4(unsigned char* tile, int tok, int half, int sub, const float* xa,
+                                         const float* xb) {
+  const int ca = 4 * half + sub;
+  uint4 va, vb;
+  __nv_bfloat162* ha = reinterpret_cast<__nv_bfloat162*>(&va);
+  __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&vb);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    ha[e] = __floats2bfloat162_rn(xa[2 * e], xa[2 * e + 1]);
+    hb[e] = __floats2bfloat162_rn(xb[2 * e], xb[2 * e + 1]);
+  }
+  *reinterpret_cast<uint4*>(tile + lswz(tok, ca)) = va;
+  *reinterpret_cast<uint4*>(tile + lswz(tok, ca + 2)) = vb;
+}
+
+__global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __grid_constant__ LinearArgs a) {
+  extern __shared__ __align__(128) unsigned char state_smem[];
+  StateSmem& ss = *reinterpret_cast<StateSmem*>(state_smem);
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x;   // grid (head, chunk): the heads of the same tokens run together
+  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
+  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
+  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
+  const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v) + (long long)h * a.hs;
+  const int tok = tid >> 2, half = (tid >> 1) & 1, sub = tid & 1;
+  const int mrow = warp & 3, grp = warp >> 2;   // channel rows 16 mrow .., column group
+  float acc[5][4];
+#pragma unroll
+  for (int j = 0; j < 5; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const int g4 = lane >> 2;
+  const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
+
+  const int nblk = (int)((n1 - n0 + 63) / 64);
+  for (int i = 0; i < LSTAGES - 1; ++i) {
+    if (i < nblk) {
+      fetch_rows_q4(lsmem(ss.k[i]), K, n0 + 64LL * i, n1, a.ts, tok, half, sub);
+      fetch_rows_q4(lsmem(ss.v[i]), Vt, n0 + 64LL * i, n1, a.ts, tok, half, sub);
+    }
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
+  for (int i = 0; i < nblk; ++i) {
+    const int st = i % LSTAGES;
+    __syncthreads();   // every warp is done with the stage refilled below and with phi
+    {
+      const int f = i + LSTAGES - 1;
+      if (f < nblk) {
+        fetch_rows_q4(lsmem(ss.k[f % LSTAGES]), K, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+        fetch_rows_q4(lsmem(ss.v[f % LSTAGES]), Vt, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+      }
+      asm volatile("cp.async.commit_group;\n" ::);
+    }
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
+    __syncthreads();
+    const long long n = n0 + 64LL * i + tok;
+    const bool valid = n < n1;
+    float xa[8], xb[8];
+    read_q4(ss.k[st], tok, half, sub, xa, xb);
+    {
+      bool sp;
+      int row, col;
+      token_pos(g, valid ? n : 0, sp, row, col);
+      features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      if (!valid) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
+      }
+    }
+    store_q4(ss.phi, tok, half, sub, xa, xb);
+    __syncthreads();
+    const uint32_t vb = lsmem(ss.v[st]);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {   // 16 tokens per k-step
+      uint32_t af[4];
+      {
+        const int mi = lane >> 3, ri = lane & 7;
+        l_ldsm_x4_t(lsmem(ss.phi) + lswz(ks * 16 + (mi >> 1) * 8 + ri, mrow * 2 + (mi & 1)), af[0], af[1], af[2],
+                    af[3]);
+      }
+#pragma unroll
+      for (int d2 = 0; d2 < 2; ++d2) {
+        const int dp = 2 * grp + d2;   // V columns 16 dp .. 16 dp + 15
+        const int mi = lane >> 3, ri = lane & 7;
+        uint32_t b0, b1, b2, b3;
+        l_ldsm_x4_t(vb + lswz(ks * 16 + (mi & 1) * 8 + ri, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
+        l_mma(acc[2 * d2], af, b0, b1);
+        l_mma(acc[2 * d2 + 1], af, b2, b3);
+      }
+      if (grp == 0) l_mma(acc[4], af, ones, ones);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;\n" ::);
+  float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
+  const int q4 = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 5; ++j) {
+    if (j == 4 && grp != 0) break;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = mrow * 16 + g4 + (e >> 1) * 8;
+      const int c = j < 4 ? 32 * grp + 8 * j + 2 * q4 + (e & 1) : 64 + 2 * q4 + (e & 1);
+      if (c <= 64) part[r * 65 + c] = acc[j][e];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ LinearArgs a) {
+  __shared__ __align__(128) unsigned char phi_s[64 * 128];   // f(Q) block, then the bf16 output block
+  __shared__ __align__(128) unsigned char q_s[LSTAGES][64 * 128];
+  __shared__ __align__(128) unsigned char b_s[NB * 128];
+  __shared__ float den_s[64];
+  const Geo& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
+  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
+  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q) + (long long)h * a.hs;
+  const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
+  for (int i = tid; i < NB * 8; i += LQ_THREADS) {
+    const int r = i >> 3, c = i & 7;
+    *reinterpret_cast<uint4*>(b_s + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
+  }
+  const int tok = tid >> 2, half = (tid >> 1) & 1, sub = tid & 1;
+  const int mrow = warp & 3, grp = warp >> 2;   // token rows 16 mrow .., column group
+  const int g4 = lane >> 2, q4 = lane & 3;
+  float bias[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = 32 * grp + 8 * j + 2 * q4;
+    bias[2 * j] = a.b ? a.b[h * 64 + c] : 0.f;
+    bias[2 * j + 1] = a.b ? a.b[h * 64 + c + 1] : 0.f;
+  }
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+  const int nblk = (int)((n1 - n0 + 63) / 64);
+  for (int i = 0; i < LSTAGES - 1; ++i) {
+    if (i < nblk) fetch_rows_q4(lsmem(q_s[i]), Q, n0 + 64LL * i, n1, a.ts, tok, half, sub);
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
+  for (int i = 0; i < nblk; ++i) {
+    const int st = i % LSTAGES;
+    const long long nb = n0 + 64LL * i;
+    __syncthreads();   // the stage refilled below and phi_s (last block's output) are free
+    {
+      const int f = i + LSTAGES - 1;
+      if (f < nblk) fetch_rows_q4(lsmem(q_s[f % LSTAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+      asm volatile("cp.async.commit_group;\n" ::);
+    }
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
+    __syncthreads();
+    const long long n = nb + tok;
+    const bool valid = n < n1;
+    float xa[8], xb[8];
+    read_q4(q_s[st], tok, half, sub, xa, xb);
+    {
+      bool sp;
+      int row, col;
+      token_pos(g, valid ? n : 0, sp, row, col);
+      features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      if (!valid) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
+      }
+    }
+    store_q4(phi_s, tok, half, sub, xa, xb);
+    __syncthreads();
+    float acc[5][4];
+#pragma unroll
+    for (int j = 0; j < 5; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {  // 16 channels per k-step
+      uint32_t af[4];
+      {
+        const int mi = lane >> 3, ri = lane & 7;
+        l_ldsm_x4(lsmem(phi_s) + lswz(mrow * 16 + (mi & 1) * 8 + ri, 2 * ks + (mi >> 1)), af[0], af[1], af[2],
+                  af[3]);
+      }
+#pragma unroll
+      for (int n2 = 0; n2 < 2; ++n2) {
+        const int np = 2 * grp + n2;   // state columns 16 np .. 16 np + 15
+        const int mi = lane >> 3, ri = lane & 7;
+        uint32_t b0, b1, b2, b3;
+        l_ldsm_x4(lsmem(b_s) + lswz(np * 16 + (mi >> 1) * 8 + ri, 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        l_mma(acc[2 * n2], af, b0, b1);
+        l_mma(acc[2 * n2 + 1], af, b2, b3);
+      }
+      if (grp == 0) {
+        const int mi = (lane >> 3) & 1, ri = lane & 7;
+        uint32_t b0, b1;
+        l_ldsm_x2(lsmem(b_s) + lswz(64 + ri, 2 * ks + mi), b0, b1);
+        l_mma(acc[4], af, b0, b1);
+      }
+    }
+    // the z column (column 64: acc[4][0] / acc[4][2] of the q4 == 0 lanes of group 0) to shared memory
+    if (grp == 0 && q4 == 0) {
+      den_s[mrow * 16 + g4] = acc[4][0];
+      den_s[mrow * 16 + g4 + 8] = acc[4][2];
+    }
+    __syncthreads();   // den_s written; every warp has read phi_s: reuse it for the output block
+#pragma unroll
+    for (int half2 = 0; half2 < 2; ++half2) {
+      const int r = mrow * 16 + g4 + half2 * 8;
+      const float il = 1.0f / den_s[r];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
+                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
+        *reinterpret_cast<__nv_bfloat162*>(phi_s + lswz(r, 4 * grp + j) + 4 * q4) = v2;
+      }
+    }
+    __syncthreads();
+    // 64 tokens x 128 bytes, written as whole 16-byte chunks of each token's head row
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int idx = tid + LQ_THREADS * c, r = idx >> 3, ch = idx & 7;
+      const long long nn = nb + r;
+      if (nn < n1)
+        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
+    }
+  }
+  asm volatile("cp.async.wait_group 0;\n" ::);
+}
+
+// --------------------------------------------------------------------------
 // fp32 state
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) linear_state_simt_kernel(const __grid_constant__ LinearArgs a) {
@@ -514,13 +825,22 @@ int linear_chunks(const Geo& g, int* chunk_tokens) {
   return (int)chunks;
 }
 
+#ifndef ZEBRA_LIN_Q4
+#define ZEBRA_LIN_Q4 1
+#endif
+
 template <>
 int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
   {
     ProfScope prof("linear_state", st);
-    cudaFuncSetAttribute(linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
-    linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, sizeof(StateSmem), st>>>(a);
+    if (ZEBRA_LIN_Q4) {
+      cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
+      linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, sizeof(StateSmem), st>>>(a);
+    } else {
+      cudaFuncSetAttribute(linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
+      linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, sizeof(StateSmem), st>>>(a);
+    }
   }
   count_launch();
   if (int rc = check_launch("linear_state_kernel")) return rc;
@@ -532,7 +852,10 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
   {
     ProfScope prof("linear_apply", st);
-    linear_apply_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
+    if (ZEBRA_LIN_Q4)
+      linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, 0, st>>>(a);
+    else
+      linear_apply_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
   }
   count_launch();
   return check_launch("linear_apply_kernel");

@@ -8,12 +8,14 @@
 // toward the lower tile index.
 //
 // Two kernels per group of heads:
-//  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 64x64-tile
+//  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 128x128-tile
 //     fp32 GEMM (K = 64) written to scratch; each score is a fixed-order fma chain.
 //  2. select_kernel: one CTA per row (h, t) loads the row into shared memory as
 //     order-preserving 32-bit keys, finds the k-th largest key with four 8-bit
 //     radix passes (histograms replicated 8 ways to spread same-bin atomics over
-//     banks), then emits the bitmask: keys above the threshold, plus the
+//     banks; in the first pass, whose byte holds the sign and exponent bits,
+//     lanes of a warp that hit the same bin add once), one warp scans the 256
+//     bins for the threshold bin, then emits the bitmask: keys above the threshold, plus the
 //     lowest-index keys equal to it (block-wide scan over the mask words).
 //     It also flags near-ties: the k-th and (k+1)-th scores within a relative
 //     gap of 1e-5.
@@ -22,49 +24,58 @@
 
 namespace zebra {
 
+// CTA = a 128 x 128 tile of S (query tiles t0.., key tiles u0..) of one head;
+// the 64-channel means are staged channel-major in shared memory and every
+// thread accumulates an 8 x 8 block (rows ty + 16 i, columns tx + 16 j) with a
+// fixed-order fma chain over the channels.
+constexpr int SC_TILE = 128;
+constexpr int SC_KC = 32;   // channels staged per step
 __global__ void __launch_bounds__(256) scores_kernel(SelectArgs a) {
-  __shared__ float sq[64][65];
-  __shared__ float sk[64][65];
+  __shared__ float sq[SC_KC][SC_TILE + 4];
+  __shared__ float sk[SC_KC][SC_TILE + 4];
   const int T = a.g.T;
   const int hh = blockIdx.z;
   const int h = a.h0 + hh;
-  const int t0 = blockIdx.y * 64, u0 = blockIdx.x * 64;
+  const int t0 = blockIdx.y * SC_TILE, u0 = blockIdx.x * SC_TILE;
   const float* qm = a.qm + (size_t)h * T * D;
   const float* km = a.km + (size_t)h * T * D;
-  for (int i = threadIdx.x; i < 64 * 16; i += 256) {
-    const int r = i / 16, c4 = (i % 16) * 4;
-    float4 q = make_float4(0, 0, 0, 0), k = q;
-    if (t0 + r < T) q = *reinterpret_cast<const float4*>(qm + (size_t)(t0 + r) * D + c4);
-    if (u0 + r < T) k = *reinterpret_cast<const float4*>(km + (size_t)(u0 + r) * D + c4);
-    sq[r][c4] = q.x; sq[r][c4 + 1] = q.y; sq[r][c4 + 2] = q.z; sq[r][c4 + 3] = q.w;
-    sk[r][c4] = k.x; sk[r][c4 + 1] = k.y; sk[r][c4 + 2] = k.z; sk[r][c4 + 3] = k.w;
-  }
-  __syncthreads();
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < D; ++c) {
-    float qv[4], kv[4];
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int c0 = 0; c0 < D; c0 += SC_KC) {
+    __syncthreads();   // the previous channel block is consumed
+    for (int i = threadIdx.x; i < SC_TILE * (SC_KC / 4); i += 256) {
+      const int r = i / (SC_KC / 4), c4 = (i % (SC_KC / 4)) * 4;
+      float4 q = make_float4(0, 0, 0, 0), k = q;
+      if (t0 + r < T) q = *reinterpret_cast<const float4*>(qm + (size_t)(t0 + r) * D + c0 + c4);
+      if (u0 + r < T) k = *reinterpret_cast<const float4*>(km + (size_t)(u0 + r) * D + c0 + c4);
+      sq[c4][r] = q.x; sq[c4 + 1][r] = q.y; sq[c4 + 2][r] = q.z; sq[c4 + 3][r] = q.w;
+      sk[c4][r] = k.x; sk[c4 + 1][r] = k.y; sk[c4 + 2][r] = k.z; sk[c4 + 3][r] = k.w;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < SC_KC; ++c) {
+      float qv[8], kv[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = sq[ty + 16 * i][c];
+      for (int i = 0; i < 8; ++i) qv[i] = sq[c][ty + 16 * i];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) kv[j] = sk[tx + 16 * j][c];
+      for (int j = 0; j < 8; ++j) kv[j] = sk[c][tx + 16 * j];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
+    }
   }
   float* out = a.scores + (size_t)hh * T * a.Tld;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const int t = t0 + ty + 16 * i;
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const int u = u0 + tx + 16 * j;
       if (u < T) out[(size_t)t * a.Tld + u] = acc[i][j];
     }
@@ -110,9 +121,21 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
     for (int i = tid; i < HCOPIES * HSTRIDE; i += SEL_THREADS) hist[i] = 0;
     __syncthreads();
     uint32_t* hc = hist + (lane & (HCOPIES - 1)) * HSTRIDE;
-    for (int i = tid; i < T; i += SEL_THREADS) {
-      const uint32_t k = keys[i];
-      if ((k & pmask) == prefix) atomicAdd(&hc[(k >> shift) & 255u], 1u);
+    if (shift == 24) {
+      // the top byte (sign and exponent bits) takes few distinct values: one
+      // atomic per distinct bin per warp (the loop bound is uniform, so the
+      // whole warp takes part in every match)
+      for (int base = 0; base < T; base += SEL_THREADS) {
+        const int i = base + tid;
+        const uint32_t bin = i < T ? keys[i] >> 24 : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hc[bin], (uint32_t)__popc(peers));
+      }
+    } else {
+      for (int i = tid; i < T; i += SEL_THREADS) {
+        const uint32_t k = keys[i];
+        if ((k & pmask) == prefix) atomicAdd(&hc[(k >> shift) & 255u], 1u);
+      }
     }
     __syncthreads();
     if (tid < 256) {
@@ -122,16 +145,39 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
       hist[tid] = s;  // copy 0 slot tid: read by this thread only above
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t cum = 0;
-      int b = 255;
-      for (; b > 0; --b) {
-        if (cum + hist[b] >= need) break;
-        cum += hist[b];
+    if (warp == 0) {
+      // the bin holding the need-th largest key: lane l owns bins 255 - 8 l
+      // down to 248 - 8 l; an inclusive scan over the lanes (high bins first)
+      // finds the lane where the running count reaches need
+      uint32_t c[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[255 - 8 * lane - e];
+        sum += c[e];
       }
-      s_bin = (uint32_t)b;
-      s_need = need - cum;
-      s_eqtotal = hist[b];
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
+      if (lane == __ffs(hit) - 1) {
+        uint32_t cum = excl;
+        int b = 255 - 8 * lane - 7;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (cum + c[e] >= need) {
+            b = 255 - 8 * lane - e;
+            break;
+          }
+          cum += c[e];
+        }
+        s_bin = (uint32_t)b;
+        s_need = need - cum;
+        s_eqtotal = hist[b];
+      }
     }
     __syncthreads();
     prefix |= s_bin << shift;
@@ -222,7 +268,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
 int launch_scores(const SelectArgs& a, cudaStream_t st) {
   const int T = a.g.T;
   if (T == 0 || a.keep >= T) return ZEBRA_OK;
-  dim3 grid((T + 63) / 64, (T + 63) / 64, a.hc);
+  dim3 grid((T + SC_TILE - 1) / SC_TILE, (T + SC_TILE - 1) / SC_TILE, a.hc);
   ProfScope prof("tile_scores", st);
   scores_kernel<<<grid, 256, 0, st>>>(a);
   count_launch();
