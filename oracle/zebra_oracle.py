@@ -413,11 +413,19 @@ def split_heads(qkv, heads: int, d: int = 64):
 
 
 def hybrid_layer(x, w_qkv, w_o, kind: str, g: Geom, A=None, b=None, keep=None,
-                 rope_base: float = 100.0, eps: float = 1e-6) -> np.ndarray:
+                 rope_base: float = 100.0, eps: float = 1e-6, qkv_round=None) -> np.ndarray:
     """x + concat_heads(Attn(split(x W_qkv^T))) W_o^T for one layer of kind
-    'linear' | 'sparse' | 'dense'. x [N, D]; w_qkv [3D, D]; w_o [D, D]."""
+    'linear' | 'sparse' | 'dense'. x [N, D]; w_qkv [3D, D]; w_o [D, D].
+
+    qkv_round (optional) maps the projection output to the precision in which
+    an implementation stores it before the attention. The tile selection is a
+    discrete decision taken on those stored values, so a comparison with such an
+    implementation takes it in the same precision; the arithmetic after it stays
+    float64."""
     x = np.asarray(x, np.float64)
     qkv = x @ np.asarray(w_qkv, np.float64).T
+    if qkv_round is not None:
+        qkv = np.asarray(qkv_round(qkv), np.float64)
     q, k, v = split_heads(qkv, g.heads, g.head_dim)
     N = x.shape[0]
     if kind == "linear":

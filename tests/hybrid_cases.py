@@ -39,7 +39,14 @@ def attention_share(x, x_out) -> float:
     return float(np.linalg.norm(x_out - x) / np.linalg.norm(x_out))
 
 
+def qkv_bf16(qkv):
+    """The kernel's storage of the QKV projection: fp32 accumulation rounded to bf16."""
+    return synth.round_to_bf16(np.asarray(qkv, np.float32))
+
+
 def oracle_out(kind: str, mod=oracle, seed: int = 17):
+    """(x, the oracle's x_out) with the projection taken in the kernel's storage
+    precision (bf16), so that both sides select key tiles from the same values."""
     x, wqkv, wo, A, b = small_case(seed)
     keep = mod.keep_count(Y, GEOM.n_tiles)
-    return x, mod.hybrid_layer(x, wqkv, wo, kind, GEOM, A=A, b=b, keep=keep)
+    return x, mod.hybrid_layer(x, wqkv, wo, kind, GEOM, A=A, b=b, keep=keep, qkv_round=qkv_bf16)

@@ -13,7 +13,9 @@ is block-diagonal (one random 64x64 block per head) and large, so that each
 head's attention output reaches its own 64 output columns and the attention
 term carries >= 90% of the output norm (asserted on the oracle). The oracle
 then needs the projections of the sampled heads only: it computes them in
-float64 for every token, normalises and rotates them, runs its sparse stage on
+float64 for every token, rounds them to bf16 as the kernel stores them (the tile
+selection is a discrete decision, taken in the kernel's precision on both sides),
+normalises and rotates them in float64, runs its sparse stage on
 8 query tiles (one of each tile shape among them) and 4 special-token rows, and
 adds x plus the block of W_o. Selections of the sampled tiles must be
 bit-exact outside near-ties.
@@ -68,7 +70,9 @@ def oracle_side(x, wqkv, wo, tiles, specials):
     proj = np.empty((N, len(cols)))
     step = 65536
     for lo in range(0, N, step):
-        proj[lo:lo + step] = np.asarray(x[lo:lo + step], np.float64) @ w.T
+        # the kernel stores the projection in bf16 and selects tiles from those values:
+        # the oracle takes the selection in the same precision (arithmetic after it is float64)
+        proj[lo:lo + step] = synth.round_to_bf16((np.asarray(x[lo:lo + step], np.float64) @ w.T).astype(np.float32))
     q, k, v = (proj[:, s * nh * 64:(s + 1) * nh * 64].reshape(N, nh, 64) for s in range(3))
     del proj
     gh = Geom(G.views, G.grid_h, G.grid_w, nh)
