@@ -436,7 +436,8 @@ def view_scaling(pk, reps: int = 10):
       sparse_v32       32 views x (32x32 + 5), 16 heads, y = 0.8, latent recipe;
       linear_v128      128 views x (37x37 + 5), 16 heads, the full linear stage;
       sidebyside_v512  512 views x (37x37 + 5), 16 heads, y = 0.6 and y = 0.8,
-                       latent recipe, against torch SDPA on identical inputs.
+                       latent recipe, against torch SDPA on identical inputs and
+                       against the library's own dense path (y = 0).
     Median of `reps` calls (3 for the 512-view calls and SDPA)."""
     import torch
 
@@ -485,14 +486,16 @@ def view_scaling(pk, reps: int = 10):
     res = {"workload": desc}
     for y in (0.6, 0.8):
         res[f"y={y}"] = sparse(g, q, k, v, y, 3)
+    # the library's own dense path: y = 0 keeps every tile (one call)
+    res["own_dense_y=0"] = sparse(g, q, k, v, 0.0, 1)
     qt, kt, vt = (x.permute(1, 0, 2).unsqueeze(0).contiguous() for x in (q, k, v))   # [1, H, N, 64]
     del q, k, v
     med, all_ms = sdpa_ms(qt, kt, vt, reps=3)
     N, H = g.n_tokens, g.heads
     res["sdpa"] = {"ms": round(med, 1), "ms_reps": [round(x, 1) for x in all_ms],
                    "tflops": round(4 * 64 * N * N * H / (med / 1e3) / 1e12, 1)}
-    for y in (0.6, 0.8):
-        res[f"y={y}"]["speedup_vs_sdpa"] = round(med / res[f"y={y}"]["ms"], 3)
+    for key in ("y=0.6", "y=0.8", "own_dense_y=0"):
+        res[key]["speedup_vs_sdpa"] = round(med / res[key]["ms"], 3)
     out["sidebyside_v512"] = res
     del qt, kt, vt
     torch.cuda.empty_cache()

@@ -106,31 +106,50 @@ constexpr bool RSUM_MMA = ZEBRA_TC_RSUM_MMA != 0;
 // MUFU ex2 unit
 constexpr int EMU = ZEBRA_TC_EMU;
 static_assert(EMU >= 0 && EMU <= 8, "EMU counts column groups");
+#ifndef ZEBRA_TC_PTMEM
+#define ZEBRA_TC_PTMEM 0
+#endif
+// 1: the softmax writes P (bf16 pairs) into TMEM and O += P V reads its A
+// operand from there. An M = 64 MMA with A in TMEM reads row m of A from the
+// datapath lane that holds row m of its accumulator, so P and O share lanes
+// 0-15 of each lane quarter (O in columns 0-63, two P buffers in 64-95 and
+// 96-127), and the two score buffers of S = Q K^T use lanes 16-31 (columns 0-63
+// and 64-127). The bias rows then live in a ring of 4 slots that the softmax
+// releases, so S of block i + 2 never waits for O += P V of block i.
+constexpr bool PTMEM = ZEBRA_TC_PTMEM != 0;
+static_assert(!PTMEM || !RSUM_MMA, "P in TMEM keeps the row sums in registers");
 constexpr int THREADS = 192;
-constexpr uint32_t COL_O = 64 * NSBUF;   // O after the score buffers
-constexpr uint32_t TMEM_COLS = COL_O + 64 <= 128 ? 128 : 256;
+constexpr uint32_t COL_O = PTMEM ? 0u : 64 * NSBUF;   // O (TMEM address offset)
+constexpr uint32_t TMEM_COLS = PTMEM || COL_O + 64 <= 128 ? 128 : 256;
+constexpr int PSM = PTMEM ? 0 : PBUF;    // shared-memory P buffers
+constexpr int BST = PTMEM ? 4 : STAGES;  // bias-row slots
+// TMEM address offsets of score buffer b and (PTMEM) P buffer b
+__host__ __device__ constexpr uint32_t s_addr(int b) { return PTMEM ? (16u << 16) + 64u * b : 64u * b; }
+__host__ __device__ constexpr uint32_t p_addr_tmem(int b) { return 64u + 32u * b; }
 constexpr uint32_t LANE_L = 16u << 16;   // TMEM lane offset of the row-sum accumulator L
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
 static_assert(NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
+static_assert(NSBUF <= 2 && PBUF <= 2, "at most two score and P buffers");
 
 struct __align__(1024) Smem {
   __nv_bfloat16 q[64 * 64];
   __nv_bfloat16 k[STAGES][64 * 64];
   __nv_bfloat16 v[STAGES][64 * 64];
-  __nv_bfloat16 p[PBUF][64 * 64];
+  __nv_bfloat16 p[PSM > 0 ? PSM : 1][PSM > 0 ? 64 * 64 : 8];
   __nv_bfloat16 ones[RSUM_MMA ? 16 * 64 : 8];  // B operand of the row-sum MMA (N = 16, K = 64), all 1.0
-  float bias[STAGES][64];       // logit bias row of the block in each stage (log2 units)
-  int all_zero[STAGES];         // 1 when every bias of the stage is 0 (a complete kept tile)
+  float bias[BST][64];          // logit bias row of a block (log2 units)
+  int all_zero[BST];            // 1 when every bias of the row is 0 (a complete kept tile)
   uint64_t q_full;
   uint64_t k_full[STAGES];
   uint64_t k_empty[STAGES];
   uint64_t v_full[STAGES];
   uint64_t v_empty[STAGES];
-  uint64_t b_full[STAGES];      // bias row written
-  uint64_t s_full[NSBUF];
-  uint64_t s_free[NSBUF];
-  uint64_t p_full[PBUF];
-  uint64_t pv_done[PBUF];
+  uint64_t b_full[BST];         // bias row written
+  uint64_t b_empty[BST];        // bias row read by the softmax (PTMEM)
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -359,6 +378,37 @@ __device__ __forceinline__ void mma_pv_only_elect(uint32_t d_o, uint64_t p, uint
       : "memory");
 }
 
+// O += P V with P (the A operand, K-major bf16 pairs) in TMEM at `a_tmem`
+// (8 columns per K = 16 step), V MN-major in shared memory; then commits to
+// `bar0` and `bar1`.
+__device__ __forceinline__ void mma_pv_tmem_elect(uint32_t d_o, uint32_t a_tmem, uint64_t v, uint32_t id_pv,
+                                                  uint32_t acc, uint64_t* bar0, uint64_t* bar1) {
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, %10, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n}\n"
+      ::"r"(d_o), "r"(a_tmem), "r"(a_tmem + 8), "r"(a_tmem + 16), "r"(a_tmem + 24), "l"(v), "l"(v + 128),
+      "l"(v + 256), "l"(v + 384), "r"(id_pv), "r"(acc), "r"(saddr(bar0)), "r"(saddr(bar1))
+      : "memory");
+}
+
+// P of one block (bf16 pairs, this thread's rows g4 and g4 + 8 of its warp's
+// 16, pair j at column 4 j + q4) into TMEM at `taddr` (32 columns)
+__device__ __forceinline__ void tmem_st_p(uint32_t taddr, const uint32_t (&pk)[8][2]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(pk[0][0]), "r"(pk[0][1]), "r"(pk[1][0]), "r"(pk[1][1]), "r"(pk[2][0]), "r"(pk[2][1]), "r"(pk[3][0]),
+      "r"(pk[3][1]), "r"(pk[4][0]), "r"(pk[4][1]), "r"(pk[5][0]), "r"(pk[5][1]), "r"(pk[6][0]), "r"(pk[6][1]),
+      "r"(pk[7][0]), "r"(pk[7][1])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;
   asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
@@ -519,13 +569,14 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
-      mbar_init(&sm.b_full[s], 1);
     }
-    for (int b = 0; b < NSBUF; ++b) {
+    for (int s = 0; s < BST; ++s) {
+      mbar_init(&sm.b_full[s], 1);
+      mbar_init(&sm.b_empty[s], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 2);   // MMA completion + the MMA thread's release after the bias row
       mbar_init(&sm.s_free[b], 4);
-    }
-    for (int b = 0; b < PBUF; ++b) {
       mbar_init(&sm.p_full[b], 4);
       mbar_init(&sm.pv_done[b], 1);
     }
@@ -598,27 +649,38 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (!ok) break;
       tma_load_2d_elect(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
       ++nk;
-      // the V tile and the bias row of this stage are free once PV of block issued - STAGES is done
+      // bias row of the block, two columns per lane, into slot issued % BST
+      auto write_bias = [&]() {
+        const int bs = issued % BST;
+        float b0, b1;
+        if (kind == 1) {
+          b0 = block_bias(a, mrow, t, kind, id, 2 * lane);
+          b1 = block_bias(a, mrow, t, kind, id, 2 * lane + 1);
+        } else {
+          b0 = 2 * lane < nv ? 0.f : -INFINITY;
+          b1 = 2 * lane + 1 < nv ? 0.f : -INFINITY;
+        }
+        *reinterpret_cast<float2*>(&sm.bias[bs][2 * lane]) = make_float2(b0, b1);
+        const int zero = __all_sync(0xffffffffu, b0 == 0.f && b1 == 0.f);
+        __threadfence_block();   // every lane's row entries precede lane 0's release below
+        __syncwarp();
+        if (lane == 0) {
+          sm.all_zero[bs] = zero;
+          mbar_arrive(&sm.b_full[bs]);
+        }
+      };
+      if constexpr (PTMEM) {
+        // the slot is free once the softmax has read the row of block issued - BST
+        if (issued >= BST) ok = mbar_wait_warp(&sm.b_empty[issued % BST], ((issued / BST) - 1) & 1, abort_flag, wl);
+        if (!ok) break;
+        write_bias();
+      }
+      // the V tile (and without PTMEM the bias row) of this stage is free once
+      // PV of block issued - STAGES is done
       if (issued >= STAGES) ok = mbar_wait_warp(&sm.v_empty[s], par, abort_flag, wl);
       if (!ok) break;
       tma_load_2d_elect(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
-      // bias row: two columns per lane
-      float b0, b1;
-      if (kind == 1) {
-        b0 = block_bias(a, mrow, t, kind, id, 2 * lane);
-        b1 = block_bias(a, mrow, t, kind, id, 2 * lane + 1);
-      } else {
-        b0 = 2 * lane < nv ? 0.f : -INFINITY;
-        b1 = 2 * lane + 1 < nv ? 0.f : -INFINITY;
-      }
-      *reinterpret_cast<float2*>(&sm.bias[s][2 * lane]) = make_float2(b0, b1);
-      const int zero = __all_sync(0xffffffffu, b0 == 0.f && b1 == 0.f);
-      __threadfence_block();   // every lane's row entries precede lane 0's release below
-      __syncwarp();
-      if (lane == 0) {
-        sm.all_zero[s] = zero;
-        mbar_arrive(&sm.b_full[s]);
-      }
+      if constexpr (!PTMEM) write_bias();
       ++issued;
     }
     if (lane == 0 && ok && issued == nb) {
@@ -641,8 +703,37 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     const uint64_t dq = desc_k(saddr(sm.q));
     const uint64_t d1 = desc_k(saddr(sm.ones));
     bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag, wl);
+    if constexpr (PTMEM) {
+      // S = Q K^T of block q into score buffer q & 1 (free once the softmax
+      // has loaded S of block q - 2), then the bias forward
+      auto issue_qk = [&](int q) -> bool {
+        const int s = q % STAGES, b = q & 1;
+        if (!mbar_wait_warp(&sm.k_full[s], (q / STAGES) & 1, abort_flag, wl)) return false;
+        if (q >= 2 && !mbar_wait_warp(&sm.s_free[b], ((q >> 1) - 1) & 1, abort_flag, wl)) return false;
+        fence_after();
+        mma_qk_elect(tmem + s_addr(b), dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
+        if (!mbar_wait_warp(&sm.b_full[q % BST], (q / BST) & 1, abort_flag, wl)) return false;
+        if (lane == 0) mbar_arrive(&sm.s_full[b]);
+        __syncwarp();
+        return true;
+      };
+      if (ok && nb > 0) ok = issue_qk(0);
+      if (ok && nb > 1) ok = issue_qk(1);
+      for (int j = 0; ok && j < nb; ++j) {
+        if (j + 2 < nb) ok = issue_qk(j + 2);
+        if (!ok) break;
+        const int s = j % STAGES, b = j & 1;
+        ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag, wl);
+        if (ok) ok = mbar_wait_warp(&sm.p_full[b], (j >> 1) & 1, abort_flag, wl);
+        if (!ok) break;
+        fence_after();
+        // O += P V, P (the A operand) from P buffer b in the accumulator's lanes
+        mma_pv_tmem_elect(tmem + COL_O, tmem + p_addr_tmem(b), desc_mn(saddr(sm.v[s])), id_pv, j > 0 ? 1u : 0u,
+                          &sm.v_empty[s], &sm.pv_done[b]);
+      }
+    }
     int qk = 0;
-    for (int j = 0; ok && j < nb; ++j) {
+    for (int j = 0; !PTMEM && ok && j < nb; ++j) {
       // S = Q K^T up to NSBUF blocks ahead of this PV (a score buffer is
       // reusable as soon as the softmax has loaded it)
       while (qk < nb && qk <= j + NSBUF) {
@@ -654,7 +745,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         mma_qk_elect(tmem + 64u * b, dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
         // forward the stage's bias row to the softmax through s_full: this
         // warp acquires it here and releases it with one arrival
-        ok = mbar_wait_warp(&sm.b_full[s], (qk / STAGES) & 1, abort_flag, wl);
+        ok = mbar_wait_warp(&sm.b_full[qk % BST], (qk / BST) & 1, abort_flag, wl);
         if (!ok) break;
         if (lane == 0) mbar_arrive(&sm.s_full[b]);
         __syncwarp();
@@ -704,11 +795,11 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     }
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
-      const int s = i % STAGES, b = i % NSBUF, pb = i % PBUF;
-      if (!mbar_wait_warp(&sm.s_full[b], (i / NSBUF) & 1, abort_flag, wl)) { ok = false; break; }
+      const int s = i % BST, b = PTMEM ? (i & 1) : i % NSBUF, pb = PTMEM ? (i & 1) : i % PBUF;
+      if (!mbar_wait_warp(&sm.s_full[b], (PTMEM ? (i >> 1) : i / NSBUF) & 1, abort_flag, wl)) { ok = false; break; }
       fence_after();
       float sv[32];
-      tmem_ld64(tmem + lane_off + 64u * b, sv);
+      tmem_ld64(tmem + lane_off + s_addr(b), sv);
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[b]);
@@ -734,6 +825,11 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         }
         mx0 = max_row<0>(sv);
         mx1 = max_row<2>(sv);
+      }
+      if constexpr (PTMEM) {
+        // this warp is done with the block's bias row
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.b_empty[s]);
       }
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -767,27 +863,37 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           p0 = make_float2(fast_exp2(e0.x), fast_exp2(e0.y));
           p1 = make_float2(fast_exp2(e1.x), fast_exp2(e1.y));
         }
-        if (!RSUM_MMA) {
-          ls0 = ffma2(p0, one2, ls0);
-          ls1 = ffma2(p1, one2, ls1);
-        }
         pk[j][0] = pack_bf16(p0.x, p0.y);
         pk[j][1] = pack_bf16(p1.x, p1.y);
+        if (!RSUM_MMA) {
+          // the row sums add exactly the bf16 values that O += P V multiplies
+          ls0 = ffma2(make_float2(__uint_as_float(pk[j][0] << 16), __uint_as_float(pk[j][0] & 0xffff0000u)), one2,
+                      ls0);
+          ls1 = ffma2(make_float2(__uint_as_float(pk[j][1] << 16), __uint_as_float(pk[j][1] & 0xffff0000u)), one2,
+                      ls1);
+        }
       }
       m0 = mn0;
       m1 = mn1;
-      // P buffer pb is free once PV of block i-PBUF has completed
-      if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag, wl)) { ok = false; break; }
-      const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
+      if constexpr (PTMEM) {
+        // P buffer b is free once PV of block i - 2 has read it
+        if (i >= 2 && !mbar_wait_warp(&sm.pv_done[b], ((i >> 1) - 1) & 1, abort_flag, wl)) { ok = false; break; }
+        tmem_st_p(tmem + lane_off + p_addr_tmem(b), pk);
+      } else {
+        // P buffer pb is free once PV of block i-PBUF has completed
+        if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag, wl)) { ok = false; break; }
+        const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        stmatrix4((p_addr ^ ((uint32_t)jj << 5)) + poff, pk[2 * jj][0], pk[2 * jj][1], pk[2 * jj + 1][0],
-                  pk[2 * jj + 1][1]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        for (int jj = 0; jj < 4; ++jj)
+          stmatrix4((p_addr ^ ((uint32_t)jj << 5)) + poff, pk[2 * jj][0], pk[2 * jj][1], pk[2 * jj + 1][0],
+                    pk[2 * jj + 1][1]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
       // rescale O and L (TMEM) when any row of this warp moved its maximum
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
-        if (!mbar_wait_warp(&sm.pv_done[jp % PBUF], (jp / PBUF) & 1, abort_flag, wl)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.pv_done[PTMEM ? (jp & 1) : jp % PBUF], (PTMEM ? (jp >> 1) : jp / PBUF) & 1,
+                            abort_flag, wl)) { ok = false; break; }
         fence_after();
         float o[32];
         tmem_ld64(tmem + lane_off + COL_O, o);
@@ -814,7 +920,10 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
     // ---------------- epilogue ----------------
-    if (ok && nb >= 1 && !mbar_wait_warp(&sm.pv_done[(nb - 1) % PBUF], ((nb - 1) / PBUF) & 1, abort_flag, wl)) ok = false;
+    if (ok && nb >= 1 &&
+        !mbar_wait_warp(&sm.pv_done[PTMEM ? ((nb - 1) & 1) : (nb - 1) % PBUF],
+                        (PTMEM ? ((nb - 1) >> 1) : (nb - 1) / PBUF) & 1, abort_flag, wl))
+      ok = false;
     if (ok) {
       fence_after();
       float o[32];
