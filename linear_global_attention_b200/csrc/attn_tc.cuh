@@ -93,10 +93,11 @@ constexpr int NSBUF = ZEBRA_TC_NSBUF;     // TMEM score buffers (QK^T lookahead)
 constexpr int PBUF = ZEBRA_TC_PBUF;       // shared-memory P buffers (softmax lead over PV)
 constexpr int CTAS_PER_SM = ZEBRA_TC_CTAS;
 #ifndef ZEBRA_TC_RSUM_MMA
-#define ZEBRA_TC_RSUM_MMA 0
+#define ZEBRA_TC_RSUM_MMA 1
 #endif
 // 1: row sums as P x ones MMAs (N = 16) on the tensor cores; 0: in the softmax
-// warps' registers (fp32 sums of the exponentials)
+// warps' registers (sums of the bf16-rounded exponentials: two more integer
+// operations per pair, measured 3% slower than the MMAs)
 constexpr bool RSUM_MMA = ZEBRA_TC_RSUM_MMA != 0;
 #ifndef ZEBRA_TC_EMU
 #define ZEBRA_TC_EMU 0
@@ -119,16 +120,38 @@ static_assert(EMU >= 0 && EMU <= 8, "EMU counts column groups");
 constexpr bool PTMEM = ZEBRA_TC_PTMEM != 0;
 static_assert(!PTMEM || !RSUM_MMA, "P in TMEM keeps the row sums in registers");
 constexpr int THREADS = 192;
-constexpr uint32_t COL_O = PTMEM ? 0u : 64 * NSBUF;   // O (TMEM address offset)
+// O (TMEM address offset): lanes 0-15 from column 0 (PTMEM) or after the
+// first score buffer; a second score buffer without PTMEM uses lanes 16-31 of
+// columns 0-63 (the row-sum accumulator L sits in lanes 16-31 of O's first 16)
+constexpr uint32_t COL_O = PTMEM ? 0u : 64u;
 constexpr uint32_t TMEM_COLS = PTMEM || COL_O + 64 <= 128 ? 128 : 256;
 constexpr int PSM = PTMEM ? 0 : PBUF;    // shared-memory P buffers
-constexpr int BST = PTMEM ? 4 : STAGES;  // bias-row slots
+// The bias rows go to a ring of 4 slots that the softmax releases when S runs
+// two blocks ahead (PTMEM, or two score buffers): the producer then writes a
+// block's row before it waits for a V stage, so S of block i + 2 never waits
+// for O += P V of block i.
+constexpr bool RING = PTMEM || NSBUF == 2;
+constexpr int BST = RING ? 4 : STAGES;  // bias-row slots
+#ifndef ZEBRA_TC_STAGGER
+#define ZEBRA_TC_STAGGER 0
+#endif
+// nanoseconds by which the k-th CTA resident on an SM delays its first copy
+// (k = its launch slot / SM count), to start the CTAs of an SM out of phase
+constexpr int STAGGER_NS = ZEBRA_TC_STAGGER;
+#ifndef ZEBRA_TC_KAHEAD
+#define ZEBRA_TC_KAHEAD 0
+#endif
+// 1: the producer issues the K tile of block i + 1 before the V tile of block
+// i, so a V stage still held by an unfinished O += P V no longer delays the
+// next K tile (needs the bias ring of PTMEM)
+constexpr bool KAHEAD = ZEBRA_TC_KAHEAD != 0;
+static_assert(!KAHEAD || RING, "K ahead of V needs the bias-row ring");
 // TMEM address offsets of score buffer b and (PTMEM) P buffer b
-__host__ __device__ constexpr uint32_t s_addr(int b) { return PTMEM ? (16u << 16) + 64u * b : 64u * b; }
+__host__ __device__ constexpr uint32_t s_addr(int b) { return PTMEM ? (16u << 16) + 64u * b : (uint32_t)b * (16u << 16); }
 __host__ __device__ constexpr uint32_t p_addr_tmem(int b) { return 64u + 32u * b; }
 constexpr uint32_t LANE_L = 16u << 16;   // TMEM lane offset of the row-sum accumulator L
 constexpr unsigned long long DRAIN_NS = 200000000ull;   // 0.2 s while draining after an abort
-static_assert(NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
+static_assert(RING || NSBUF + 1 <= STAGES, "QK^T lookahead needs that many K stages");
 static_assert(NSBUF <= 2 && PBUF <= 2, "at most two score and P buffers");
 
 struct __align__(1024) Smem {
@@ -623,8 +646,9 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
 
   if (warp == 0) {
     // ---------------- producer (whole warp; one elected lane issues) ----------------
-    int issued = 0, nk = 0;   // blocks whose V (and K) copies were issued; K copies issued
+    int issued = 0, nk = 0, nvv = 0;   // blocks taken from the stream; K and V copies issued
     const int inject = *(volatile int*)&g_inject_block;   // error-path test hook (-1: off)
+    if (STAGGER_NS > 0) __nanosleep((unsigned)(STAGGER_NS * (((int)blockIdx.x / 148) & 3)));
     BlockIter it{};
     if constexpr (MODE == 0) {
       tma_load_2d_elect(sm.q, &P.tq, 0, (h * g.T + t) * 64, &sm.q_full);
@@ -637,6 +661,15 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     int kind, id, nv;
     long long keys = 0;   // visible keys per query row (for the logit counter)
     bool ok = true;
+    // V copy of block nvv (its stage's release is that of O += P V of block nvv - STAGES)
+    auto issue_v = [&](int vkind, int vrow) -> bool {
+      const int vs = nvv % STAGES;
+      if (nvv >= STAGES && !mbar_wait_warp(&sm.v_empty[vs], ((nvv / STAGES) - 1) & 1, abort_flag, wl)) return false;
+      tma_load_2d_elect(sm.v[vs], vkind == 0 ? &P.tv : vkind == 1 ? &P.tvl : &P.tvs, 0, vrow, &sm.v_full[vs]);
+      ++nvv;
+      return true;
+    };
+    int pend_kind = -1, pend_row = 0;   // KAHEAD: the block whose V copy is still to be issued
     while (ok && (MODE == 0 ? next_block_sparse(it, g, mrow, t, true, kind, id, nv)
                             : next_block_dense(it, g, sp == 0, kind, id, nv))) {
       // test hook: stop before this block, so the MMA warp's wait for its K tile runs out
@@ -669,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
           mbar_arrive(&sm.b_full[bs]);
         }
       };
-      if constexpr (PTMEM) {
+      if constexpr (RING) {
         // the slot is free once the softmax has read the row of block issued - BST
         if (issued >= BST) ok = mbar_wait_warp(&sm.b_empty[issued % BST], ((issued / BST) - 1) & 1, abort_flag, wl);
         if (!ok) break;
@@ -677,24 +710,31 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       }
       // the V tile (and without PTMEM the bias row) of this stage is free once
       // PV of block issued - STAGES is done
-      if (issued >= STAGES) ok = mbar_wait_warp(&sm.v_empty[s], par, abort_flag, wl);
-      if (!ok) break;
-      tma_load_2d_elect(sm.v[s], kind == 0 ? &P.tv : kind == 1 ? &P.tvl : &P.tvs, 0, row, &sm.v_full[s]);
-      if constexpr (!PTMEM) write_bias();
+      if constexpr (KAHEAD) {
+        if (pend_kind >= 0) ok = issue_v(pend_kind, pend_row);
+        if (!ok) break;
+        pend_kind = kind;
+        pend_row = row;
+      } else {
+        ok = issue_v(kind, row);
+        if (!ok) break;
+      }
+      if constexpr (!RING) write_bias();
       ++issued;
     }
+    if (KAHEAD && ok && pend_kind >= 0) ok = issue_v(pend_kind, pend_row);   // V of the last block
     if (lane == 0 && ok && issued == nb) {
       const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);   // the own-tile extras of the epilogue
       atomicAdd(&g_logits[MODE], (unsigned long long)((long long)n_t * (keys + extra)));
     }
-    if (lane == 0 && (issued < nb || *abort_flag)) {
+    if (lane == 0 && (issued < nb || nvv < nb || *abort_flag)) {
       // stopped early: let the copies already in flight land before the CTA
       // frees its shared memory (the last STAGES copies into each ring are the
       // only ones whose landing nobody may have waited for)
       mbar_drain(&sm.q_full, 0, DRAIN_NS);
       for (int i = nk > STAGES ? nk - STAGES : 0; i < nk; ++i)
         mbar_drain(&sm.k_full[i % STAGES], (i / STAGES) & 1, DRAIN_NS);
-      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+      for (int i = nvv > STAGES ? nvv - STAGES : 0; i < nvv; ++i)
         mbar_drain(&sm.v_full[i % STAGES], (i / STAGES) & 1, DRAIN_NS);
     }
   } else if (warp == 1) {
@@ -742,7 +782,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag, wl);
         if (!ok) break;
         fence_after();
-        mma_qk_elect(tmem + 64u * b, dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
+        mma_qk_elect(tmem + s_addr(b), dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
         // forward the stage's bias row to the softmax through s_full: this
         // warp acquires it here and releases it with one arrival
         ok = mbar_wait_warp(&sm.b_full[qk % BST], (qk / BST) & 1, abort_flag, wl);
@@ -826,7 +866,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         mx0 = max_row<0>(sv);
         mx1 = max_row<2>(sv);
       }
-      if constexpr (PTMEM) {
+      if constexpr (RING) {
         // this warp is done with the block's bias row
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.b_empty[s]);

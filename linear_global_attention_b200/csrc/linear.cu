@@ -639,14 +639,18 @@ __global__ void __launch_bounds__(256) linear_state_simt_kernel(const __grid_con
 // --------------------------------------------------------------------------
 // 2. reduce + fold A: state[h][c][i] = sum_j S[c][j] A[i][j]; state[h][c][64] = z[c]
 // --------------------------------------------------------------------------
+// CTA = (head, 8 channel rows): sums its rows of the chunk partials in chunk
+// order (deterministic), then folds A into them.
+constexpr int RED_ROWS = 8;
 __global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constant__ LinearArgs a, int want_bf16) {
-  __shared__ float S[64][65];
+  __shared__ float S[RED_ROWS][65];
   __shared__ float As[64][65];
-  const int h = blockIdx.x, tid = threadIdx.x;
+  const int h = blockIdx.x, c0 = blockIdx.y * RED_ROWS, tid = threadIdx.x;
   const Geo& g = a.g;
-  for (int e = tid; e < 64 * 65; e += 256) {
+  for (int e = tid; e < RED_ROWS * 65; e += 256) {
     float s = 0.f;
-    for (int ch = 0; ch < a.chunks; ++ch) s += a.part[((size_t)ch * g.H + h) * 64 * 65 + e];
+    const float* p = a.part + ((size_t)h * 64 + c0) * 65 + e;
+    for (int ch = 0; ch < a.chunks; ++ch) s += p[(size_t)ch * g.H * 64 * 65];
     S[e / 65][e % 65] = s;
   }
   for (int e = tid; e < 64 * 64; e += 256) {
@@ -656,13 +660,13 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constan
   __syncthreads();
   float* st = a.state + (size_t)h * 64 * 65;
   __nv_bfloat16* sb = want_bf16 ? static_cast<__nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64 : nullptr;
-  for (int e = tid; e < 64 * NB; e += 256) {
-    const int c = e / NB, i = e % NB;  // channel c, output column i
+  for (int e = tid; e < RED_ROWS * NB; e += 256) {
+    const int r = e / NB, i = e % NB, c = c0 + r;  // channel c, output column i
     float val = 0.f;
     if (i < 64) {
-      for (int j = 0; j < 64; ++j) val = fmaf(S[c][j], As[i][j], val);
+      for (int jj = 0; jj < 64; ++jj) val = fmaf(S[r][jj], As[i][jj], val);
     } else if (i == 64) {
-      val = S[c][64];
+      val = S[r][64];
     }
     if (i <= 64) st[c * 65 + i] = val;
     if (sb) sb[(size_t)i * 64 + c] = __float2bfloat16_rn(val);  // B operand stored [n][k]
@@ -846,7 +850,7 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_state_kernel")) return rc;
   {
     ProfScope prof("linear_reduce", st);
-    linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 1);
+    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), 256, 0, st>>>(a, 1);
   }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
@@ -872,7 +876,7 @@ int launch_linear<float>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_state_simt_kernel")) return rc;
   {
     ProfScope prof("linear_reduce", st);
-    linear_reduce_kernel<<<a.g.H, 256, 0, st>>>(a, 0);
+    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), 256, 0, st>>>(a, 0);
   }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
