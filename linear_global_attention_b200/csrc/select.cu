@@ -11,11 +11,11 @@
 //  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 128x128-tile
 //     fp32 GEMM (K = 64) written to scratch; each score is a fixed-order fma chain.
 //  2. select_kernel: one CTA per row (h, t) loads the row into shared memory as
-//     order-preserving 32-bit keys, finds the k-th largest key with four 8-bit
-//     radix passes (histograms replicated 8 ways to spread same-bin atomics over
-//     banks; in the first pass, whose byte holds the sign and exponent bits,
-//     lanes of a warp that hit the same bin add once), one warp scans the 256
-//     bins for the threshold bin, then emits the bitmask: keys above the threshold, plus the
+//     order-preserving 32-bit keys, finds the k-th largest key from a 2,048-bin
+//     histogram over the row's value range (a non-decreasing bin map; the bin
+//     that holds the k-th key is found by a suffix scan and its keys, at most
+//     1,024, are sorted exactly; rows with a more crowded bin take four 8-bit
+//     radix passes instead), then emits the bitmask: keys above the threshold, plus the
 //     lowest-index keys equal to it (block-wide scan over the mask words).
 //     It also flags near-ties: the k-th and (k+1)-th scores within a relative
 //     gap of 1e-5.
@@ -94,13 +94,18 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 constexpr int SEL_THREADS = 512;
 constexpr int HCOPIES = 8;
 constexpr int HSTRIDE = 257;
+constexpr int VBINS = 2048;      // bins of the value histogram (4 per thread)
+constexpr int CAND_MAX = 1024;   // candidates of the threshold bin sorted exactly
+constexpr int HIST_WORDS = HCOPIES * HSTRIDE > VBINS ? HCOPIES * HSTRIDE : VBINS;
 
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[HCOPIES * HSTRIDE];
-  __shared__ uint32_t s_bin, s_need, s_eqtotal;
+  __shared__ uint32_t hist[HIST_WORDS];
+  __shared__ uint32_t cand[CAND_MAX];
+  __shared__ uint32_t s_bin, s_need, s_eqtotal, s_ncand;
   __shared__ uint32_t s_wsum[SEL_THREADS / 32];
   __shared__ uint32_t s_max[SEL_THREADS / 32];
+  __shared__ float s_vmin[SEL_THREADS / 32], s_vmax[SEL_THREADS / 32];
   const int T = a.g.T, W = a.g.W;
   const int t = blockIdx.x, hh = blockIdx.y, h = a.h0 + hh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -114,80 +119,221 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
     return;
   }
   const float* srow = a.scores + ((size_t)hh * T + t) * a.Tld;
-  for (int i = tid; i < T; i += SEL_THREADS) keys[i] = order_key(srow[i]);
-
-  uint32_t prefix = 0, pmask = 0, need = (uint32_t)a.keep;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < HCOPIES * HSTRIDE; i += SEL_THREADS) hist[i] = 0;
+  float vmin = INFINITY, vmax = -INFINITY;
+  for (int i = tid; i < T; i += SEL_THREADS) {
+    const float v = srow[i];
+    keys[i] = order_key(v);
+    vmin = fminf(vmin, v);
+    vmax = fmaxf(vmax, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  }
+  if (lane == 0) {
+    s_vmin[warp] = vmin;
+    s_vmax[warp] = vmax;
+  }
+  for (int i = tid; i < VBINS; i += SEL_THREADS) hist[i] = 0;
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  vmin = s_vmin[0];
+  vmax = s_vmax[0];
+  for (int w = 1; w < SEL_THREADS / 32; ++w) {
+    vmin = fminf(vmin, s_vmin[w]);
+    vmax = fmaxf(vmax, s_vmax[w]);
+  }
+  // Value histogram: bin(v) = floor((v - vmin) * VBINS / (vmax - vmin)), a
+  // non-decreasing function of v, so every key in a higher bin is larger than
+  // every key in a lower one. The bin that holds the keep-th largest key is
+  // found by a suffix scan; its keys are sorted exactly. Rows whose threshold
+  // bin holds more than CAND_MAX keys (heavy ties) take the radix passes.
+  const float span = vmax - vmin;
+  const float scale = (float)VBINS / span;
+  const bool binned = span > 0.f && isfinite(scale);
+  uint32_t thr = 0, eq_take = 0, eq_total = 0;
+  bool exact = false;
+  if (binned) {
+    for (int i = tid; i < T; i += SEL_THREADS) {
+      const int bin = min(max((int)((key_value(keys[i]) - vmin) * scale), 0), VBINS - 1);
+      atomicAdd(&hist[bin], 1u);
+    }
     __syncthreads();
-    uint32_t* hc = hist + (lane & (HCOPIES - 1)) * HSTRIDE;
-    if (shift == 24) {
-      // the top byte (sign and exponent bits) takes few distinct values: one
-      // atomic per distinct bin per warp (the loop bound is uniform, so the
-      // whole warp takes part in every match)
-      for (int base = 0; base < T; base += SEL_THREADS) {
-        const int i = base + tid;
-        const uint32_t bin = i < T ? keys[i] >> 24 : 256u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-        if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hc[bin], (uint32_t)__popc(peers));
+    // suffix scan over the bins: thread tid owns bins 4 (511 - tid) .. + 3, so
+    // an inclusive prefix scan over tid runs from the top bin down
+    const int b0 = 4 * (SEL_THREADS - 1 - tid);
+    uint32_t c[4], sum = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      c[e] = hist[b0 + 3 - e];
+      sum += c[e];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    uint32_t base = 0;
+    for (int w = 0; w < warp; ++w) base += s_wsum[w];
+    incl += base;
+    const uint32_t excl = incl - sum, need0 = (uint32_t)a.keep;
+    if (excl < need0 && incl >= need0) {
+      uint32_t cum = excl;
+      int b = b0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (cum + c[e] >= need0) {
+          b = b0 + 3 - e;
+          break;
+        }
+        cum += c[e];
       }
-    } else {
+      s_bin = (uint32_t)b;
+      s_need = need0 - cum;
+      s_eqtotal = hist[b];
+    }
+    __syncthreads();
+    const int bsel = (int)s_bin;
+    const uint32_t nbin = s_eqtotal, need_b = s_need;
+    if (nbin <= (uint32_t)CAND_MAX) {
+      // the threshold bin's keys, sorted in descending order (bitonic, padded
+      // with 0, below every order key of a finite score)
       for (int i = tid; i < T; i += SEL_THREADS) {
         const uint32_t k = keys[i];
-        if ((k & pmask) == prefix) atomicAdd(&hc[(k >> shift) & 255u], 1u);
+        if (min(max((int)((key_value(k) - vmin) * scale), 0), VBINS - 1) == bsel) cand[atomicAdd(&s_ncand, 1u)] = k;
       }
-    }
-    __syncthreads();
-    if (tid < 256) {
-      uint32_t s = 0;
-#pragma unroll
-      for (int c = 0; c < HCOPIES; ++c) s += hist[c * HSTRIDE + tid];
-      hist[tid] = s;  // copy 0 slot tid: read by this thread only above
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // the bin holding the need-th largest key: lane l owns bins 255 - 8 l
-      // down to 248 - 8 l; an inclusive scan over the lanes (high bins first)
-      // finds the lane where the running count reaches need
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = hist[255 - 8 * lane - e];
-        sum += c[e];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t excl = incl - sum;
-      const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
-      if (lane == __ffs(hit) - 1) {
-        uint32_t cum = excl;
-        int b = 255 - 8 * lane - 7;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (cum + c[e] >= need) {
-            b = 255 - 8 * lane - e;
-            break;
+      __syncthreads();
+      int np = 1;
+      while (np < (int)nbin) np <<= 1;
+      for (int i = (int)nbin + tid; i < np; i += SEL_THREADS) cand[i] = 0u;
+      __syncthreads();
+      for (int kk = 2; kk <= np; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+          for (int i = tid; i < np; i += SEL_THREADS) {
+            const int l = i ^ jj;
+            if (l > i) {
+              const uint32_t x = cand[i], y = cand[l];
+              const bool desc = (i & kk) == 0;
+              if (desc ? x < y : x > y) {
+                cand[i] = y;
+                cand[l] = x;
+              }
+            }
           }
-          cum += c[e];
+          __syncthreads();
         }
-        s_bin = (uint32_t)b;
-        s_need = need - cum;
-        s_eqtotal = hist[b];
       }
+      thr = cand[need_b - 1];
+      // keys equal to the threshold: how many the bin holds, how many are taken
+      uint32_t gt = 0, eq = 0;
+      for (int i = tid; i < (int)nbin; i += SEL_THREADS) {
+        gt += cand[i] > thr ? 1u : 0u;
+        eq += cand[i] == thr ? 1u : 0u;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        gt += __shfl_xor_sync(0xffffffffu, gt, o);
+        eq += __shfl_xor_sync(0xffffffffu, eq, o);
+      }
+      __syncthreads();   // s_wsum / s_max are reused below
+      if (lane == 0) {
+        s_wsum[warp] = gt;
+        s_max[warp] = eq;
+      }
+      __syncthreads();
+      gt = 0;
+      eq = 0;
+      for (int w = 0; w < SEL_THREADS / 32; ++w) {
+        gt += s_wsum[w];
+        eq += s_max[w];
+      }
+      eq_take = need_b - gt;
+      eq_total = eq;
+      exact = true;
     }
-    __syncthreads();
-    prefix |= s_bin << shift;
-    pmask |= 255u << shift;
-    need = s_need;
     __syncthreads();
   }
-  const uint32_t thr = prefix;          // the k-th largest key
-  const uint32_t eq_take = need;        // how many keys equal to thr are kept (lowest index first)
-  const uint32_t eq_total = s_eqtotal;  // how many keys equal thr
+  if (!exact) {
+    // radix passes over the whole row (all scores equal, or a crowded bin)
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)a.keep;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < HCOPIES * HSTRIDE; i += SEL_THREADS) hist[i] = 0;
+      __syncthreads();
+      uint32_t* hc = hist + (lane & (HCOPIES - 1)) * HSTRIDE;
+      if (shift == 24) {
+        // the top byte (sign and exponent bits) takes few distinct values: one
+        // atomic per distinct bin per warp (the loop bound is uniform, so the
+        // whole warp takes part in every match)
+        for (int base = 0; base < T; base += SEL_THREADS) {
+          const int i = base + tid;
+          const uint32_t bin = i < T ? keys[i] >> 24 : 256u;
+          const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+          if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hc[bin], (uint32_t)__popc(peers));
+        }
+      } else {
+        for (int i = tid; i < T; i += SEL_THREADS) {
+          const uint32_t k = keys[i];
+          if ((k & pmask) == prefix) atomicAdd(&hc[(k >> shift) & 255u], 1u);
+        }
+      }
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t sum = 0;
+#pragma unroll
+        for (int c = 0; c < HCOPIES; ++c) sum += hist[c * HSTRIDE + tid];
+        hist[tid] = sum;  // copy 0 slot tid: read by this thread only above
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // the bin holding the need-th largest key: lane l owns bins 255 - 8 l
+        // down to 248 - 8 l; an inclusive scan over the lanes (high bins first)
+        // finds the lane where the running count reaches need
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[255 - 8 * lane - e];
+          sum += c[e];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - sum;
+        const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
+        if (lane == __ffs(hit) - 1) {
+          uint32_t cum = excl;
+          int b = 255 - 8 * lane - 7;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (cum + c[e] >= need) {
+              b = 255 - 8 * lane - e;
+              break;
+            }
+            cum += c[e];
+          }
+          s_bin = (uint32_t)b;
+          s_need = need - cum;
+          s_eqtotal = hist[b];
+        }
+      }
+      __syncthreads();
+      prefix |= s_bin << shift;
+      pmask |= 255u << shift;
+      need = s_need;
+      __syncthreads();
+    }
+    thr = prefix;
+    eq_take = need;
+    eq_total = s_eqtotal;
+  }
+  // thr: the keep-th largest key; eq_take of the eq_total keys equal to it are
+  // kept, lowest index first
 
   // mask words: thread tid owns a contiguous run of words
   const int per = (W + SEL_THREADS - 1) / SEL_THREADS;

@@ -99,6 +99,45 @@ def test_select_ties_go_to_the_lower_index():
     assert nt.all()                # a full tie is a near-tie
 
 
+@pytest.mark.parametrize("tied", [3000, 700], ids=["crowded_bin", "exact_ties"])
+def test_select_threshold_ties(tied):
+    """Key means built so that `tied` key tiles score exactly the same for every
+    query tile and the keep-th score falls inside that group: the group lands in
+    one histogram bin (more than 1,024 keys: the radix passes; fewer: the exact
+    sort of the bin), and equal scores must go to the lower tile index on both
+    sides. The other key tiles score far from the tied value, so the
+    comparison is exact for every row."""
+    g = Geom(60, 64, 64, 1)                       # 3,840 tiles (only the geometry matters here)
+    T = g.n_tiles
+    rng = np.random.default_rng(61)
+    q_mean = np.abs(rng.standard_normal((1, T, 64))).astype(np.float32) + 0.5
+    base = np.full(64, 0.25, np.float32)
+    k_mean = np.empty((1, T, 64), np.float32)
+    order = rng.permutation(T)
+    tied_idx, rest = order[:tied], order[tied:]
+    k_mean[0, tied_idx] = base                      # identical key means: identical scores
+    hi = rest[: (T - tied) // 2]
+    lo = rest[(T - tied) // 2:]
+    k_mean[0, hi] = base + 1.0 + rng.random((len(hi), 64)).astype(np.float32)   # clearly above
+    k_mean[0, lo] = base - 1.0 - rng.random((len(lo), 64)).astype(np.float32)   # clearly below
+    keep = len(hi) + tied // 3                      # the cut falls inside the tied group
+    y = 1.0 - (keep - 0.5) / T
+    assert oracle.keep_count(y, T) == keep
+    zg = ph.zgeom(g)
+    qd, kd = torch.from_numpy(q_mean).cuda(), torch.from_numpy(k_mean).cuda()
+    mask = torch.empty((1, T, zg.mask_words), dtype=torch.int32, device="cuda")
+    ws = zb.workspace(zg, zb.ZEBRA_OP_SELECT, zb.ZEBRA_BF16, y)
+    got_keep = zb.zebra_tile_select(zg, qd, kd, y, mask, None, ws)
+    torch.cuda.synchronize()
+    assert got_keep == keep
+    gsel = ph.unpack_mask(mask, T)[0]
+    want, _ = oracle.select_tiles(q_mean[0].astype(np.float64), k_mean[0].astype(np.float64), keep)
+    assert (gsel == want).all()
+    # the tie rule: exactly the lowest-index members of the tied group are kept
+    first = np.sort(tied_idx)[: keep - len(hi)]
+    assert gsel[:, first].all() and not gsel[:, np.setdiff1d(tied_idx, first)].any()
+
+
 def test_select_sparse_v32_full():
     w, g = _w("sparse_v32")
     q, k, _ = synth.qkv(w)
