@@ -10,13 +10,15 @@
 // Two kernels per group of heads:
 //  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 128x128-tile
 //     fp32 GEMM (K = 64) written to scratch; each score is a fixed-order fma chain.
-//  2. select_kernel: one CTA per row (h, t) loads the row into shared memory as
+//  2. select_kernel: one CTA per row (h, t) copies the row into shared memory
+//     (16-byte asynchronous copies, all in flight at once) and turns it into
 //     order-preserving 32-bit keys, finds the k-th largest key from a 2,048-bin
 //     histogram over the row's value range (a non-decreasing bin map; the bin
-//     that holds the k-th key is found by a suffix scan and its keys, at most
-//     1,024, are sorted exactly; rows with a more crowded bin take four 8-bit
-//     radix passes instead), then emits the bitmask: keys above the threshold, plus the
-//     lowest-index keys equal to it (block-wide scan over the mask words).
+//     that holds the k-th key is found by a suffix scan; up to 256 of its keys
+//     are ranked in one pass, up to 1,024 sorted; rows with a more crowded bin
+//     take four 8-bit radix passes instead), then emits the bitmask: keys above
+//     the threshold, plus the lowest-index keys equal to it (warp ballots per
+//     mask word, a scan over warps when only some equal keys are kept).
 //     It also flags near-ties: the k-th and (k+1)-th scores within a relative
 //     gap of 1e-5.
 #include "common.cuh"
@@ -26,8 +28,10 @@ namespace zebra {
 
 // CTA = a 128 x 128 tile of S (query tiles t0.., key tiles u0..) of one head;
 // the 64-channel means are staged channel-major in shared memory and every
-// thread accumulates an 8 x 8 block (rows ty + 16 i, columns tx + 16 j) with a
-// fixed-order fma chain over the channels.
+// thread accumulates an 8 x 8 block with a fixed-order fma chain over the
+// channels: rows 4 ty + i and 64 + 4 ty + i, columns 4 tx + j and 64 + 4 tx + j
+// (i, j < 4), so each channel step reads four 16-byte vectors and each output
+// row segment is stored as 16-byte vectors.
 constexpr int SC_TILE = 128;
 constexpr int SC_KC = 32;   // channels staged per step
 __global__ void __launch_bounds__(256) scores_kernel(SelectArgs a) {
@@ -59,10 +63,10 @@ __global__ void __launch_bounds__(256) scores_kernel(SelectArgs a) {
 #pragma unroll 4
     for (int c = 0; c < SC_KC; ++c) {
       float qv[8], kv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qv[i] = sq[c][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) kv[j] = sk[c][tx + 16 * j];
+      *reinterpret_cast<float4*>(qv) = *reinterpret_cast<const float4*>(&sq[c][4 * ty]);
+      *reinterpret_cast<float4*>(qv + 4) = *reinterpret_cast<const float4*>(&sq[c][64 + 4 * ty]);
+      *reinterpret_cast<float4*>(kv) = *reinterpret_cast<const float4*>(&sk[c][4 * tx]);
+      *reinterpret_cast<float4*>(kv + 4) = *reinterpret_cast<const float4*>(&sk[c][64 + 4 * tx]);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -70,14 +74,18 @@ __global__ void __launch_bounds__(256) scores_kernel(SelectArgs a) {
     }
   }
   float* out = a.scores + (size_t)hh * T * a.Tld;
+  // Tld is a multiple of 4, so every 4-column group starts on a 16-byte boundary
+  // and lies wholly inside the row (columns T .. Tld - 1 are padding nobody reads)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int t = t0 + ty + 16 * i;
+    const int t = t0 + 4 * ty + (i & 3) + (i >> 2) * 64;
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int u = u0 + tx + 16 * j;
-      if (u < T) out[(size_t)t * a.Tld + u] = acc[i][j];
+    for (int jh = 0; jh < 2; ++jh) {
+      const int u = u0 + 4 * tx + jh * 64;
+      if (u < a.Tld)
+        *reinterpret_cast<float4*>(out + (size_t)t * a.Tld + u) =
+            make_float4(acc[i][4 * jh], acc[i][4 * jh + 1], acc[i][4 * jh + 2], acc[i][4 * jh + 3]);
     }
   }
 }
@@ -96,13 +104,14 @@ constexpr int HCOPIES = 8;
 constexpr int HSTRIDE = 257;
 constexpr int VBINS = 2048;      // bins of the value histogram (4 per thread)
 constexpr int CAND_MAX = 1024;   // candidates of the threshold bin sorted exactly
+constexpr int RANK_MAX = 256;    // up to this many candidates: ranks by one pass instead of a sort
 constexpr int HIST_WORDS = HCOPIES * HSTRIDE > VBINS ? HCOPIES * HSTRIDE : VBINS;
 
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[HIST_WORDS];
   __shared__ uint32_t cand[CAND_MAX];
-  __shared__ uint32_t s_bin, s_need, s_eqtotal, s_ncand;
+  __shared__ uint32_t s_bin, s_need, s_eqtotal, s_ncand, s_thr, s_gt, s_eqn;
   __shared__ uint32_t s_wsum[SEL_THREADS / 32];
   __shared__ uint32_t s_max[SEL_THREADS / 32];
   __shared__ float s_vmin[SEL_THREADS / 32], s_vmax[SEL_THREADS / 32];
@@ -118,10 +127,20 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
     if (a.near_tie && tid == 0) a.near_tie[(size_t)h * T + t] = 0;
     return;
   }
+  // The row (Tld floats, a multiple of 4 starting on a 16-byte boundary) comes in
+  // as 16-byte asynchronous copies, all in flight at once, and is then turned
+  // into order keys in place.
   const float* srow = a.scores + ((size_t)hh * T + t) * a.Tld;
+  for (int c = tid; c < (a.Tld >> 2); c += SEL_THREADS)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(keys + 4 * c))),
+                 "l"(srow + 4 * c));
+  asm volatile("cp.async.commit_group;\n" ::);
+  asm volatile("cp.async.wait_group 0;\n" ::);
+  __syncthreads();
   float vmin = INFINITY, vmax = -INFINITY;
   for (int i = tid; i < T; i += SEL_THREADS) {
-    const float v = srow[i];
+    const float v = __uint_as_float(keys[i]);
     keys[i] = order_key(v);
     vmin = fminf(vmin, v);
     vmax = fmaxf(vmax, v);
@@ -200,56 +219,81 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
     const int bsel = (int)s_bin;
     const uint32_t nbin = s_eqtotal, need_b = s_need;
     if (nbin <= (uint32_t)CAND_MAX) {
-      // the threshold bin's keys, sorted in descending order (bitonic, padded
-      // with 0, below every order key of a finite score)
       for (int i = tid; i < T; i += SEL_THREADS) {
         const uint32_t k = keys[i];
         if (min(max((int)((key_value(k) - vmin) * scale), 0), VBINS - 1) == bsel) cand[atomicAdd(&s_ncand, 1u)] = k;
       }
       __syncthreads();
-      int np = 1;
-      while (np < (int)nbin) np <<= 1;
-      for (int i = (int)nbin + tid; i < np; i += SEL_THREADS) cand[i] = 0u;
-      __syncthreads();
-      for (int kk = 2; kk <= np; kk <<= 1) {
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-          for (int i = tid; i < np; i += SEL_THREADS) {
-            const int l = i ^ jj;
-            if (l > i) {
-              const uint32_t x = cand[i], y = cand[l];
-              const bool desc = (i & kk) == 0;
-              if (desc ? x < y : x > y) {
-                cand[i] = y;
-                cand[l] = x;
+      uint32_t gt = 0, eq = 0;
+      if (nbin <= (uint32_t)RANK_MAX) {
+        // few candidates: candidate i's rank (larger keys, then equal keys at
+        // lower slots) takes one pass over the candidates, read by all threads
+        // at once; the candidate of rank need_b - 1 is the threshold
+        if (tid < (int)nbin) {
+          const uint32_t x = cand[tid];
+          uint32_t n_gt = 0, n_eq = 0, n_eq_lo = 0;
+          for (int j = 0; j < (int)nbin; ++j) {
+            const uint32_t y = cand[j];
+            n_gt += y > x ? 1u : 0u;
+            n_eq += y == x ? 1u : 0u;
+            n_eq_lo += (y == x && j < tid) ? 1u : 0u;
+          }
+          if (n_gt + n_eq_lo == need_b - 1) {
+            s_thr = x;
+            s_gt = n_gt;
+            s_eqn = n_eq;
+          }
+        }
+        __syncthreads();
+        thr = s_thr;
+        gt = s_gt;
+        eq = s_eqn;
+      } else {
+        // the threshold bin's keys, sorted in descending order (bitonic, padded
+        // with 0, below every order key of a finite score)
+        int np = 1;
+        while (np < (int)nbin) np <<= 1;
+        for (int i = (int)nbin + tid; i < np; i += SEL_THREADS) cand[i] = 0u;
+        __syncthreads();
+        for (int kk = 2; kk <= np; kk <<= 1) {
+          for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < np; i += SEL_THREADS) {
+              const int l = i ^ jj;
+              if (l > i) {
+                const uint32_t x = cand[i], y = cand[l];
+                const bool desc = (i & kk) == 0;
+                if (desc ? x < y : x > y) {
+                  cand[i] = y;
+                  cand[l] = x;
+                }
               }
             }
+            __syncthreads();
           }
-          __syncthreads();
         }
-      }
-      thr = cand[need_b - 1];
-      // keys equal to the threshold: how many the bin holds, how many are taken
-      uint32_t gt = 0, eq = 0;
-      for (int i = tid; i < (int)nbin; i += SEL_THREADS) {
-        gt += cand[i] > thr ? 1u : 0u;
-        eq += cand[i] == thr ? 1u : 0u;
-      }
+        thr = cand[need_b - 1];
+        // keys equal to the threshold: how many the bin holds, how many are taken
+        for (int i = tid; i < (int)nbin; i += SEL_THREADS) {
+          gt += cand[i] > thr ? 1u : 0u;
+          eq += cand[i] == thr ? 1u : 0u;
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        gt += __shfl_xor_sync(0xffffffffu, gt, o);
-        eq += __shfl_xor_sync(0xffffffffu, eq, o);
-      }
-      __syncthreads();   // s_wsum / s_max are reused below
-      if (lane == 0) {
-        s_wsum[warp] = gt;
-        s_max[warp] = eq;
-      }
-      __syncthreads();
-      gt = 0;
-      eq = 0;
-      for (int w = 0; w < SEL_THREADS / 32; ++w) {
-        gt += s_wsum[w];
-        eq += s_max[w];
+        for (int o = 16; o > 0; o >>= 1) {
+          gt += __shfl_xor_sync(0xffffffffu, gt, o);
+          eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        __syncthreads();   // s_wsum / s_max are reused below
+        if (lane == 0) {
+          s_wsum[warp] = gt;
+          s_max[warp] = eq;
+        }
+        __syncthreads();
+        gt = 0;
+        eq = 0;
+        for (int w = 0; w < SEL_THREADS / 32; ++w) {
+          gt += s_wsum[w];
+          eq += s_max[w];
+        }
       }
       eq_take = need_b - gt;
       eq_total = eq;
@@ -335,49 +379,46 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
   // thr: the keep-th largest key; eq_take of the eq_total keys equal to it are
   // kept, lowest index first
 
-  // mask words: thread tid owns a contiguous run of words
-  const int per = (W + SEL_THREADS - 1) / SEL_THREADS;
-  const int w0 = tid * per, w1 = min(W, w0 + per);
-  uint32_t my_eq = 0;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t eqb = 0;
-    for (int j = 0; j < 32; ++j) {
-      const int i = w * 32 + j;
-      if (i < T && keys[i] == thr) eqb |= 1u << j;
+  // mask words: warp w owns a contiguous run of words and reads them a word at a
+  // time, lane j holding key 32 word + j (bank-conflict free); two ballots give
+  // the word's "greater" and "equal" bits.
+  constexpr int NWARP = SEL_THREADS / 32;
+  const int wpw = (W + NWARP - 1) / NWARP;
+  const int wa = min(W, warp * wpw), wb = min(W, wa + wpw);
+  uint32_t before = 0;   // equal keys at lower indices than the current word
+  if (eq_take < eq_total) {
+    // only some equal keys are kept: the lowest-index ones, so each warp needs
+    // the count of equal keys in the words of the warps before it
+    uint32_t cnt = 0;
+    for (int w = wa; w < wb; ++w) {
+      const int i = w * 32 + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, i < T && keys[i] == thr));
     }
-    my_eq += __popc(eqb);
+    if (lane == 0) s_wsum[warp] = cnt;
+    __syncthreads();
+    for (int x = 0; x < warp; ++x) before += s_wsum[x];
   }
-  // exclusive scan of my_eq over threads
-  uint32_t incl = my_eq;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) s_wsum[warp] = incl;
-  __syncthreads();
-  uint32_t base = 0;
-  for (int i = 0; i < warp; ++i) base += s_wsum[i];
-  uint32_t before = base + incl - my_eq;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t gt = 0, eqb = 0;
-    for (int j = 0; j < 32; ++j) {
-      const int i = w * 32 + j;
-      if (i < T) {
-        const uint32_t k = keys[i];
-        if (k > thr) gt |= 1u << j;
-        else if (k == thr) eqb |= 1u << j;
+  for (int w = wa; w < wb; ++w) {
+    const int i = w * 32 + lane;
+    const uint32_t k = i < T ? keys[i] : 0u;
+    const uint32_t gt = __ballot_sync(0xffffffffu, i < T && k > thr);
+    uint32_t eqb = __ballot_sync(0xffffffffu, i < T && k == thr);
+    const uint32_t ne = (uint32_t)__popc(eqb);
+    // with every equal key kept (eq_take >= eq_total) the local count suffices:
+    // it never exceeds the global one, so take == ne
+    uint32_t take = before >= eq_take ? 0u : min(eq_take - before, ne);
+    before += ne;
+    uint32_t keepb = 0;
+    if (take == ne) {
+      keepb = eqb;
+    } else {
+      while (take--) {
+        const uint32_t low = eqb & (~eqb + 1u);
+        keepb |= low;
+        eqb ^= low;
       }
     }
-    uint32_t take = before >= eq_take ? 0u : min(eq_take - before, (uint32_t)__popc(eqb));
-    before += __popc(eqb);
-    uint32_t keepb = 0;
-    while (take--) {
-      const uint32_t low = eqb & (~eqb + 1u);
-      keepb |= low;
-      eqb ^= low;
-    }
-    mrow[w] = gt | keepb;
+    if (lane == 0) mrow[w] = gt | keepb;
   }
 
   if (a.near_tie) {
@@ -424,7 +465,7 @@ int launch_scores(const SelectArgs& a, cudaStream_t st) {
 int launch_select(const SelectArgs& a, cudaStream_t st) {
   const int T = a.g.T;
   if (T == 0) return ZEBRA_OK;
-  const size_t smem = (size_t)T * sizeof(uint32_t);
+  const size_t smem = (size_t)a.Tld * sizeof(uint32_t);   // whole 16-byte chunks of the row
   cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SELECT_MAX_T * 4);
   dim3 grid(T, a.hc);
   ProfScope prof("tile_select", st);

@@ -99,14 +99,14 @@ def test_select_ties_go_to_the_lower_index():
     assert nt.all()                # a full tie is a near-tie
 
 
-@pytest.mark.parametrize("tied", [3000, 700], ids=["crowded_bin", "exact_ties"])
+@pytest.mark.parametrize("tied", [3000, 700, 100], ids=["crowded_bin", "sorted_ties", "ranked_ties"])
 def test_select_threshold_ties(tied):
     """Key means built so that `tied` key tiles score exactly the same for every
     query tile and the keep-th score falls inside that group: the group lands in
-    one histogram bin (more than 1,024 keys: the radix passes; fewer: the exact
-    sort of the bin), and equal scores must go to the lower tile index on both
-    sides. The other key tiles score far from the tied value, so the
-    comparison is exact for every row."""
+    one histogram bin (more than 1,024 keys: the radix passes; up to 1,024: the
+    exact sort of the bin; up to 256: the one-pass ranks), and equal scores must
+    go to the lower tile index on both sides. The other key tiles score far from
+    the tied value, so the comparison is exact for every row."""
     g = Geom(60, 64, 64, 1)                       # 3,840 tiles (only the geometry matters here)
     T = g.n_tiles
     rng = np.random.default_rng(61)
