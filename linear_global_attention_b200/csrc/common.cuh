@@ -56,6 +56,8 @@ struct Geo {
   int Tpad;              // T padded to a multiple of 64
   long long N;           // tokens
   FastDiv fTv, fTc;      // division by Tv and Tc
+  FastDiv fL, fWp;       // division by L and Wp
+  int RPV;               // rows per view of the 8-row-granular dense K/V layout (dense_tile_row)
 };
 
 inline Geo make_geo(const zebra_geom& g) {
@@ -73,6 +75,13 @@ inline Geo make_geo(const zebra_geom& g) {
   o.N = (long long)o.V * o.L;
   o.fTv = make_fastdiv((uint32_t)(o.Tv > 0 ? o.Tv : 1));
   o.fTc = make_fastdiv((uint32_t)(o.Tc > 0 ? o.Tc : 1));
+  o.fL = make_fastdiv((uint32_t)(o.L > 0 ? o.L : 1));
+  o.fWp = make_fastdiv((uint32_t)(o.Wp > 0 ? o.Wp : 1));
+  {
+    // every tile but the corner one holds a multiple of 8 tokens (8 x cols or rows x 8)
+    const int rl = o.Hp - TILE * (o.Tr - 1), cl = o.Wp - TILE * (o.Tc - 1);
+    o.RPV = TILE * o.Wp * (o.Tr - 1) + rl * TILE * (o.Tc - 1) + ((rl * cl + 7) & ~7);
+  }
   return o;
 }
 
@@ -90,6 +99,20 @@ __host__ __device__ __forceinline__ TileShape tile_shape(const Geo& g, int u) {
   s.rows = min(TILE, g.Hp - s.r0);
   s.cols = min(TILE, g.Wp - s.c0);
   return s;
+}
+
+// Dense K/V layout of the tcgen05 sparse kernel: per head, the tiles of each
+// view in order, each tile's rows (row-major inside the tile) followed by zero
+// rows up to a multiple of 8 (only the corner tile of a view needs them). Tile
+// u starts at row dense_tile_row(g, u) of its head; a head holds V * RPV rows.
+// All tiles before row band br of a view are full 8-row bands (8 * Wp tokens
+// each), and the tiles before column bc in band br have 8 columns each.
+__host__ __device__ __forceinline__ int dense_tile_row(const Geo& g, int u) {
+  const int view = fdiv(u, g.fTv);
+  const int p = u - view * g.Tv;
+  const int br = fdiv(p, g.fTc), bc = p - br * g.Tc;
+  const int rows = min(TILE, g.Hp - br * TILE);
+  return view * g.RPV + TILE * g.Wp * br + rows * TILE * bc;
 }
 
 // token index of row a (row-major inside the tile) of tile shape s

@@ -14,14 +14,15 @@
 // (S' = S A^T) makes the epilogue one 64x65 contraction per token.
 //
 // Three kernels:
-//  1. state:  per (token chunk, head) CTA: prologue on K in registers (2 threads
-//     per token, 32 channels each), f(K) -> shared as bf16, then
+//  1. state:  per (head, token chunk) CTA: prologue on K in registers (4 threads
+//     per token, 16 channels each), f(K) -> shared as bf16, then
 //     [S | z] += f(K)^T [V | 1] on mma.sync (M = 64 channels, N = 64 + 8 with a
 //     column of ones for z, K = 64 tokens), fp32 partials per chunk.
 //  2. reduce: per head, sums the chunk partials in a fixed order (deterministic),
 //     forms S' = S A^T, and writes the bf16 B operand [S' | z] of the apply kernel.
-//  3. apply:  per (token chunk, head) CTA: prologue on Q, f(Q) [S' | z] on
-//     mma.sync, divide by the z column, add b, store bf16.
+//  3. apply:  per (head, token chunk) CTA: prologue on Q (f(Q) overwrites its
+//     own ring stage), f(Q) [S' | z] on mma.sync, divide by the z column, add b,
+//     store bf16 straight from registers.
 // The fp32 variants run the same three steps with plain fp32 arithmetic.
 #include <math.h>
 
@@ -40,42 +41,16 @@ __device__ __forceinline__ void token_pos(const Geo& g, long long n, bool& speci
   col = special ? 0 : p - (p / g.Wp) * g.Wp;
 }
 
-// Prologue on 32 channels (half 0: channels 0-31, rotated by row; half 1:
-// channels 32-63, rotated by column); the partner half lives in lane ^ 1.
-__device__ __forceinline__ void features_half(float* x, int half, bool special, int row, int col,
-                                              const float2* __restrict__ tab, float eps) {
-  float ss = 0.f;
-#pragma unroll
-  for (int c = 0; c < 32; ++c) ss = fmaf(x[c], x[c], ss);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  const float sc = rsqrtf(ss * (1.0f / D) + eps);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) x[c] *= sc;
-  if (!special) {
-    const int pos = half ? col : row;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float2 cs = tab[pos * 16 + j];
-      const float a = x[j], b = x[j + 16];
-      x[j] = a * cs.x - b * cs.y;
-      x[j + 16] = b * cs.x + a * cs.y;
-    }
-  }
-  float mx = x[0];
-#pragma unroll
-  for (int c = 1; c < 32; ++c) mx = fmaxf(mx, x[c]);
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  float sum = 0.f;
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    x[c] = fast_exp2((x[c] - mx) * LOG2E);
-    sum += x[c];
-  }
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-  const float inv = 1.0f / sum;
-#pragma unroll
-  for (int c = 0; c < 32; ++c) x[c] *= inv;
+// Position j (0 <= j < L) of a token within its view: special token, or patch
+// (row, col). Multiply-shift division; exact for every int32 j and divisor.
+__device__ __forceinline__ void view_pos(const Geo& g, int j, bool& special, int& row, int& col) {
+  special = j < g.S;
+  const int p = special ? 0 : j - g.S;
+  row = fdiv(p, g.fWp);
+  col = p - row * g.Wp;
 }
+// j mod L for 0 <= j < 2^31
+__device__ __forceinline__ int mod_L(const Geo& g, int j) { return j - fdiv(j, g.fL) * g.L; }
 
 // full 64-channel prologue in one thread (fp32 path)
 __device__ __forceinline__ void features_full(float* x, bool special, int row, int col,
@@ -128,51 +103,21 @@ __device__ __forceinline__ void l_mma(float* c, const uint32_t* a, uint32_t b0, 
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void store_row_half_bf16(unsigned char* tile, int row, int half, const float* x) {
-  // 32 channels = 4 chunks of 8, swizzled
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 v;
-    __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) hv[i] = __floats2bfloat162_rn(x[8 * q + 2 * i], x[8 * q + 2 * i + 1]);
-    *reinterpret_cast<uint4*>(tile + lswz(row, half * 4 + q)) = v;
-  }
-}
-
 // --------------------------------------------------------------------------
-// 1. state (bf16)
+// 1/3. state and apply (bf16), four threads per token
 // --------------------------------------------------------------------------
 // Raw bf16 rows of a 64-token block, one 128-byte head slice per token, land in
-// a 3-deep ring of swizzled shared tiles through cp.async, two blocks ahead of
-// the block being computed (padding tokens are zero-filled).
+// a ring of swizzled shared tiles through cp.async (padding tokens are
+// zero-filled): 3 stages of K and V in the state kernel, LA_STAGES of Q in the
+// apply kernel, each refilled once every warp is done with the block it held.
 constexpr int LSTAGES = 3;
-
-__device__ __forceinline__ void fetch_rows(uint32_t tile, const __nv_bfloat16* base, long long nb, long long n1,
-                                           long long ts, int tok, int half) {
-  const long long n = nb + tok;
-  const bool ok = n < n1;
-  const __nv_bfloat16* p = base + (ok ? n : 0) * ts + half * 32;
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, half * 4 + q)),
-                 "l"(p + 8 * q), "r"(ok ? 16 : 0));
-}
-
-// this thread's 32 channels of its token, from a swizzled raw tile
-__device__ __forceinline__ void read_half(const unsigned char* tile, int tok, int half, float* x) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 w = *reinterpret_cast<const uint4*>(tile + lswz(tok, half * 4 + q));
-    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(hv[e]);
-      x[8 * q + 2 * e] = f.x;
-      x[8 * q + 2 * e + 1] = f.y;
-    }
-  }
-}
+#ifndef ZEBRA_LIN_ASTAGES
+#define ZEBRA_LIN_ASTAGES 4
+#endif
+constexpr int LA_STAGES = ZEBRA_LIN_ASTAGES;   // Q ring depth of the apply kernel
+#ifndef ZEBRA_LIN_STAGED_OUT
+#define ZEBRA_LIN_STAGED_OUT 1   // apply: output through shared memory (1) or from registers (0)
+#endif
 
 struct StateSmem {
   unsigned char phi[64 * 128];
@@ -180,109 +125,6 @@ struct StateSmem {
   unsigned char v[LSTAGES][64 * 128];
 };
 
-__global__ void __launch_bounds__(128, 4) linear_state_kernel(const __grid_constant__ LinearArgs a) {
-  extern __shared__ __align__(128) unsigned char state_smem[];
-  StateSmem& ss = *reinterpret_cast<StateSmem*>(state_smem);
-  unsigned char* phi_s = ss.phi;
-  auto& k_s = ss.k;
-  auto& v_s = ss.v;
-  const Geo& g = a.g;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // grid (head, chunk): the CTAs resident together cover all heads of the same
-  // tokens, so their 128-byte head slices of each token row are fetched together
-  const int h = blockIdx.x;
-  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
-  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
-  const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
-  const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v) + (long long)h * a.hs;
-  const int tok = tid >> 1, half = tid & 1;
-
-  float acc[9][4];
-#pragma unroll
-  for (int j = 0; j < 9; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  const int g4 = lane >> 2;
-  const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
-
-  const int nblk = (int)((n1 - n0 + 63) / 64);
-  for (int i = 0; i < LSTAGES - 1; ++i) {
-    if (i < nblk) {
-      fetch_rows(lsmem(k_s[i]), K, n0 + 64LL * i, n1, a.ts, tok, half);
-      fetch_rows(lsmem(v_s[i]), Vt, n0 + 64LL * i, n1, a.ts, tok, half);
-    }
-    asm volatile("cp.async.commit_group;\n" ::);
-  }
-  for (int i = 0; i < nblk; ++i) {
-    const int st = i % LSTAGES;
-    __syncthreads();   // every warp is done with the stage refilled below and with phi_s
-    {
-      const int f = i + LSTAGES - 1;
-      if (f < nblk) {
-        fetch_rows(lsmem(k_s[f % LSTAGES]), K, n0 + 64LL * f, n1, a.ts, tok, half);
-        fetch_rows(lsmem(v_s[f % LSTAGES]), Vt, n0 + 64LL * f, n1, a.ts, tok, half);
-      }
-      asm volatile("cp.async.commit_group;\n" ::);
-    }
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));   // block i has landed (own copies)
-    __syncthreads();                                                 // ... and everyone's
-    const long long n = n0 + 64LL * i + tok;
-    const bool valid = n < n1;
-    float x[32];
-    read_half(k_s[st], tok, half, x);
-    {
-      // every lane runs the prologue (it shuffles with lane ^ 1); padding tokens are zeroed after
-      bool sp;
-      int row, col;
-      token_pos(g, valid ? n : 0, sp, row, col);
-      features_half(x, half, sp, row, col, a.rope, a.eps);
-      if (!valid) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = 0.f;
-      }
-    }
-    store_row_half_bf16(phi_s, tok, half, x);
-    __syncthreads();
-    const uint32_t vb = lsmem(v_s[st]);
-    // [S | z] (rows = channels 16*warp..) += phi^T [V | 1]
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {  // 16 tokens per k-step
-      uint32_t af[4];
-      {
-        // A = phi^T: 8x8 blocks [tok, ch] read transposed
-        const int mi = lane >> 3, ri = lane & 7;
-        const int trow = ks * 16 + (mi >> 1) * 8 + ri;   // token
-        const int chk = warp * 2 + (mi & 1);             // channel chunk
-        l_ldsm_x4_t(lsmem(phi_s) + lswz(trow, chk), af[0], af[1], af[2], af[3]);
-      }
-#pragma unroll
-      for (int dp = 0; dp < 4; ++dp) {
-        const int mi = lane >> 3, ri = lane & 7;
-        const int trow = ks * 16 + (mi & 1) * 8 + ri;
-        uint32_t b0, b1, b2, b3;
-        l_ldsm_x4_t(vb + lswz(trow, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-        l_mma(acc[2 * dp], af, b0, b1);
-        l_mma(acc[2 * dp + 1], af, b2, b3);
-      }
-      l_mma(acc[8], af, ones, ones);
-    }
-  }
-  asm volatile("cp.async.wait_group 0;\n" ::);
-  // write partial [64][65]: row = channel, col = 0..63 (S), 64 (z)
-  float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
-  const int q4 = lane & 3;
-#pragma unroll
-  for (int j = 0; j < 9; ++j) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int r = warp * 16 + g4 + (e >> 1) * 8;
-      const int c = 8 * j + 2 * q4 + (e & 1);
-      if (c <= 64) part[r * 65 + c] = acc[j][e];
-    }
-  }
-}
-
-// --------------------------------------------------------------------------
-// 1'/3'. state and apply (bf16), four threads per token
-// --------------------------------------------------------------------------
 // 256 threads, 64 tokens per step. Thread (tok = tid / 4, part = tid % 4) owns
 // 16 channels of its token that form 8 whole rotation pairs: half = part / 2
 // (channels 0-31 turn by patch row, 32-63 by column), sub = part % 2 (pairs
@@ -305,12 +147,17 @@ __device__ __forceinline__ void fetch_rows_q4(uint32_t tile, const __nv_bfloat16
                "r"(ok ? 16 : 0));
 }
 
-// f(x) on this thread's 16 channels (xa: the "a" channels, xb: their partners)
+// f(x) on this thread's 16 channels (xa: the "a" channels, xb: their partners).
+// The sums and the maximum are short trees over independent partials, so the
+// dependent chains stay a few operations deep.
 __device__ __forceinline__ void features_q4(float* xa, float* xb, int half, int sub, bool special, int row, int col,
                                             const float2* __restrict__ tab, float eps) {
-  float ss = 0.f;
+  float s4[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) ss = fmaf(xa[e], xa[e], fmaf(xb[e], xb[e], ss));
+  for (int e = 0; e < 4; ++e) s4[e] = fmaf(xa[e], xa[e], xa[e + 4] * xa[e + 4]);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s4[e] = fmaf(xb[e], xb[e], fmaf(xb[e + 4], xb[e + 4], s4[e]));
+  float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   ss += __shfl_xor_sync(0xffffffffu, ss, 2);
   const float sc = rsqrtf(ss * (1.0f / D) + eps);
@@ -329,19 +176,21 @@ __device__ __forceinline__ void features_q4(float* xa, float* xb, int half, int 
       xb[e] = b * cs.x + a * cs.y;
     }
   }
-  float mx = fmaxf(xa[0], xb[0]);
+  float m4[4];
 #pragma unroll
-  for (int e = 1; e < 8; ++e) mx = fmaxf(mx, fmaxf(xa[e], xb[e]));
+  for (int e = 0; e < 4; ++e) m4[e] = fmaxf(fmaxf(xa[e], xa[e + 4]), fmaxf(xb[e], xb[e + 4]));
+  float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   const float off = -mx * LOG2E;
-  float sum = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     xa[e] = fast_exp2(fmaf(xa[e], LOG2E, off));
     xb[e] = fast_exp2(fmaf(xb[e], LOG2E, off));
-    sum += xa[e] + xb[e];
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s4[e] = (xa[e] + xa[e + 4]) + (xb[e] + xb[e + 4]);
+  float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   const float inv = 1.0f / sum;
@@ -402,6 +251,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
 
   const int nblk = (int)((n1 - n0 + 63) / 64);
+  int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LSTAGES - 1; ++i) {
     if (i < nblk) {
       fetch_rows_q4(lsmem(ss.k[i]), K, n0 + 64LL * i, n1, a.ts, tok, half, sub);
@@ -411,7 +261,10 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   }
   for (int i = 0; i < nblk; ++i) {
     const int st = i % LSTAGES;
-    __syncthreads();   // every warp is done with the stage refilled below and with phi
+    // Block i's copies are the oldest but LSTAGES - 2 groups in flight. After the barrier every
+    // warp is done with block i - 1 (its stage and phi), so that stage is refilled only now.
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 2));
+    __syncthreads();
     {
       const int f = i + LSTAGES - 1;
       if (f < nblk) {
@@ -420,8 +273,6 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
       }
       asm volatile("cp.async.commit_group;\n" ::);
     }
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
-    __syncthreads();
     const long long n = n0 + 64LL * i + tok;
     const bool valid = n < n1;
     float xa[8], xb[8];
@@ -429,7 +280,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
     {
       bool sp;
       int row, col;
-      token_pos(g, valid ? n : 0, sp, row, col);
+      view_pos(g, mod_L(g, jb + tok), sp, row, col);
+      jb = mod_L(g, jb + 64);
       features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
       if (!valid) {
 #pragma unroll
@@ -475,10 +327,10 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
 }
 
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ LinearArgs a) {
-  __shared__ __align__(128) unsigned char phi_s[64 * 128];   // f(Q) block, then the bf16 output block
-  __shared__ __align__(128) unsigned char q_s[LSTAGES][64 * 128];
+  // Q ring; f(Q) of a block overwrites its own stage in place (each thread rewrites exactly the
+  // 32 bytes it read), so the MMA reads its A operand from the stage.
+  __shared__ __align__(128) unsigned char q_s[LA_STAGES][64 * 128];
   __shared__ __align__(128) unsigned char b_s[NB * 128];
-  __shared__ float den_s[64];
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
@@ -502,21 +354,23 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
   const int nblk = (int)((n1 - n0 + 63) / 64);
-  for (int i = 0; i < LSTAGES - 1; ++i) {
+  int jb = (int)(n0 % g.L);   // view position of the current block's first token
+  for (int i = 0; i < LA_STAGES - 1; ++i) {
     if (i < nblk) fetch_rows_q4(lsmem(q_s[i]), Q, n0 + 64LL * i, n1, a.ts, tok, half, sub);
     asm volatile("cp.async.commit_group;\n" ::);
   }
   for (int i = 0; i < nblk; ++i) {
-    const int st = i % LSTAGES;
+    const int st = i % LA_STAGES;
     const long long nb = n0 + 64LL * i;
-    __syncthreads();   // the stage refilled below and phi_s (last block's output) are free
+    // Block i's copies are the oldest but LA_STAGES - 2 groups in flight. After the barrier every
+    // warp is done with block i - 1, whose stage is refilled only now.
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
+    __syncthreads();
     {
-      const int f = i + LSTAGES - 1;
-      if (f < nblk) fetch_rows_q4(lsmem(q_s[f % LSTAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+      const int f = i + LA_STAGES - 1;
+      if (f < nblk) fetch_rows_q4(lsmem(q_s[f % LA_STAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half, sub);
       asm volatile("cp.async.commit_group;\n" ::);
     }
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
-    __syncthreads();
     const long long n = nb + tok;
     const bool valid = n < n1;
     float xa[8], xb[8];
@@ -524,13 +378,15 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     {
       bool sp;
       int row, col;
-      token_pos(g, valid ? n : 0, sp, row, col);
+      view_pos(g, mod_L(g, jb + tok), sp, row, col);
+      jb = mod_L(g, jb + 64);
       features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
       if (!valid) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
       }
     }
+    unsigned char* phi_s = q_s[st];
     store_q4(phi_s, tok, half, sub, xa, xb);
     __syncthreads();
     float acc[5][4];
@@ -553,23 +409,22 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
         l_mma(acc[2 * n2], af, b0, b1);
         l_mma(acc[2 * n2 + 1], af, b2, b3);
       }
-      if (grp == 0) {
+      {   // the z column: both column groups compute it, so no exchange is needed
         const int mi = (lane >> 3) & 1, ri = lane & 7;
         uint32_t b0, b1;
         l_ldsm_x2(lsmem(b_s) + lswz(64 + ri, 2 * ks + mi), b0, b1);
         l_mma(acc[4], af, b0, b1);
       }
     }
-    // the z column (column 64: acc[4][0] / acc[4][2] of the q4 == 0 lanes of group 0) to shared memory
-    if (grp == 0 && q4 == 0) {
-      den_s[mrow * 16 + g4] = acc[4][0];
-      den_s[mrow * 16 + g4 + 8] = acc[4][2];
-    }
-    __syncthreads();   // den_s written; every warp has read phi_s: reuse it for the output block
+    // z = column 64 sits in acc[4][0] (row g4) / acc[4][2] (row g4 + 8) of the quad's first lane.
+#if ZEBRA_LIN_STAGED_OUT
+    // Staged output: every warp is done reading the stage as its A operand, so
+    // the bf16 output block goes there and leaves as whole 128-byte token rows.
+    __syncthreads();
 #pragma unroll
     for (int half2 = 0; half2 < 2; ++half2) {
       const int r = mrow * 16 + g4 + half2 * 8;
-      const float il = 1.0f / den_s[r];
+      const float il = 1.0f / __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
@@ -578,7 +433,6 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       }
     }
     __syncthreads();
-    // 64 tokens x 128 bytes, written as whole 16-byte chunks of each token's head row
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int idx = tid + LQ_THREADS * c, r = idx >> 3, ch = idx & 7;
@@ -588,6 +442,40 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
             *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
     }
   }
+#else
+    // Output from registers: each quad transposes its 4 x 4 words so that lane q4 owns chunk
+    // 4 grp + q4 of both rows and stores it as one 16-byte write (8 rows x 64 bytes per warp store).
+#pragma unroll
+    for (int half2 = 0; half2 < 2; ++half2) {
+      const int r = mrow * 16 + g4 + half2 * 8;
+      const float den = __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3);
+      const float il = 1.0f / den;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
+                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
+        w[j] = *reinterpret_cast<const uint32_t*>(&v2);
+      }
+      // lane q4 holds word q4 of every chunk j; after the exchange it holds all words of chunk q4
+      uint32_t o[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // send w[q4 ^ k] to lane q4 ^ k, receive that lane's w[q4]: word (q4 ^ k) of chunk q4
+        const int sel = q4 ^ k;
+        const uint32_t send = sel == 0 ? w[0] : sel == 1 ? w[1] : sel == 2 ? w[2] : w[3];
+        const uint32_t got = k == 0 ? send : __shfl_xor_sync(0xffffffffu, send, k);
+        if (sel == 0) o[0] = got;
+        if (sel == 1) o[1] = got;
+        if (sel == 2) o[2] = got;
+        if (sel == 3) o[3] = got;
+      }
+      const long long nn = nb + r;
+      if (nn < n1)
+        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + (4 * grp + q4) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+#endif
   asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
@@ -673,122 +561,6 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constan
   }
 }
 
-// --------------------------------------------------------------------------
-// 3. apply (bf16): CTA = 128 threads, 64 tokens per step, state B operand in smem
-// --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128, 4) linear_apply_kernel(const __grid_constant__ LinearArgs a) {
-  __shared__ __align__(128) unsigned char phi_s[64 * 128];   // f(Q) block, then the bf16 output block
-  __shared__ __align__(128) unsigned char q_s[LSTAGES][64 * 128];
-  __shared__ __align__(128) unsigned char b_s[NB * 128];
-  const Geo& g = a.g;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
-  const long long n0 = (long long)blockIdx.y * a.chunk_tokens;
-  const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
-  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q) + (long long)h * a.hs;
-  const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
-  for (int i = tid; i < NB * 8; i += 128) {
-    const int r = i >> 3, c = i & 7;
-    *reinterpret_cast<uint4*>(b_s + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
-  }
-  const int tok = tid >> 1, half = tid & 1;
-  const int g4 = lane >> 2, q4 = lane & 3;
-  float bias[16];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    bias[2 * j] = a.b ? a.b[h * 64 + 8 * j + 2 * q4] : 0.f;
-    bias[2 * j + 1] = a.b ? a.b[h * 64 + 8 * j + 2 * q4 + 1] : 0.f;
-  }
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-  const int nblk = (int)((n1 - n0 + 63) / 64);
-  for (int i = 0; i < LSTAGES - 1; ++i) {
-    if (i < nblk) fetch_rows(lsmem(q_s[i]), Q, n0 + 64LL * i, n1, a.ts, tok, half);
-    asm volatile("cp.async.commit_group;\n" ::);
-  }
-  for (int i = 0; i < nblk; ++i) {
-    const int st = i % LSTAGES;
-    const long long nb = n0 + 64LL * i;
-    __syncthreads();   // the stage refilled below and phi_s (last block's output) are free
-    {
-      const int f = i + LSTAGES - 1;
-      if (f < nblk) fetch_rows(lsmem(q_s[f % LSTAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half);
-      asm volatile("cp.async.commit_group;\n" ::);
-    }
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 1));
-    __syncthreads();
-    const long long n = nb + tok;
-    const bool valid = n < n1;
-    float x[32];
-    read_half(q_s[st], tok, half, x);
-    {
-      bool sp;
-      int row, col;
-      token_pos(g, valid ? n : 0, sp, row, col);
-      features_half(x, half, sp, row, col, a.rope, a.eps);
-      if (!valid) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = 0.f;
-      }
-    }
-    store_row_half_bf16(phi_s, tok, half, x);
-    __syncthreads();
-    float acc[9][4];
-#pragma unroll
-    for (int j = 0; j < 9; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {  // 16 channels per k-step
-      uint32_t af[4];
-      {
-        const int mi = lane >> 3, ri = lane & 7;
-        const int row = warp * 16 + (mi & 1) * 8 + ri;
-        l_ldsm_x4(lsmem(phi_s) + lswz(row, 2 * ks + (mi >> 1)), af[0], af[1], af[2], af[3]);
-      }
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        const int mi = lane >> 3, ri = lane & 7;
-        const int row = np * 16 + (mi >> 1) * 8 + ri;
-        uint32_t b0, b1, b2, b3;
-        l_ldsm_x4(lsmem(b_s) + lswz(row, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-        l_mma(acc[2 * np], af, b0, b1);
-        l_mma(acc[2 * np + 1], af, b2, b3);
-      }
-      {
-        const int mi = (lane >> 3) & 1, ri = lane & 7;
-        uint32_t b0, b1;
-        l_ldsm_x2(lsmem(b_s) + lswz(64 + ri, 2 * ks + mi), b0, b1);
-        l_mma(acc[8], af, b0, b1);
-      }
-    }
-    // column 64 (z . phi) sits in acc[8][0] / acc[8][2] of the q4 == 0 lane of each quad
-    const float den0 = __shfl_sync(0xffffffffu, acc[8][0], lane & ~3);
-    const float den1 = __shfl_sync(0xffffffffu, acc[8][2], lane & ~3);
-    const float i0 = 1.0f / den0, i1 = 1.0f / den1;
-    __syncthreads();   // every warp has read phi_s: reuse it for the output block
-#pragma unroll
-    for (int half2 = 0; half2 < 2; ++half2) {
-      const int r = warp * 16 + g4 + half2 * 8;
-      const float il = half2 ? i1 : i0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
-                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
-        *reinterpret_cast<__nv_bfloat162*>(phi_s + lswz(r, j) + 4 * q4) = v2;
-      }
-    }
-    __syncthreads();
-    // 64 tokens x 128 bytes, written as whole 16-byte chunks of each token's head row
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int idx = tid + 128 * c, r = idx >> 3, ch = idx & 7;
-      const long long nn = nb + r;
-      if (nn < n1)
-        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + ch * 8) =
-            *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
-    }
-  }
-  asm volatile("cp.async.wait_group 0;\n" ::);
-}
-
 // fp32 apply: one thread per token
 __global__ void __launch_bounds__(128) linear_apply_simt_kernel(const __grid_constant__ LinearArgs a) {
   __shared__ float st[64][65];
@@ -829,25 +601,16 @@ int linear_chunks(const Geo& g, int* chunk_tokens) {
   return (int)chunks;
 }
 
-#ifndef ZEBRA_LIN_Q4
-#define ZEBRA_LIN_Q4 1
-#endif
-
 template <>
 int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
   {
     ProfScope prof("linear_state", st);
-    if (ZEBRA_LIN_Q4) {
-      cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
-      linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, sizeof(StateSmem), st>>>(a);
-    } else {
-      cudaFuncSetAttribute(linear_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
-      linear_state_kernel<<<dim3(a.g.H, a.chunks), 128, sizeof(StateSmem), st>>>(a);
-    }
+    cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
+    linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, sizeof(StateSmem), st>>>(a);
   }
   count_launch();
-  if (int rc = check_launch("linear_state_kernel")) return rc;
+  if (int rc = check_launch("linear_state_q4_kernel")) return rc;
   {
     ProfScope prof("linear_reduce", st);
     linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), 256, 0, st>>>(a, 1);
@@ -856,13 +619,10 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
   {
     ProfScope prof("linear_apply", st);
-    if (ZEBRA_LIN_Q4)
-      linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, 0, st>>>(a);
-    else
-      linear_apply_kernel<<<dim3(a.g.H, a.chunks), 128, 0, st>>>(a);
+    linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, 0, st>>>(a);
   }
   count_launch();
-  return check_launch("linear_apply_kernel");
+  return check_launch("linear_apply_q4_kernel");
 }
 
 template <>
