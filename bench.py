@@ -97,7 +97,9 @@ def stage_rates(kern: dict, g, hbm_gbs: float) -> dict:
 
     kern: {name: (records, total_ms)} of the profile report; g: the layer
     geometry (bf16). pool_pack: algorithmic bytes = patch rows of Q, K, V read
-    once; packed [H, T, 64, 64] tiles, fp32 means and landmark rows written.
+    once; packed Q tiles [H, T, 64, 64], K and V in the dense layout of 8-row
+    groups (H x views x rows-per-view rows), fp32 means and landmark rows
+    written.
     tile_scores: 2 * 64 FLOPs per (query tile, key tile) score (fp32 ALU).
     tile_select: the T x T fp32 scores read once per head.
     """
@@ -109,7 +111,11 @@ def stage_rates(kern: dict, g, hbm_gbs: float) -> dict:
     patches = g.views * g.grid_h * g.grid_w
     out = {}
     ms = kern["pool_pack"][1] / layers
-    nbytes = 3 * patches * H * 128 + 3 * H * T * 64 * 128 + 3 * H * T * 64 * 4 + 2 * H * t_pad * 128
+    tr, tc = (g.grid_h + 7) // 8, (g.grid_w + 7) // 8
+    rl, cl = g.grid_h - 8 * (tr - 1), g.grid_w - 8 * (tc - 1)
+    rows_per_view = 8 * g.grid_w * (tr - 1) + rl * 8 * (tc - 1) + (rl * cl + 7) // 8 * 8
+    nbytes = (3 * patches * H * 128 + H * T * 64 * 128 + 2 * H * g.views * rows_per_view * 128
+              + 3 * H * T * 64 * 4 + 2 * H * t_pad * 128)
     gbs = nbytes / (ms / 1e3) / 1e9
     out["pool_pack"] = {"ms_per_layer": round(ms, 3), "bytes_per_layer": nbytes, "gbs": round(gbs, 1),
                         "frac_hbm": round(gbs / hbm_gbs, 4)}

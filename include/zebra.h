@@ -24,7 +24,8 @@
  * Conventions.
  *  - Ownership: the caller owns every buffer; all data pointers are DEVICE
  *    pointers unless stated. The library allocates and frees no memory; scratch
- *    comes from the caller's workspace (size: zebra_workspace_bytes).
+ *    comes from the caller's workspace (size: zebra_workspace_bytes; base
+ *    256-byte aligned, as cudaMalloc returns).
  *  - Streams: each call enqueues its kernels on `stream` (a cudaStream_t passed
  *    as void*; NULL = legacy default stream) and returns without synchronising.
  *  - Errors: argument errors return a nonzero status before anything is enqueued;
@@ -54,7 +55,7 @@ extern "C" {
 #define ZEBRA_OK 0
 #define ZEBRA_ERR_INVALID_ARG 1   /* null pointer, bad size, y outside [0,1), ... */
 #define ZEBRA_ERR_UNSUPPORTED 2   /* d != 64, tile != 8, too many tiles, no sm_100 device */
-#define ZEBRA_ERR_WORKSPACE 3     /* workspace smaller than zebra_workspace_bytes() */
+#define ZEBRA_ERR_WORKSPACE 3     /* workspace smaller than zebra_workspace_bytes() or not 256-byte aligned */
 #define ZEBRA_ERR_CUDA 4          /* a CUDA runtime or cuBLASLt call failed */
 #define ZEBRA_ERR_TIMEOUT 5       /* a device-side bounded wait gave up (sticky) */
 #define ZEBRA_ERR_NUMERIC 6       /* a device-side numerical check failed (sticky): the affine

@@ -1,6 +1,7 @@
 // C ABI of the Zebra3D global-attention library: argument validation,
 // workspace carving and kernel orchestration. See include/zebra.h for the
 // contract of every entry point.
+#include <type_traits>
 #include <math.h>
 #include <string.h>
 
@@ -116,6 +117,14 @@ int check_layout(const zebra_geom* g, zebra_dtype dt, const zebra_layout* lay, l
   const long long vec = 16 / (long long)esize(dt);
   if (*ts < 0 || *hs < 0) return fail(ZEBRA_ERR_INVALID_ARG, "strides must be non-negative");
   if (*ts % vec || *hs % vec) return fail(ZEBRA_ERR_INVALID_ARG, "strides must be multiples of 16 bytes");
+  return ZEBRA_OK;
+}
+
+// Workspaces are carved into 256-byte-aligned pieces that TMA and 16-byte
+// asynchronous copies read, so the base must be 256-byte aligned (cudaMalloc's are).
+static int check_workspace(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(ZEBRA_ERR_WORKSPACE, "workspace not 256-byte aligned");
   return ZEBRA_OK;
 }
 
@@ -306,6 +315,7 @@ static int run_sparse(const Geo& G, const void* q, const void* k, const void* v,
   pa.rope = norm_rope ? w.rope : nullptr;
   pa.eps = eps;
   pa.counts = nullptr;
+  pa.dense_kv = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;   // the tcgen05 kernel's K/V layout
   if (G.T > 0) ZTRY(launch_pool_pack<T>(pa, 3, st));
   SpecialArgs<T> sa{};
   sa.g = G;
@@ -472,7 +482,7 @@ int zebra_tile_select(const zebra_geom* g, const float* q_mean, const float* k_m
   Carver c(workspace);
   SelectWs w;
   carve_select(G, c, w);
-  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_workspace(workspace, ws_bytes, c.used()));
   ZTRY(check_device());
   return run_select(G, q_mean, k_mean, keep, mask, near_tie, w, static_cast<cudaStream_t>(stream));
 }
@@ -497,7 +507,7 @@ int zebra_sparse_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const 
   Carver c(workspace);
   SparseWs w;
   carve_sparse(G, dt, c, w);
-  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_workspace(workspace, ws_bytes, c.used()));
   ZTRY(check_device());
   const int keep = G.T > 0 ? keep_of(y, G.T) : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -523,7 +533,7 @@ int zebra_linear_attn(const zebra_geom* g, zebra_dtype dt, const void* q, const 
   Carver c(workspace);
   LinearWs w;
   carve_linear(G, c, w);
-  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_workspace(workspace, ws_bytes, c.used()));
   ZTRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == ZEBRA_BF16) return run_linear<__nv_bfloat16>(G, q, k, v, ts, hs, A, b, rope_base, eps, out, w, st);
@@ -556,7 +566,7 @@ int zebra_affine_moments(const zebra_geom* g, zebra_dtype dt, const void* x, con
   a.moments = moments;
   Carver c(workspace);
   a.part = c.take<double>((size_t)G.H * a.chunks * AF_STRIDE);
-  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_workspace(workspace, ws_bytes, c.used()));
   ZTRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return dt == ZEBRA_BF16 ? launch_affine_moments<__nv_bfloat16>(a, st) : launch_affine_moments<float>(a, st);
@@ -676,7 +686,7 @@ int zebra_hybrid_layer(const zebra_geom* g, int kind, const void* x, const void*
   Carver c(workspace);
   HybridWs w;
   carve_hybrid(G, kind, c, w);
-  if (!workspace || ws_bytes < c.used()) return fail(ZEBRA_ERR_WORKSPACE, "workspace too small");
+  ZTRY(check_workspace(workspace, ws_bytes, c.used()));
   ZTRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const long long Dm = (long long)G.H * D;

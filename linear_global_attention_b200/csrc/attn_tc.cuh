@@ -5,14 +5,18 @@
 // full softmax interactions, omitted tiles become mean key/value landmarks,
 // special-token keys stay visible and each patch query keeps its self key.
 // Section "Speedup scales with the number of input views": keys and values are
-// packed tile-major, so every kept tile is one contiguous 64x64 block.
+// packed tile-major. Here K and V use a dense layout of 8-row groups (the
+// tile's rows, zero rows up to a multiple of 8), and the kept tiles' groups are
+// packed 8 to a 64-key block, so the 37 x 37 grids' 40- and 25-token edge
+// tiles fill whole blocks instead of leaving masked columns.
 //
 // One CTA = one (query tile, head): a 64-row query block against the stream of
-// 64-key blocks (kept tiles, landmark blocks, special-key blocks) described in
-// attn.cu. The block count is known up front (a pre-pass over the selection
-// row), so only the producer walks the stream. Warp roles:
-//   warp 0      producer: one elected lane issues TMA loads of Q once and of
-//               the K and V tile of every block into rings of STAGES
+// 64-key blocks (packed kept tiles, landmark blocks, special-key blocks)
+// described in attn.cu. The block count is known up front (a pre-pass over the
+// selection row), so only the producer walks the stream. Warp roles:
+//   warp 0      producer: TMA loads of Q once and of the K and V tile of every
+//               block (one 64-row copy, or for packed blocks eight 8-row group
+//               copies from eight lanes) into rings of STAGES
 //               128-byte-swizzled 64x64 bf16 tiles (separate K and V barriers:
 //               QK^T may start as soon as K has landed); the whole warp writes
 //               the block's 64 logit biases (log2 units: 0, ln(n_u) for
@@ -161,7 +165,7 @@ struct __align__(1024) Smem {
   __nv_bfloat16 p[PSM > 0 ? PSM : 1][PSM > 0 ? 64 * 64 : 8];
   __nv_bfloat16 ones[RSUM_MMA ? 16 * 64 : 8];  // B operand of the row-sum MMA (N = 16, K = 64), all 1.0
   float bias[BST][64];          // logit bias row of a block (log2 units)
-  int all_zero[BST];            // 1 when every bias of the row is 0 (a complete kept tile)
+  int all_zero[BST];            // 1 when every bias of the row is 0 (64 real keys, nothing masked)
   uint64_t q_full;
   uint64_t k_full[STAGES];
   uint64_t k_empty[STAGES];
@@ -177,6 +181,7 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort;
   int nblocks;
+  long long own_kv_row;         // packed: the own tile's first K/V row in the dense layout
 };
 // Shared memory per CTA: the layout, padded so that at most CTAS_PER_SM CTAs
 // fit on an SM (their TMEM, CTAS_PER_SM x TMEM_COLS columns, must fit in 512).
@@ -188,7 +193,9 @@ static_assert(SMEM_BYTES * CTAS_PER_SM <= SMEM_CAP, "shared memory layout");
 static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "TMEM columns");
 
 struct alignas(64) Params {
-  CUtensorMap tq, tk, tv, tkl, tvl, tks, tvs, tqs;
+  // 64-row boxes; tkg / tvg: the dense K/V layout with boxes of 8 (m + 1) rows
+  CUtensorMap tq, tkl, tvl, tks, tvs, tqs;
+  CUtensorMap tkg[8], tvg[8];
   AttnArgs a;
   int item0;   // first work item of this launch; CTA b takes item0 + b
 };
@@ -316,6 +323,37 @@ __device__ __forceinline__ void tma_load_2d_elect(void* dst, const CUtensorMap* 
       " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n}\n"
       ::"r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar)), "r"(64 * 64 * 2)
       : "memory");
+}
+
+// One packed 64-row stage from the dense K/V layout: lane p copies piece p of
+// the block (p_ng consecutive 8-row groups from row p_src, through the map
+// whose box is 8 p_ng rows) to groups p_slot.. of the stage; lanes without a
+// piece have p_ng = 0. The pieces, a zero-filled tail piece included (rows
+// wholly outside the tensor), always cover the 8 groups, so lane 0 arms `bar`
+// with the stage's full 8 KB before any copy starts. Every piece lands on a
+// 1024-byte boundary, so the 128-byte swizzle gives the same layout as one
+// 64-row copy.
+__device__ __forceinline__ void tma_load_pieces(void* dst, const CUtensorMap* maps, int p_src, int p_slot, int p_ng,
+                                                uint64_t* bar, int lane) {
+  // one piece of all 8 groups (a whole 64-row tile): lane 0 arms and copies
+  if (__shfl_sync(0xffffffffu, p_ng, 0) == 8) {
+    if (lane == 0) {
+      mbar_expect_tx(bar, 64 * 64 * 2);
+      tma_load_2d(dst, maps + 7, 0, p_src, bar);
+    }
+    __syncwarp();
+    return;
+  }
+  if (lane == 0) mbar_expect_tx(bar, 64 * 64 * 2);
+  __syncwarp();
+  if (p_ng > 0) tma_load_2d(static_cast<unsigned char*>(dst) + p_slot * 1024, maps + (p_ng - 1), 0, p_src, bar);
+  __syncwarp();
+}
+
+// 8-row groups of tile u in the dense K/V layout
+__device__ __forceinline__ int tile_groups(const Geo& g, int u) {
+  const TileShape s = tile_shape(g, u);
+  return (s.rows * s.cols + 7) >> 3;
 }
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -560,7 +598,10 @@ __device__ __forceinline__ int block_row(const Geo& g, int h, int kind, int id) 
 // sp (the key tiles [T sp / splits, T (sp + 1) / splits), plus every special
 // key in split 0); it writes the split's unnormalised output, row maximum and
 // row sum for special_combine_kernel.
-template <int MODE>
+// PACK: the grid has partial tiles, so kept tiles are packed 8 groups to a
+// block; without partial tiles every tile is one whole block (the dense layout
+// then coincides with 64-row tiles) and the packing code is compiled out.
+template <int MODE, bool PACK>
 __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -605,6 +646,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
+    if (MODE == 0 && PACK) sm.own_kv_row = (long long)h * g.V * g.RPV + dense_tile_row(g, t);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the all-ones operand of the row-sum MMA (read by the tensor cores: async proxy)
@@ -614,18 +656,37 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   if (warp == 0) {
     if constexpr (MODE == 0) {
       // pre-pass, lane-parallel: the number of blocks the walk below will
-      // produce (kept tiles, landmark blocks with a visible landmark, special
-      // blocks)
-      int n = 0;
-      for (int w = lane; w < g.W; w += 32) n += __popc(mask_word(mrow, w, g.T));
+      // produce (packed blocks of 8 groups of the kept tiles' rows, landmark
+      // blocks with a visible landmark, special blocks)
+      int ng = 0, nl = 0;
+      for (int w = lane; w < g.W; w += 32) {
+        uint32_t m = mask_word(mrow, w, g.T);
+        if constexpr (PACK) {
+          while (m) {
+            const int b = __ffs(m) - 1;
+            m &= m - 1;
+            ng += tile_groups(g, w * 32 + b);
+          }
+        } else {
+          ng += 8 * __popc(m);
+        }
+      }
       for (int lb = lane; lb < g.Tpad / 64; lb += 32) {
         int nvis;
-        n += lmk_visible(mrow, g, t, lb, nvis) != 0u ? 1 : 0;
+        nl += lmk_visible(mrow, g, t, lb, nvis) != 0u ? 1 : 0;
       }
-      n = __reduce_add_sync(0xffffffffu, n);
-      if (lane == 0) sm.nblocks = n + g.NSp / 64;
+      ng = __reduce_add_sync(0xffffffffu, ng);
+      nl = __reduce_add_sync(0xffffffffu, nl);
+      if (lane == 0) sm.nblocks = (ng + 7) / 8 + nl + g.NSp / 64;
     } else {
-      if (lane == 0) sm.nblocks = (u1 - u0) + (sp == 0 ? g.NSp / 64 : 0);
+      int ng = 0;
+      if constexpr (PACK) {
+        for (int u = u0 + lane; u < u1; u += 32) ng += tile_groups(g, u);
+        ng = __reduce_add_sync(0xffffffffu, ng);
+      } else {
+        ng = 8 * (u1 - u0);
+      }
+      if (lane == 0) sm.nblocks = (ng + 7) / 8 + (sp == 0 ? g.NSp / 64 : 0);
     }
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sm.tmem_base)),
@@ -661,26 +722,101 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     int kind, id, nv;
     long long keys = 0;   // visible keys per query row (for the logit counter)
     bool ok = true;
+    // Key tiles (kind 0) are packed: their rows, in walk order and in the
+    // dense layout's 8-row groups (real rows, then zero rows up to a multiple
+    // of 8), fill the blocks 8 groups at a time, so an edge tile of 40 rows
+    // and a corner tile of 25 share blocks with the next tiles instead of
+    // leaving 24 or 39 masked columns each. For the current block, lane j < 8
+    // holds the count of real rows of group j (gcnt), and lane p the p-th
+    // piece (a run of groups of one tile, or the zero-filled tail): its source
+    // row, first group and group count (p_src, p_slot, p_ng).
+    // cur_row: the current tile's next group (its source row), cur_left: the
+    // tile's real rows from there on (<= 0 once it is used up)
+    int cur_row = 0, cur_left = 0;
+    bool tiles_done = false;
+    int gcnt = 0, p_src = 0, p_slot = 0, p_ng = 0;
+    auto next_block = [&](int& bk, int& bid, int& bnv) -> bool {
+      if (PACK && !tiles_done) {
+        int slot = 0, np = 0;
+        gcnt = 0;
+        p_ng = 0;
+        while (slot < 8) {
+          if (cur_left <= 0) {
+            int k2, i2, n2;
+            const bool more = MODE == 0 ? next_block_sparse(it, g, mrow, t, true, k2, i2, n2)
+                                        : next_block_dense(it, g, sp == 0, k2, i2, n2);
+            if (!more || k2 != 0) {
+              // the first landmark or special block: put it back, the walk
+              // yields it again after the last packed block
+              tiles_done = true;
+              if (more) {
+                if (k2 == 1)
+                  --it.lb;
+                else
+                  --it.sb;
+              }
+              break;
+            }
+            cur_row = h * g.V * g.RPV + dense_tile_row(g, i2);
+            cur_left = n2;
+            keys += n2;
+          }
+          const int take = min(8 - slot, (cur_left + 7) >> 3);
+          const int j = lane - slot;
+          if (j >= 0 && j < take) gcnt = min(8, cur_left - 8 * j);
+          if (lane == np) {
+            p_src = cur_row;
+            p_slot = slot;
+            p_ng = take;
+          }
+          ++np;
+          slot += take;
+          cur_row += 8 * take;
+          cur_left -= 8 * take;
+        }
+        if (slot > 0) {
+          if (slot < 8 && lane == np) {   // zero-filled tail: rows wholly before the tensor
+            p_src = -64;
+            p_slot = slot;
+            p_ng = 8 - slot;
+          }
+          bk = 0;
+          bid = 0;
+          bnv = 0;   // the packed tiles' keys were counted as they were fetched
+          return true;
+        }
+      }
+      const bool more = MODE == 0 ? next_block_sparse(it, g, mrow, t, true, bk, bid, bnv)
+                                  : next_block_dense(it, g, sp == 0, bk, bid, bnv);
+      return more;
+    };
     // V copy of block nvv (its stage's release is that of O += P V of block nvv - STAGES)
-    auto issue_v = [&](int vkind, int vrow) -> bool {
+    auto issue_v = [&](int vkind, int vrow, int vsrc, int vslot, int vng) -> bool {
       const int vs = nvv % STAGES;
       if (nvv >= STAGES && !mbar_wait_warp(&sm.v_empty[vs], ((nvv / STAGES) - 1) & 1, abort_flag, wl)) return false;
-      tma_load_2d_elect(sm.v[vs], vkind == 0 ? &P.tv : vkind == 1 ? &P.tvl : &P.tvs, 0, vrow, &sm.v_full[vs]);
+      if (PACK && vkind == 0)
+        tma_load_pieces(sm.v[vs], P.tvg, vsrc, vslot, vng, &sm.v_full[vs], lane);
+      else
+        tma_load_2d_elect(sm.v[vs], vkind == 0 ? &P.tvg[7] : vkind == 1 ? &P.tvl : &P.tvs, 0, vrow, &sm.v_full[vs]);
       ++nvv;
       return true;
     };
-    int pend_kind = -1, pend_row = 0;   // KAHEAD: the block whose V copy is still to be issued
-    while (ok && (MODE == 0 ? next_block_sparse(it, g, mrow, t, true, kind, id, nv)
-                            : next_block_dense(it, g, sp == 0, kind, id, nv))) {
+    // KAHEAD: the block whose V copy is still to be issued
+    int pend_kind = -1, pend_row = 0, pend_src = 0, pend_slot = 0, pend_ng = 0;
+    while (ok && next_block(kind, id, nv)) {
       // test hook: stop before this block, so the MMA warp's wait for its K tile runs out
       if (issued == inject) break;
       keys += nv;
       const int s = issued % STAGES;
       const uint32_t par = ((issued / STAGES) - 1) & 1;
-      const int row = block_row(g, h, kind, id);
+      // without packing a kept tile's rows start at (h T + id) 64, as in 64-row tiles
+      const int row = kind == 0 && PACK ? 0 : block_row(g, h, kind, id);
       if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag, wl);
       if (!ok) break;
-      tma_load_2d_elect(sm.k[s], kind == 0 ? &P.tk : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
+      if (PACK && kind == 0)
+        tma_load_pieces(sm.k[s], P.tkg, p_src, p_slot, p_ng, &sm.k_full[s], lane);
+      else
+        tma_load_2d_elect(sm.k[s], kind == 0 ? &P.tkg[7] : kind == 1 ? &P.tkl : &P.tks, 0, row, &sm.k_full[s]);
       ++nk;
       // bias row of the block, two columns per lane, into slot issued % BST
       auto write_bias = [&]() {
@@ -689,6 +825,20 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         if (kind == 1) {
           b0 = block_bias(a, mrow, t, kind, id, 2 * lane);
           b1 = block_bias(a, mrow, t, kind, id, 2 * lane + 1);
+        } else if (PACK && kind == 0) {
+          // a block of 64 real keys needs no row: the softmax skips the bias
+          if (__all_sync(0xffffffffu, lane >= 8 || gcnt == 8)) {
+            if (lane == 0) {
+              sm.all_zero[bs] = 1;
+              mbar_arrive(&sm.b_full[bs]);
+            }
+            return;
+          }
+          // columns 2 lane, 2 lane + 1 sit in group lane / 4 at rows (2 lane) % 8, + 1
+          const int vc = __shfl_sync(0xffffffffu, gcnt, lane >> 2);
+          const int c0 = (2 * lane) & 7;
+          b0 = c0 < vc ? 0.f : -INFINITY;
+          b1 = c0 + 1 < vc ? 0.f : -INFINITY;
         } else {
           b0 = 2 * lane < nv ? 0.f : -INFINITY;
           b1 = 2 * lane + 1 < nv ? 0.f : -INFINITY;
@@ -711,18 +861,22 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       // the V tile (and without PTMEM the bias row) of this stage is free once
       // PV of block issued - STAGES is done
       if constexpr (KAHEAD) {
-        if (pend_kind >= 0) ok = issue_v(pend_kind, pend_row);
+        if (pend_kind >= 0) ok = issue_v(pend_kind, pend_row, pend_src, pend_slot, pend_ng);
         if (!ok) break;
         pend_kind = kind;
         pend_row = row;
+        pend_src = p_src;
+        pend_slot = p_slot;
+        pend_ng = p_ng;
       } else {
-        ok = issue_v(kind, row);
+        ok = issue_v(kind, row, p_src, p_slot, p_ng);
         if (!ok) break;
       }
       if constexpr (!RING) write_bias();
       ++issued;
     }
-    if (KAHEAD && ok && pend_kind >= 0) ok = issue_v(pend_kind, pend_row);   // V of the last block
+    if (KAHEAD && ok && pend_kind >= 0)
+      ok = issue_v(pend_kind, pend_row, pend_src, pend_slot, pend_ng);   // V of the last block
     if (lane == 0 && ok && issued == nb) {
       const long long extra = own_kept ? 0 : (n_t > 1 ? 2 : 1);   // the own-tile extras of the epilogue
       atomicAdd(&g_logits[MODE], (unsigned long long)((long long)n_t * (keys + extra)));
@@ -1002,10 +1156,11 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         }
       } else if (!own_kept) {
         // exact self key + landmark of the other n_t - 1 tokens of the own tile
-        const size_t tb = ((size_t)h * g.T + t) * TOK * D;
+        const size_t tb = ((size_t)h * g.T + t) * TOK * D;                                 // Q: 64-row tiles
+        const size_t kb = PACK ? (size_t)sm.own_kv_row * D : tb;                           // K, V
         const __nv_bfloat16* Qp = static_cast<const __nv_bfloat16*>(a.Qp) + tb;
-        const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp) + tb;
-        const __nv_bfloat16* Vp = static_cast<const __nv_bfloat16*>(a.Vp) + tb;
+        const __nv_bfloat16* Kp = static_cast<const __nv_bfloat16*>(a.Kp) + kb;
+        const __nv_bfloat16* Vp = static_cast<const __nv_bfloat16*>(a.Vp) + kb;
         const float* km = a.km + ((size_t)h * g.T + t) * D;
         const float* vm = a.vm + ((size_t)h * g.T + t) * D;
         const float nt = (float)n_t;
@@ -1090,14 +1245,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 map over [rows, 64] with a 64 x 64 box and 128-byte swizzle
-static bool make_map(CUtensorMap* m, const void* base, unsigned long long rows) {
+// 2D bf16 map over [rows, 64] with a 64 x box_rows box and 128-byte swizzle
+static bool make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned box_rows = 64) {
   auto fn = encode_fn();
   if (!fn) return false;
   if (rows == 0) rows = 64;  // never read: keep the encoder happy
   cuuint64_t dims[2] = {64, (cuuint64_t)rows};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1116,15 +1271,20 @@ static int launch_tc(const AttnArgs& a, int mode, cudaStream_t st) {
   p.a = a;
   const unsigned long long tile_rows = (unsigned long long)g.H * g.T * 64;
   const unsigned long long spec_rows = (unsigned long long)g.H * g.NSp;
-  bool ok = make_map(&p.tq, a.Qp, tile_rows) && make_map(&p.tk, a.Kp, tile_rows) && make_map(&p.tv, a.Vp, tile_rows) &&
+  const unsigned long long dense_rows = (unsigned long long)g.H * g.V * g.RPV;   // K, V: dense layout, 8-row groups
+  bool ok = make_map(&p.tq, a.Qp, tile_rows) &&
             make_map(&p.tkl, a.Kl, (unsigned long long)g.H * g.Tpad) &&
             make_map(&p.tvl, a.Vl, (unsigned long long)g.H * g.Tpad) && make_map(&p.tks, a.Ks, spec_rows) &&
             make_map(&p.tvs, a.Vs, spec_rows) && make_map(&p.tqs, a.Qs, spec_rows);
+  for (unsigned m = 0; m < 8 && ok; ++m)
+    ok = make_map(&p.tkg[m], a.Kp, dense_rows, 8 * (m + 1)) && make_map(&p.tvg[m], a.Vp, dense_rows, 8 * (m + 1));
   if (!ok) {
     set_error("cuTensorMapEncodeTiled failed");
     return ZEBRA_ERR_CUDA;
   }
-  auto kern = mode == 0 ? tc::attn_tc_kernel<0> : tc::attn_tc_kernel<1>;
+  const bool pack = (g.Hp % TILE) != 0 || (g.Wp % TILE) != 0;   // partial tiles to pack
+  auto kern = mode == 0 ? (pack ? tc::attn_tc_kernel<0, true> : tc::attn_tc_kernel<0, false>)
+                        : (pack ? tc::attn_tc_kernel<1, true> : tc::attn_tc_kernel<1, false>);
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM_BYTES);
   // Work items go out in launches of one resident wave each. All CTAs of a
   // launch start together and walk their key blocks in ascending order at

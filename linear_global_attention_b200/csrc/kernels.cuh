@@ -11,7 +11,8 @@ struct PoolArgs {
   const T* x[3];        // up to three [N, H, d] inputs (Q, K, V); null = skip
   long long ts, hs;     // token / head strides in elements (shared)
   float* mean[3];       // [H, T, d] fp32 or null
-  T* packed[3];         // [H, T, 64, d] or null
+  T* packed[3];         // [H, T, 64, d] or null; K and V (z = 1, 2) in the dense layout when dense_kv
+  int dense_kv;         // K/V rows at h * V * RPV + dense_tile_row (see common.cuh), zero-padded to 8
   T* lmk[3];            // [H, Tpad, d] landmark rows (mean rounded to T) or null
   int norm_rope[3];     // apply RMS norm (+ rotation when rope != null)
   const float2* rope;   // [maxpos, 16] cos/sin table or null

@@ -12,7 +12,8 @@
 // head and walks the tile's tokens, so a warp reads whole 128-byte head rows
 // and consecutive heads of a token are contiguous: every load is a coalesced
 // 16-byte vector load. The same pass writes the packed tile rows (zero-padded
-// to 64) and, at the end, the fp32 mean and its landmark copy.
+// to 64, or for K and V of the tcgen05 kernel to a multiple of 8 in the dense
+// layout) and, at the end, the fp32 mean and its landmark copy.
 //
 // Optional prologue (stacked sparse/dense layers): RMS-normalise each head row
 // (x / sqrt(mean(x^2) + eps)) and turn channel pairs (j, j+16) of channels 0-31
@@ -73,7 +74,10 @@ __global__ void __launch_bounds__(128) pool_pack_kernel(PoolArgs<T> a) {
   const TileShape s = tile_shape(g, u);
   const int n = s.rows * s.cols;
   const bool nr = a.norm_rope[z] != 0;
-  T* packed = a.packed[z] ? a.packed[z] + (((size_t)hh * g.T + u) * TOK) * D + chunk * P : nullptr;
+  const bool dense = a.dense_kv && z > 0;
+  const size_t prow = dense ? (size_t)hh * g.V * g.RPV + dense_tile_row(g, u) : ((size_t)hh * g.T + u) * TOK;
+  T* packed = a.packed[z] ? a.packed[z] + prow * D + chunk * P : nullptr;
+  const int pad_to = dense ? (n + 7) & ~7 : TOK;   // zero rows after the tile's n rows
 
   float sum[P];
 #pragma unroll
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(128) pool_pack_kernel(PoolArgs<T> a) {
     }
   }
   if (packed && hv)
-    for (int r = n; r < TOK; ++r) store16_zero(packed + (size_t)r * D);
+    for (int r = n; r < pad_to; ++r) store16_zero(packed + (size_t)r * D);
   if (!hv) return;
   const float inv = 1.0f / (float)n;
 #pragma unroll

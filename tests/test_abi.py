@@ -95,6 +95,8 @@ def test_sparse_argument_errors(L):
     assert _sparse(L, _g(), ptr=4100) == zb.ZEBRA_ERR_INVALID_ARG       # misaligned
     assert _sparse(L, _g(), nbytes=16) == zb.ZEBRA_ERR_WORKSPACE
     assert _sparse(L, _g(), ws=0) == zb.ZEBRA_ERR_WORKSPACE
+    assert _sparse(L, _g(), ws=4096 + 16) == zb.ZEBRA_ERR_WORKSPACE       # base not 256-byte aligned
+    assert "aligned" in zb.zebra_last_error()
     bad_layout = zb.Layout(130, 64)
     assert _sparse(L, _g(), layout=ctypes.byref(bad_layout)) == zb.ZEBRA_ERR_INVALID_ARG
     assert "strides" in zb.zebra_last_error()
