@@ -241,31 +241,6 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
-// Slow path of mbar_wait: keep testing until the phase completes, another warp
-// raises the abort flag, or `limit_ns` passes (then record the error status
-// and raise the flag).
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                            unsigned long long limit_ns) {
-  const unsigned long long t0 = gtime();
-  while (true) {
-    if (mbar_try(b, parity)) return true;
-    if (*abort_flag) return false;
-    if (gtime() - t0 > limit_ns) {
-      atomicExch(&g_status, ZEBRA_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
-// Wait for the phase of `parity` to complete; true when it did. `limit_ns` is
-// the kernel's wait limit (g_wait_ns, read once at kernel start).
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          unsigned long long limit_ns) {
-  if (mbar_try(b, parity)) return true;
-  return mbar_wait_slow(b, parity, abort_flag, limit_ns);
-}
-
 // Drain wait after an abort: waits for the phase whatever the abort flag says
 // (copies or MMAs still in flight must land before the CTA frees its shared
 // memory and TMEM), and gives up after `limit_ns`.
@@ -283,10 +258,14 @@ __device__ __noinline__ bool mbar_drain_warp(uint64_t* b, uint32_t parity, unsig
   }
 }
 
-// Whole-warp form (all 32 lanes call it): the result is the same in every lane,
-// so the loops around it stay converged for the elected issues below.
-__device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                                 unsigned long long limit_ns) {
+// Wait (all 32 lanes of a warp) for the phase of `parity` to complete; true
+// when it did. The slow path keeps testing until the phase completes, another
+// warp raises the abort flag, or the kernel's wait limit (g_wait_ns) passes;
+// then it records the error status and raises the flag. The result is the
+// same in every lane, so the loops around it stay converged for the elected
+// issues below.
+__device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+  const unsigned long long limit_ns = *(volatile unsigned long long*)&g_wait_ns;
   const unsigned long long t0 = gtime();
   while (true) {
     if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
@@ -301,10 +280,9 @@ __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* b, uint32_t parity, v
     }
   }
 }
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                               unsigned long long limit_ns) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
   if (__all_sync(0xffffffffu, mbar_try(b, parity))) return true;
-  return mbar_wait_warp_slow(b, parity, abort_flag, limit_ns);
+  return mbar_wait_warp_slow(b, parity, abort_flag);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -624,7 +602,6 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
   }
   const uint32_t* mrow = MODE == 0 ? a.mask + ((size_t)h * g.T + t) * g.W : nullptr;
   volatile int* abort_flag = &sm.abort;
-  const unsigned long long wl = *(volatile unsigned long long*)&g_wait_ns;   // limit of every wait
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
@@ -742,24 +719,33 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         p_ng = 0;
         while (slot < 8) {
           if (cur_left <= 0) {
-            int k2, i2, n2;
-            const bool more = MODE == 0 ? next_block_sparse(it, g, mrow, t, true, k2, i2, n2)
-                                        : next_block_dense(it, g, sp == 0, k2, i2, n2);
-            if (!more || k2 != 0) {
-              // the first landmark or special block: put it back, the walk
-              // yields it again after the last packed block
-              tiles_done = true;
-              if (more) {
-                if (k2 == 1)
-                  --it.lb;
-                else
-                  --it.sb;
+            // the next kept tile (MODE 1: the next tile of the key split)
+            int u;
+            bool more;
+            if constexpr (MODE == 0) {
+              while (it.bits == 0 && it.w + 1 < g.W) {
+                ++it.w;
+                it.bits = it.nxt;
+                it.nxt = it.w + 1 < g.W ? mask_word(mrow, it.w + 1, g.T) : 0u;
               }
+              more = it.bits != 0;
+              u = it.w * 32 + __ffs(it.bits) - 1;
+              it.bits &= it.bits - 1;
+            } else {
+              more = it.w < it.t_end;
+              u = it.w++;
+            }
+            if (!more) {
+              // the tiles are done: the walk goes on with the landmark
+              // (MODE 0) or special blocks
+              tiles_done = true;
+              it.phase = MODE == 0 ? 1 : 2;
               break;
             }
-            cur_row = h * g.V * g.RPV + dense_tile_row(g, i2);
-            cur_left = n2;
-            keys += n2;
+            const TileShape sh = tile_shape(g, u);
+            cur_row = h * g.V * g.RPV + sh.view * g.RPV + TILE * g.Wp * (sh.r0 / TILE) + sh.rows * sh.c0;
+            cur_left = sh.rows * sh.cols;
+            keys += cur_left;
           }
           const int take = min(8 - slot, (cur_left + 7) >> 3);
           const int j = lane - slot;
@@ -793,7 +779,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     // V copy of block nvv (its stage's release is that of O += P V of block nvv - STAGES)
     auto issue_v = [&](int vkind, int vrow, int vsrc, int vslot, int vng) -> bool {
       const int vs = nvv % STAGES;
-      if (nvv >= STAGES && !mbar_wait_warp(&sm.v_empty[vs], ((nvv / STAGES) - 1) & 1, abort_flag, wl)) return false;
+      if (nvv >= STAGES && !mbar_wait_warp(&sm.v_empty[vs], ((nvv / STAGES) - 1) & 1, abort_flag)) return false;
       if (PACK && vkind == 0)
         tma_load_pieces(sm.v[vs], P.tvg, vsrc, vslot, vng, &sm.v_full[vs], lane);
       else
@@ -811,7 +797,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       const uint32_t par = ((issued / STAGES) - 1) & 1;
       // without packing a kept tile's rows start at (h T + id) 64, as in 64-row tiles
       const int row = kind == 0 && PACK ? 0 : block_row(g, h, kind, id);
-      if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag, wl);
+      if (issued >= STAGES) ok = mbar_wait_warp(&sm.k_empty[s], par, abort_flag);
       if (!ok) break;
       if (PACK && kind == 0)
         tma_load_pieces(sm.k[s], P.tkg, p_src, p_slot, p_ng, &sm.k_full[s], lane);
@@ -854,7 +840,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       };
       if constexpr (RING) {
         // the slot is free once the softmax has read the row of block issued - BST
-        if (issued >= BST) ok = mbar_wait_warp(&sm.b_empty[issued % BST], ((issued / BST) - 1) & 1, abort_flag, wl);
+        if (issued >= BST) ok = mbar_wait_warp(&sm.b_empty[issued % BST], ((issued / BST) - 1) & 1, abort_flag);
         if (!ok) break;
         write_bias();
       }
@@ -896,17 +882,17 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     const uint32_t id_qk = idesc(false), id_pv = idesc(true), id_sum = idesc(false, 16);
     const uint64_t dq = desc_k(saddr(sm.q));
     const uint64_t d1 = desc_k(saddr(sm.ones));
-    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag, wl);
+    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
     if constexpr (PTMEM) {
       // S = Q K^T of block q into score buffer q & 1 (free once the softmax
       // has loaded S of block q - 2), then the bias forward
       auto issue_qk = [&](int q) -> bool {
         const int s = q % STAGES, b = q & 1;
-        if (!mbar_wait_warp(&sm.k_full[s], (q / STAGES) & 1, abort_flag, wl)) return false;
-        if (q >= 2 && !mbar_wait_warp(&sm.s_free[b], ((q >> 1) - 1) & 1, abort_flag, wl)) return false;
+        if (!mbar_wait_warp(&sm.k_full[s], (q / STAGES) & 1, abort_flag)) return false;
+        if (q >= 2 && !mbar_wait_warp(&sm.s_free[b], ((q >> 1) - 1) & 1, abort_flag)) return false;
         fence_after();
         mma_qk_elect(tmem + s_addr(b), dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
-        if (!mbar_wait_warp(&sm.b_full[q % BST], (q / BST) & 1, abort_flag, wl)) return false;
+        if (!mbar_wait_warp(&sm.b_full[q % BST], (q / BST) & 1, abort_flag)) return false;
         if (lane == 0) mbar_arrive(&sm.s_full[b]);
         __syncwarp();
         return true;
@@ -917,8 +903,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         if (j + 2 < nb) ok = issue_qk(j + 2);
         if (!ok) break;
         const int s = j % STAGES, b = j & 1;
-        ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag, wl);
-        if (ok) ok = mbar_wait_warp(&sm.p_full[b], (j >> 1) & 1, abort_flag, wl);
+        ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag);
+        if (ok) ok = mbar_wait_warp(&sm.p_full[b], (j >> 1) & 1, abort_flag);
         if (!ok) break;
         fence_after();
         // O += P V, P (the A operand) from P buffer b in the accumulator's lanes
@@ -932,14 +918,14 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       // reusable as soon as the softmax has loaded it)
       while (qk < nb && qk <= j + NSBUF) {
         const int s = qk % STAGES, b = qk % NSBUF;
-        ok = mbar_wait_warp(&sm.k_full[s], (qk / STAGES) & 1, abort_flag, wl);
-        if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag, wl);
+        ok = mbar_wait_warp(&sm.k_full[s], (qk / STAGES) & 1, abort_flag);
+        if (ok && qk >= NSBUF) ok = mbar_wait_warp(&sm.s_free[b], ((qk / NSBUF) - 1) & 1, abort_flag);
         if (!ok) break;
         fence_after();
         mma_qk_elect(tmem + s_addr(b), dq, desc_k(saddr(sm.k[s])), id_qk, &sm.k_empty[s], &sm.s_full[b]);
         // forward the stage's bias row to the softmax through s_full: this
         // warp acquires it here and releases it with one arrival
-        ok = mbar_wait_warp(&sm.b_full[qk % BST], (qk / BST) & 1, abort_flag, wl);
+        ok = mbar_wait_warp(&sm.b_full[qk % BST], (qk / BST) & 1, abort_flag);
         if (!ok) break;
         if (lane == 0) mbar_arrive(&sm.s_full[b]);
         __syncwarp();
@@ -948,8 +934,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (!ok) break;
       // O += P V and L += P ones of block j
       const int s = j % STAGES, pb = j % PBUF;
-      ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag, wl);
-      if (ok) ok = mbar_wait_warp(&sm.p_full[pb], (j / PBUF) & 1, abort_flag, wl);
+      ok = mbar_wait_warp(&sm.v_full[s], (j / STAGES) & 1, abort_flag);
+      if (ok) ok = mbar_wait_warp(&sm.p_full[pb], (j / PBUF) & 1, abort_flag);
       if (!ok) break;
       fence_after();
       if (RSUM_MMA)
@@ -962,7 +948,10 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     // drain: every MMA this warp issued completes before TMEM is freed
     if (elect_one()) mma_commit(&sm.drain);
     __syncwarp();
-    mbar_drain_warp(&sm.drain, 0, *abort_flag ? DRAIN_NS : wl);
+    {
+      const unsigned long long lim = *(volatile unsigned long long*)&g_wait_ns;
+      mbar_drain_warp(&sm.drain, 0, *abort_flag ? DRAIN_NS + 0ull : lim);
+    }
   } else {
     // ---------------- softmax warpgroup ----------------
     const int rb = warp & 3;                  // TMEM lane quarter this warp may access
@@ -990,7 +979,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const int s = i % BST, b = PTMEM ? (i & 1) : i % NSBUF, pb = PTMEM ? (i & 1) : i % PBUF;
-      if (!mbar_wait_warp(&sm.s_full[b], (PTMEM ? (i >> 1) : i / NSBUF) & 1, abort_flag, wl)) { ok = false; break; }
+      if (!mbar_wait_warp(&sm.s_full[b], (PTMEM ? (i >> 1) : i / NSBUF) & 1, abort_flag)) { ok = false; break; }
       fence_after();
       float sv[32];
       tmem_ld64(tmem + lane_off + s_addr(b), sv);
@@ -1071,11 +1060,11 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       m1 = mn1;
       if constexpr (PTMEM) {
         // P buffer b is free once PV of block i - 2 has read it
-        if (i >= 2 && !mbar_wait_warp(&sm.pv_done[b], ((i >> 1) - 1) & 1, abort_flag, wl)) { ok = false; break; }
+        if (i >= 2 && !mbar_wait_warp(&sm.pv_done[b], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
         tmem_st_p(tmem + lane_off + p_addr_tmem(b), pk);
       } else {
         // P buffer pb is free once PV of block i-PBUF has completed
-        if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag, wl)) { ok = false; break; }
+        if (i >= PBUF && !mbar_wait_warp(&sm.pv_done[pb], ((i / PBUF) - 1) & 1, abort_flag)) { ok = false; break; }
         const uint32_t poff = (uint32_t)pb * (64u * 64u * 2u);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
@@ -1087,7 +1076,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       if (i >= 1 && __any_sync(0xffffffffu, up0 || up1)) {
         const int jp = i - 1;
         if (!mbar_wait_warp(&sm.pv_done[PTMEM ? (jp & 1) : jp % PBUF], (PTMEM ? (jp >> 1) : jp / PBUF) & 1,
-                            abort_flag, wl)) { ok = false; break; }
+                            abort_flag)) { ok = false; break; }
         fence_after();
         float o[32];
         tmem_ld64(tmem + lane_off + COL_O, o);
@@ -1116,7 +1105,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
     // ---------------- epilogue ----------------
     if (ok && nb >= 1 &&
         !mbar_wait_warp(&sm.pv_done[PTMEM ? ((nb - 1) & 1) : (nb - 1) % PBUF],
-                        (PTMEM ? ((nb - 1) >> 1) : (nb - 1) / PBUF) & 1, abort_flag, wl))
+                        (PTMEM ? ((nb - 1) >> 1) : (nb - 1) / PBUF) & 1, abort_flag))
       ok = false;
     if (ok) {
       fence_after();
