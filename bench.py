@@ -100,7 +100,9 @@ def stage_rates(kern: dict, g, hbm_gbs: float) -> dict:
     once; packed Q tiles [H, T, 64, 64], K and V in the dense layout of 8-row
     groups (H x views x rows-per-view rows), fp32 means and landmark rows
     written.
-    tile_scores: 2 * 64 FLOPs per (query tile, key tile) score (fp32 ALU).
+    tile_scores: 2 * 64 FLOPs per (query tile, key tile) score (the rate of fp32
+    scores it delivers; it computes them as one bf16 tensor-core GEMM with
+    K = 6 x 64 over the means' bf16 parts, 2 * 384 FLOPs per score).
     tile_select: the T x T fp32 scores read once per head.
     """
     layers = kern.get("pool_pack", (0, 0.0))[0]
@@ -122,7 +124,8 @@ def stage_rates(kern: dict, g, hbm_gbs: float) -> dict:
     if "tile_scores" in kern:
         ms = kern["tile_scores"][1] / layers
         out["tile_scores"] = {"ms_per_layer": round(ms, 3),
-                              "fp32_tflops": round(2 * 64 * T * T * H / (ms / 1e3) / 1e12, 2)}
+                              "fp32_score_tflops": round(2 * 64 * T * T * H / (ms / 1e3) / 1e12, 2),
+                              "bf16_gemm_tflops": round(2 * 384 * T * T * H / (ms / 1e3) / 1e12, 1)}
     if "tile_select" in kern:
         ms = kern["tile_select"][1] / layers
         out["tile_select"] = {"ms_per_layer": round(ms, 3), "score_gbs": round(4 * T * T * H / (ms / 1e3) / 1e9, 1)}

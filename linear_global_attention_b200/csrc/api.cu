@@ -163,6 +163,7 @@ static int max_pos(const Geo& G) { return G.Hp > G.Wp ? G.Hp : G.Wp; }
 struct SelectWs {
   float* scores;
   int hc, Tld;
+  void *qsplit, *ksplit, *gemm_ws;
 };
 static void carve_select(const Geo& G, Carver& c, SelectWs& w) {
   w.Tld = (G.T + 3) / 4 * 4;
@@ -173,6 +174,9 @@ static void carve_select(const Geo& G, Carver& c, SelectWs& w) {
   if (hc > G.H) hc = G.H;
   w.hc = (int)hc;
   w.scores = c.take<float>((size_t)w.hc * G.T * w.Tld);
+  w.qsplit = c.take<__nv_bfloat16>((size_t)w.hc * G.T * SPLIT_K);
+  w.ksplit = c.take<__nv_bfloat16>((size_t)w.hc * G.T * SPLIT_K);
+  w.gemm_ws = c.take<char>(GEMM_WS_BYTES);
 }
 
 struct SparseWs {
@@ -279,6 +283,10 @@ static int run_select(const Geo& G, const float* qm, const float* km, int keep, 
   a.keep = keep;
   a.mask = mask;
   a.near_tie = near_tie;
+  a.qsplit = w.qsplit;
+  a.ksplit = w.ksplit;
+  a.gemm_ws = w.gemm_ws;
+  a.gemm_ws_bytes = GEMM_WS_BYTES;
   for (int h0 = 0; h0 < G.H; h0 += w.hc) {
     a.h0 = h0;
     a.hc = G.H - h0 < w.hc ? G.H - h0 : w.hc;

@@ -45,7 +45,12 @@ struct SelectArgs {
   int keep;
   uint32_t* mask;       // [H, T, W]
   uint8_t* near_tie;    // [H, T] or null
+  void* qsplit;         // [hc, T, 384] bf16: the query means as bf16 parts (see scores_split_kernel)
+  void* ksplit;         // [hc, T, 384] bf16: the key means, parts in the matching order
+  void* gemm_ws;        // cuBLASLt workspace for the score GEMM
+  size_t gemm_ws_bytes;
 };
+constexpr int SPLIT_K = 6 * 64;   // the score GEMM's K: six products of bf16 parts
 int launch_scores(const SelectArgs& a, cudaStream_t st);
 int launch_select(const SelectArgs& a, cudaStream_t st);
 constexpr int SELECT_MAX_T = 49152;

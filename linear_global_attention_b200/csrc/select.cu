@@ -7,9 +7,12 @@
 // mean-pooled query and key (fp32), keeps the top k, and breaks equal scores
 // toward the lower tile index.
 //
-// Two kernels per group of heads:
-//  1. scores_kernel: S[h][t][u] = qm[h][t] . km[h][u] for all t, u — a 128x128-tile
-//     fp32 GEMM (K = 64) written to scratch; each score is a fixed-order fma chain.
+// Per group of heads:
+//  1. the scores S[h][t][u] = qm[h][t] . km[h][u] for all t, u, written to scratch:
+//     scores_split_kernel splits the fp32 means into bf16 parts and one bf16
+//     tensor-core GEMM (cuBLASLt, K = 6 x 64, fp32 accumulate, no split-K) sums the
+//     part products to fp32 accuracy; scores_kernel, a 128x128-tile fp32 GEMM
+//     with a fixed-order fma chain per score, is the CUDA-core alternative.
 //  2. select_kernel: one CTA per row (h, t) copies the row into shared memory
 //     (16-byte asynchronous copies, all in flight at once) and turns it into
 //     order-preserving 32-bit keys, finds the k-th largest key from a 2,048-bin
@@ -22,6 +25,7 @@
 //     It also flags near-ties: the k-th and (k+1)-th scores within a relative
 //     gap of 1e-5.
 #include "common.cuh"
+#include "gemm.cuh"
 #include "kernels.cuh"
 
 namespace zebra {
@@ -452,11 +456,51 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectArgs a) {
   }
 }
 
+// Scores on the tensor cores. Each fp32 mean x is split into three bf16 parts,
+// x = x0 + x1 + x2 up to 2^-24 relative (x0 = bf16(x), x1 = bf16(x - x0),
+// x2 = bf16(x - x0 - x1); both subtractions are exact in fp32). The score
+// q . k = sum over the part pairs of q_a . k_b; the six pairs with a + b <= 2
+// leave out terms of relative size 2^-24 and below. Laid out as one bf16 GEMM
+// with K = 6 x 64, Q'[t] = [q0 q0 q1 q0 q1 q2] and K'[u] = [k0 k1 k0 k2 k1 k0],
+// with fp32 accumulation: the score error is that of an fp32 dot product,
+// and equal key means give equal scores (every element sums its products in
+// the same order).
+__global__ void __launch_bounds__(128) scores_split_kernel(SelectArgs a) {
+  const int T = a.g.T;
+  const int t = blockIdx.x * 2 + (threadIdx.x >> 6), c = threadIdx.x & 63;
+  const int hh = blockIdx.y, h = a.h0 + hh;
+  if (t >= T) return;
+  auto parts = [](float x, __nv_bfloat16& p0, __nv_bfloat16& p1, __nv_bfloat16& p2) {
+    p0 = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(p0);
+    p1 = __float2bfloat16_rn(r1);
+    p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+  };
+  __nv_bfloat16 q0, q1, q2, k0, k1, k2;
+  parts(a.qm[((size_t)h * T + t) * D + c], q0, q1, q2);
+  parts(a.km[((size_t)h * T + t) * D + c], k0, k1, k2);
+  __nv_bfloat16* qs = static_cast<__nv_bfloat16*>(a.qsplit) + ((size_t)hh * T + t) * SPLIT_K + c;
+  __nv_bfloat16* ks = static_cast<__nv_bfloat16*>(a.ksplit) + ((size_t)hh * T + t) * SPLIT_K + c;
+  qs[0] = q0; qs[64] = q0; qs[128] = q1; qs[192] = q0; qs[256] = q1; qs[320] = q2;
+  ks[0] = k0; ks[64] = k1; ks[128] = k0; ks[192] = k2; ks[256] = k1; ks[320] = k0;
+}
+
+#ifndef ZEBRA_SCORES_TC
+#define ZEBRA_SCORES_TC 1
+#endif
+
 int launch_scores(const SelectArgs& a, cudaStream_t st) {
   const int T = a.g.T;
   if (T == 0 || a.keep >= T) return ZEBRA_OK;
-  dim3 grid((T + SC_TILE - 1) / SC_TILE, (T + SC_TILE - 1) / SC_TILE, a.hc);
   ProfScope prof("tile_scores", st);
+  if (ZEBRA_SCORES_TC && a.qsplit) {
+    scores_split_kernel<<<dim3((T + 1) / 2, a.hc), 128, 0, st>>>(a);
+    count_launch();
+    if (int rc = check_launch("scores_split_kernel")) return rc;
+    return gemm_bf16_nt_f32(a.qsplit, a.ksplit, a.scores, T, T, SPLIT_K, a.Tld, a.hc, (long long)T * SPLIT_K,
+                            (long long)T * SPLIT_K, (long long)T * a.Tld, a.gemm_ws, a.gemm_ws_bytes, st);
+  }
+  dim3 grid((T + SC_TILE - 1) / SC_TILE, (T + SC_TILE - 1) / SC_TILE, a.hc);
   scores_kernel<<<grid, 256, 0, st>>>(a);
   count_launch();
   return check_launch("scores_kernel");
