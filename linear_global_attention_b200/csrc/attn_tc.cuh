@@ -135,7 +135,18 @@ constexpr int PSM = PTMEM ? 0 : PBUF;    // shared-memory P buffers
 // block's row before it waits for a V stage, so S of block i + 2 never waits
 // for O += P V of block i.
 constexpr bool RING = PTMEM || NSBUF == 2;
-constexpr int BST = RING ? 4 : STAGES;  // bias-row slots
+#ifndef ZEBRA_TC_BIAS3
+#define ZEBRA_TC_BIAS3 1
+#endif
+// Bias rows in STAGES + 1 slots, written right after the block's K copy: the
+// slot of block i + 3 is free once QK^T of block i + 1 has completed (the
+// producer has just waited for that to reuse the K stage), since that MMA
+// was issued only after every softmax warp had signalled, after reading the
+// row of block i, that it was done with block i's scores. Tied to the V stage
+// instead, the row of block i waited for O += P V of block i - 2, and the MMA
+// warp, which forwards the row to the softmax, waited with it.
+constexpr bool BIAS3 = !RING && ZEBRA_TC_BIAS3 != 0;
+constexpr int BST = RING ? 4 : (BIAS3 ? STAGES + 1 : STAGES);  // bias-row slots
 #ifndef ZEBRA_TC_STAGGER
 #define ZEBRA_TC_STAGGER 0
 #endif
@@ -844,6 +855,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         if (!ok) break;
         write_bias();
       }
+      if constexpr (BIAS3) write_bias();
       // the V tile (and without PTMEM the bias row) of this stage is free once
       // PV of block issued - STAGES is done
       if constexpr (KAHEAD) {
@@ -858,7 +870,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         ok = issue_v(kind, row, p_src, p_slot, p_ng);
         if (!ok) break;
       }
-      if constexpr (!RING) write_bias();
+      if constexpr (!RING && !BIAS3) write_bias();
       ++issued;
     }
     if (KAHEAD && ok && pend_kind >= 0)
@@ -983,9 +995,11 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
       fence_after();
       float sv[32];
       tmem_ld64(tmem + lane_off + s_addr(b), sv);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[b]);
+      if constexpr (!BIAS3) {
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[b]);
+      }
 
       // scale, bias (log2 units) and row maxima; sv[4j], sv[4j+1] belong to
       // row r0 and sv[4j+2], sv[4j+3] to row r1
@@ -1013,6 +1027,12 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM) attn_tc_kernel(const __g
         // this warp is done with the block's bias row
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.b_empty[s]);
+      }
+      if constexpr (BIAS3) {
+        // done with the block's scores and its bias row
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[b]);
       }
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
