@@ -15,12 +15,14 @@
 // described in attn.cu. The block count is known up front (a pre-pass over the
 // selection row), so only the producer walks the stream. Warp roles:
 //   warp 0      producer: TMA loads of Q once and of the K and V tile of every
-//               block (one 64-row copy, or for packed blocks eight 8-row group
-//               copies from eight lanes) into rings of STAGES
-//               128-byte-swizzled 64x64 bf16 tiles (separate K and V barriers:
-//               QK^T may start as soon as K has landed); the whole warp writes
-//               the block's 64 logit biases (log2 units: 0, ln(n_u) for
-//               landmarks, -inf for masked columns) into the stage's bias row;
+//               block (one 64-row copy, or for a packed block one copy per run
+//               of a tile's 8-row groups, each issued by its own lane) into
+//               rings of STAGES 128-byte-swizzled 64x64 bf16 tiles (separate K
+//               and V barriers: QK^T may start as soon as K has landed); right
+//               after the K copy the whole warp writes the block's 64 logit
+//               biases (log2 units: 0, ln(n_u) for landmarks, -inf for masked
+//               columns) into one of STAGES + 1 bias slots, or only flags a
+//               block of 64 real keys as bias-free;
 //   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of NSBUF TMEM
 //               score buffers (tcgen05.mma M=64 N=64, K-major A/B), issued up
 //               to NSBUF blocks ahead of O += P V (P from shared memory,
