@@ -201,6 +201,103 @@ __device__ __forceinline__ void features_q4(float* xa, float* xb, int half, int 
   }
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+__device__ __forceinline__ float2 l_fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n mov.b64 rc, {%6,%7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0,%1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 l_mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n"
+      " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0,%1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 l_add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0,%1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+#ifndef ZEBRA_LIN_F32X2
+#define ZEBRA_LIN_F32X2 1
+#endif
+
+// features_q4 with the elementwise steps on f32x2 pairs (channels 2p, 2p + 1 of
+// xa and of xb): sums of squares, scaling, rotation, the exponent argument,
+// the sum and the normalisation take half the instructions; the maximum,
+// the exponentials and the shuffles stay scalar.
+__device__ __forceinline__ void features_q4_x2(float* xa, float* xb, int half, int sub, bool special, int row,
+                                               int col, const float2* __restrict__ tab, float eps) {
+  float2* A = reinterpret_cast<float2*>(xa);
+  float2* B = reinterpret_cast<float2*>(xb);
+  float2 s0 = l_mul2(A[0], A[0]), s1 = l_mul2(A[1], A[1]);
+  s0 = l_fma2(A[2], A[2], s0);
+  s1 = l_fma2(A[3], A[3], s1);
+  s0 = l_fma2(B[0], B[0], s0);
+  s1 = l_fma2(B[1], B[1], s1);
+  s0 = l_fma2(B[2], B[2], s0);
+  s1 = l_fma2(B[3], B[3], s1);
+  s0 = l_add2(s0, s1);
+  float ss = s0.x + s0.y;
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float sc = rsqrtf(ss * (1.0f / D) + eps);
+  const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    A[p] = l_mul2(A[p], sc2);
+    B[p] = l_mul2(B[p], sc2);
+  }
+  if (!special) {
+    const float2* t = tab + (half ? col : row) * 16 + 8 * sub;
+    const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 cs0 = __ldg(t + 2 * p), cs1 = __ldg(t + 2 * p + 1);
+      const float2 c = make_float2(cs0.x, cs1.x), sn = make_float2(cs0.y, cs1.y);
+      const float2 a = A[p], b = B[p];
+      A[p] = l_fma2(a, c, l_mul2(b, l_mul2(sn, m1)));   // a cos - b sin
+      B[p] = l_fma2(b, c, l_mul2(a, sn));               // b cos + a sin
+    }
+  }
+  float m4[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) m4[e] = fmaxf(fmaxf(xa[e], xa[e + 4]), fmaxf(xb[e], xb[e + 4]));
+  float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float2 l2e = make_float2(LOG2E, LOG2E), off = make_float2(-mx * LOG2E, -mx * LOG2E);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float2 ea = l_fma2(A[p], l2e, off), eb = l_fma2(B[p], l2e, off);
+    A[p] = make_float2(fast_exp2(ea.x), fast_exp2(ea.y));
+    B[p] = make_float2(fast_exp2(eb.x), fast_exp2(eb.y));
+  }
+  float2 t0 = l_add2(l_add2(A[0], A[1]), l_add2(A[2], A[3]));
+  const float2 t1 = l_add2(l_add2(B[0], B[1]), l_add2(B[2], B[3]));
+  t0 = l_add2(t0, t1);
+  float sum = t0.x + t0.y;
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const float inv = 1.0f / sum;
+  const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    A[p] = l_mul2(A[p], inv2);
+    B[p] = l_mul2(B[p], inv2);
+  }
+}
+
+
 __device__ __forceinline__ void read_q4(const unsigned char* tile, int tok, int half, int sub, float* xa, float* xb) {
   const int ca = 4 * half + sub;
   const uint4 wa = *reinterpret_cast<const uint4*>(tile + lswz(tok, ca));
@@ -282,7 +379,10 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
       int row, col;
       view_pos(g, mod_L(g, jb + tok), sp, row, col);
       jb = mod_L(g, jb + 64);
-      features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      if (ZEBRA_LIN_F32X2)
+        features_q4_x2(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      else
+        features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
       if (!valid) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
@@ -380,7 +480,10 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       int row, col;
       view_pos(g, mod_L(g, jb + tok), sp, row, col);
       jb = mod_L(g, jb + 64);
-      features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      if (ZEBRA_LIN_F32X2)
+        features_q4_x2(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
+      else
+        features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
       if (!valid) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
