@@ -187,6 +187,7 @@ struct SparseWs {
   float *part_o, *part_ml;
   int splits;
   float2* rope;
+  float* lmk_bias;
 };
 static void carve_sparse(const Geo& G, zebra_dtype dt, Carver& c, SparseWs& w) {
   const size_t es = esize(dt);
@@ -206,6 +207,7 @@ static void carve_sparse(const Geo& G, zebra_dtype dt, Carver& c, SparseWs& w) {
   w.km = c.take<float>(means);
   w.vm = c.take<float>(means);
   w.mask = c.take<uint32_t>((size_t)G.H * G.T * G.W);
+  w.lmk_bias = c.take<float>((size_t)G.T);
   carve_select(G, c, w.sel);
   // key splits of the special-token rows: about 8 resident waves of work
   // items (148 SMs x 4 CTAs each) over all query blocks and heads
@@ -256,9 +258,9 @@ static void carve_hybrid(const Geo& G, int kind, Carver& c, HybridWs& w) {
     carve_sparse(G, ZEBRA_BF16, c, w.sp);
 }
 
-static void fill_ln_tab(AttnArgs& a) {
-  a.ln_tab[0] = 0.f;
-  for (int m = 1; m <= TOK; ++m) a.ln_tab[m] = (float)std::log((double)m);
+static void fill_ln_tab(float* tab) {
+  tab[0] = 0.f;
+  for (int m = 1; m <= TOK; ++m) tab[m] = (float)std::log((double)m);
 }
 
 static int keep_of(double y, int T) {
@@ -323,6 +325,8 @@ static int run_sparse(const Geo& G, const void* q, const void* k, const void* v,
   pa.rope = norm_rope ? w.rope : nullptr;
   pa.eps = eps;
   pa.counts = nullptr;
+  pa.lmk_bias = w.lmk_bias;
+  fill_ln_tab(pa.ln_tab);
   pa.dense_kv = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;   // the tcgen05 kernel's K/V layout
   if (G.T > 0) ZTRY(launch_pool_pack<T>(pa, 3, st));
   SpecialArgs<T> sa{};
@@ -356,7 +360,8 @@ static int run_sparse(const Geo& G, const void* q, const void* k, const void* v,
   aa.part_o = w.part_o;
   aa.part_ml = w.part_ml;
   aa.splits = w.splits;
-  fill_ln_tab(aa);
+  aa.lmk_bias = w.lmk_bias;
+  fill_ln_tab(aa.ln_tab);
   if (G.T > 0) ZTRY(launch_sparse_attn<T>(aa, st));
   ZTRY(launch_special_rows<T>(aa, st));
   return ZEBRA_OK;

@@ -175,8 +175,7 @@ __device__ __forceinline__ float block_bias(const AttnArgs& a, const uint32_t* _
     const int u = id * 64 + j;
     if (u >= g.T || u == t) return NEG;
     if ((__ldg(mrow + (u >> 5)) >> (u & 31)) & 1u) return NEG;
-    const TileShape s = tile_shape(g, u);
-    return a.ln_tab[s.rows * s.cols] * LOG2E;
+    return __ldg(a.lmk_bias + u);   // ln(n_u) log2(e), written by the pooling pass
   }
   return id * 64 + j < g.NS ? 0.f : NEG;
 }

@@ -18,6 +18,8 @@ struct PoolArgs {
   const float2* rope;   // [maxpos, 16] cos/sin table or null
   float eps;
   int32_t* counts;      // [T] or null
+  float* lmk_bias;      // [T] or null: ln(n_u) log2(e), the logit bias of tile u's landmark
+  float ln_tab[TOK + 1];   // ln(m), m = 0..64, for lmk_bias
 };
 
 template <typename T>
@@ -70,6 +72,7 @@ struct AttnArgs {
   float* part_ml;                                     // [splits, H, NSp, 2] (max in log2 units, sum)
   int splits;
   float ln_tab[TOK + 1];                              // ln(m), m = 0..64 (ln_tab[0] unused)
+  const float* lmk_bias;                              // [T] ln(n_u) log2(e) per tile (landmark logit bias)
 };
 template <typename T> int launch_sparse_attn(const AttnArgs& a, cudaStream_t st);
 int launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t st);

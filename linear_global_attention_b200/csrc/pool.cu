@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(128) pool_pack_kernel(PoolArgs<T> a) {
   }
   if (a.lmk[z]) store16(a.lmk[z] + ((size_t)hh * g.Tpad + u) * D + chunk * P, sum);
   if (a.counts && z == 0 && h == 0 && chunk == 0) a.counts[u] = n;
+  if (a.lmk_bias && z == 0 && h == 0 && chunk == 0) a.lmk_bias[u] = a.ln_tab[n] * LOG2E;
 }
 
 // Special tokens of all views, packed per head: out[h][i][:] for i < NSp
