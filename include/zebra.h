@@ -118,9 +118,11 @@ ZEBRA_API int zebra_tile_pool(const zebra_geom* g, zebra_dtype dt, const void* x
                     float* x_mean, void* x_packed, int32_t* tile_counts, void* stream);
 
 /* Per-query-tile key-tile selector (section "Linear-centered stages plus
- * tile-sparse stages"). Scores key tile u for query tile t by the fp32 dot
- * q_mean[h,t] . k_mean[h,u] over all T tiles (own tile included) and keeps the
- * top k = zebra_keep_count(y, T); equal scores go to the lower tile index.
+ * tile-sparse stages"). Scores key tile u for query tile t by the dot
+ * q_mean[h,t] . k_mean[h,u] over all T tiles (own tile included), to fp32
+ * accuracy (tensor cores on the means' bf16 parts, fp32 accumulation; equal
+ * key means give equal scores), and keeps the top k = zebra_keep_count(y, T);
+ * equal scores go to the lower tile index.
  *   q_mean, k_mean [H, T, d] fp32 (from zebra_tile_pool)
  *   mask      out [H, T, W] uint32, W = ceil(T/32): bit (u%32) of word u/32 of
  *             row (h, t) is set iff key tile u is kept for query tile t
