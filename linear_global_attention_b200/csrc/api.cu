@@ -230,6 +230,7 @@ struct LinearWs {
   float* state;
   void* state_b;
   float2* rope;
+  float4* rope_g;
   int chunks, chunk_tokens;
 };
 static void carve_linear(const Geo& G, Carver& c, LinearWs& w) {
@@ -238,6 +239,7 @@ static void carve_linear(const Geo& G, Carver& c, LinearWs& w) {
   w.state = c.take<float>((size_t)G.H * 64 * 65);
   w.state_b = c.take<__nv_bfloat16>((size_t)G.H * 72 * 64);
   w.rope = c.take<float2>((size_t)max_pos(G) * 16);
+  w.rope_g = c.take<float4>((size_t)max_pos(G) * 8);
 }
 
 struct HybridWs {
@@ -303,7 +305,7 @@ static int run_sparse(const Geo& G, const void* q, const void* k, const void* v,
                       const uint32_t* mask_in, void* out, const SparseWs& w, bool norm_rope, float rope_base,
                       float eps, cudaStream_t st) {
   if (G.N == 0) return ZEBRA_OK;
-  if (norm_rope) ZTRY(launch_rope_table(w.rope, max_pos(G), (double)rope_base, st));
+  if (norm_rope) ZTRY(launch_rope_table(w.rope, nullptr, max_pos(G), (double)rope_base, st));
   PoolArgs<T> pa{};
   pa.g = G;
   pa.x[0] = static_cast<const T*>(q);
@@ -372,7 +374,7 @@ static int run_linear(const Geo& G, const void* q, const void* k, const void* v,
                       const float* A, const float* b, float rope_base, float eps, void* out, const LinearWs& w,
                       cudaStream_t st) {
   if (G.N == 0) return ZEBRA_OK;
-  ZTRY(launch_rope_table(w.rope, max_pos(G), (double)rope_base, st));
+  ZTRY(launch_rope_table(w.rope, w.rope_g, max_pos(G), (double)rope_base, st));
   LinearArgs a{};
   a.g = G;
   a.q = q; a.k = k; a.v = v;
@@ -380,6 +382,8 @@ static int run_linear(const Geo& G, const void* q, const void* k, const void* v,
   a.A = A; a.b = b;
   a.eps = eps;
   a.rope = w.rope;
+  a.rope_g = w.rope_g;
+  a.maxpos = max_pos(G);
   a.part = w.part;
   a.chunks = w.chunks;
   a.chunk_tokens = w.chunk_tokens;

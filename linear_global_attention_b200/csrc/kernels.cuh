@@ -34,7 +34,8 @@ struct SpecialArgs {
 
 template <typename T> int launch_pool_pack(const PoolArgs<T>& a, int ntensors, cudaStream_t st);
 template <typename T> int launch_pack_special(const SpecialArgs<T>& a, int ntensors, cudaStream_t st);
-int launch_rope_table(float2* tab, int maxpos, double base, cudaStream_t st);
+// tab_g (optional): the same table as packed-pair operands of the linear kernels
+int launch_rope_table(float2* tab, float4* tab_g, int maxpos, double base, cudaStream_t st);
 
 // ---- selector ----
 struct SelectArgs {
@@ -106,6 +107,8 @@ struct LinearArgs {
   const float* A; const float* b;   // [H, d, d], [H, d] or null
   float eps;
   const float2* rope;               // [maxpos, 16]
+  const float4* rope_g;             // [8 pair groups, maxpos] (launch_rope_table's tab_g)
+  int maxpos;
   float* part;                      // [chunks, H, d, 65] partial (S | z)
   int chunks, chunk_tokens;
   float* state;                     // [H, d, 65] fp32  S' = S A^T | z

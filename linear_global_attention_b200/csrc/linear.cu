@@ -21,8 +21,10 @@
 //  2. reduce: per head, sums the chunk partials in a fixed order (deterministic),
 //     forms S' = S A^T, and writes the bf16 B operand [S' | z] of the apply kernel.
 //  3. apply:  per (head, token chunk) CTA: prologue on Q (f(Q) overwrites its
-//     own ring stage), f(Q) [S' | z] on mma.sync, divide by the z column, add b,
-//     store bf16 straight from registers.
+//     own ring stage; the softmax's division by its sum is left out, since it
+//     cancels in the ratio below), f(Q) [S' | z] on mma.sync, divide by the z
+//     column, add b, stage the bf16 block in the same ring stage and store
+//     whole 128-byte token rows.
 // The fp32 variants run the same three steps with plain fp32 arithmetic.
 #include <math.h>
 
@@ -115,9 +117,6 @@ constexpr int LSTAGES = 3;
 #define ZEBRA_LIN_ASTAGES 4
 #endif
 constexpr int LA_STAGES = ZEBRA_LIN_ASTAGES;   // Q ring depth of the apply kernel
-#ifndef ZEBRA_LIN_STAGED_OUT
-#define ZEBRA_LIN_STAGED_OUT 1   // apply: output through shared memory (1) or from registers (0)
-#endif
 
 struct StateSmem {
   unsigned char phi[64 * 128];
@@ -135,71 +134,25 @@ struct StateSmem {
 // z column (warp / 4 = 0) or columns 32-63 (warp / 4 = 1).
 constexpr int LQ_THREADS = 256;
 
-__device__ __forceinline__ void fetch_rows_q4(uint32_t tile, const __nv_bfloat16* base, long long nb, long long n1,
-                                              long long ts, int tok, int half, int sub) {
-  const long long n = nb + tok;
-  const bool ok = n < n1;
-  const __nv_bfloat16* p = base + (ok ? n : 0) * ts + 32 * half + 8 * sub;
-  const int ca = 4 * half + sub;   // 16-byte chunk of the "a" channels; the partners are 2 chunks on
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, ca)), "l"(p),
-               "r"(ok ? 16 : 0));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tile + lswz(tok, ca + 2)), "l"(p + 16),
-               "r"(ok ? 16 : 0));
-}
-
-// f(x) on this thread's 16 channels (xa: the "a" channels, xb: their partners).
-// The sums and the maximum are short trees over independent partials, so the
-// dependent chains stay a few operations deep.
-__device__ __forceinline__ void features_q4(float* xa, float* xb, int half, int sub, bool special, int row, int col,
-                                            const float2* __restrict__ tab, float eps) {
-  float s4[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) s4[e] = fmaf(xa[e], xa[e], xa[e + 4] * xa[e + 4]);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) s4[e] = fmaf(xb[e], xb[e], fmaf(xb[e + 4], xb[e + 4], s4[e]));
-  float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  const float sc = rsqrtf(ss * (1.0f / D) + eps);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    xa[e] *= sc;
-    xb[e] *= sc;
+// This thread's part of its token's row in one tensor: two 16-byte pieces per
+// 64-token block (the "a" channels and, 2 chunks on, their partners), copied
+// into a ring stage at the fixed swizzled offsets oa, ob. The source walks
+// down the chunk by 64 token rows per fetched block; pieces of rows past the
+// chunk's end are zero-filled (read from the tensor's base, never past it).
+struct RowFetch {
+  const __nv_bfloat16* base;
+  const __nv_bfloat16* p;   // this thread's row in the next block to fetch
+  long long step;           // 64 token rows
+  __device__ __forceinline__ RowFetch(const __nv_bfloat16* t, long long n0, long long ts, int tok, int half, int sub)
+      : base(t), p(t + (n0 + tok) * ts + 32 * half + 8 * sub), step(64 * ts) {}
+  __device__ __forceinline__ void fetch(uint32_t stage, uint32_t oa, uint32_t ob, bool ok) {
+    const __nv_bfloat16* src = ok ? p : base;
+    const int n = ok ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(stage + oa), "l"(src), "r"(n));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(stage + ob), "l"(src + 16), "r"(n));
+    p += step;
   }
-  if (!special) {
-    const float2* t = tab + (half ? col : row) * 16 + 8 * sub;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float2 cs = __ldg(t + e);
-      const float a = xa[e], b = xb[e];
-      xa[e] = a * cs.x - b * cs.y;
-      xb[e] = b * cs.x + a * cs.y;
-    }
-  }
-  float m4[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) m4[e] = fmaxf(fmaxf(xa[e], xa[e + 4]), fmaxf(xb[e], xb[e + 4]));
-  float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const float off = -mx * LOG2E;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    xa[e] = fast_exp2(fmaf(xa[e], LOG2E, off));
-    xb[e] = fast_exp2(fmaf(xb[e], LOG2E, off));
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) s4[e] = (xa[e] + xa[e + 4]) + (xb[e] + xb[e + 4]);
-  float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-  const float inv = 1.0f / sum;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    xa[e] *= inv;
-    xb[e] *= inv;
-  }
-}
+};
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
 __device__ __forceinline__ float2 l_fma2(float2 a, float2 b, float2 c) {
@@ -226,17 +179,33 @@ __device__ __forceinline__ float2 l_add2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 l_sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n"
+      " sub.rn.f32x2 rd, ra, rb;\n mov.b64 {%0,%1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 
-#ifndef ZEBRA_LIN_F32X2
-#define ZEBRA_LIN_F32X2 1
-#endif
-
-// features_q4 with the elementwise steps on f32x2 pairs (channels 2p, 2p + 1 of
-// xa and of xb): sums of squares, scaling, rotation, the exponent argument,
-// the sum and the normalisation take half the instructions; the maximum,
-// the exponentials and the shuffles stay scalar.
-__device__ __forceinline__ void features_q4_x2(float* xa, float* xb, int half, int sub, bool special, int row,
-                                               int col, const float2* __restrict__ tab, float eps) {
+// f(x) on this thread's 16 channels (xa: the "a" channels of its 8 rotation
+// pairs, xb: their partners), the elementwise steps on f32x2 pairs (channels
+// 2p, 2p + 1 of xa and of xb). It rests on three facts:
+//  - the rotation keeps the norm of each pair, so the RMS scale sc of the raw
+//    channels is that of the rotated ones, and, the rotation being linear, sc
+//    goes into the exponent: exp(sc r_c) = exp2(r_c (sc log2 e));
+//  - every channel of sc x has |sc x_c| <= sqrt(64) = 8 (the RMS of the 64
+//    channels is at most 1), so exp(sc r_c) lies in [e^-8, e^8] and the
+//    channel softmax needs no maximum shift;
+//  - with NORMALISE = false the division by the sum is left out: the apply
+//    kernel's output is a ratio of two contractions that are both linear in
+//    f(q), so the sum cancels.
+// The sum of squares goes across the token's 4 threads while the rotation runs.
+// Padding tokens (valid = false, zero-filled) get exponent arguments 0 and,
+// when normalised, features 0.
+template <bool NORMALISE>
+__device__ __forceinline__ void features_lin(float* xa, float* xb, int half, int sub, bool special, int row, int col,
+                                             const float4* __restrict__ tab, int maxpos, float eps, bool valid) {
   float2* A = reinterpret_cast<float2*>(xa);
   float2* B = reinterpret_cast<float2*>(xb);
   float2 s0 = l_mul2(A[0], A[0]), s1 = l_mul2(A[1], A[1]);
@@ -250,58 +219,47 @@ __device__ __forceinline__ void features_q4_x2(float* xa, float* xb, int half, i
   float ss = s0.x + s0.y;
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  const float sc = rsqrtf(ss * (1.0f / D) + eps);
-  const float2 sc2 = make_float2(sc, sc);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    A[p] = l_mul2(A[p], sc2);
-    B[p] = l_mul2(B[p], sc2);
-  }
   if (!special) {
-    const float2* t = tab + (half ? col : row) * 16 + 8 * sub;
-    const float2 m1 = make_float2(-1.f, -1.f);
+    // pair group 4 sub + p at the half's position: (cos, cos', sin, sin'). Consecutive
+    // tokens of a warp read consecutive positions of a group: few L1 lines per load.
+    const float4* t = tab + 4 * sub * maxpos + (half ? col : row);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const float2 cs0 = __ldg(t + 2 * p), cs1 = __ldg(t + 2 * p + 1);
-      const float2 c = make_float2(cs0.x, cs1.x), sn = make_float2(cs0.y, cs1.y);
+      const float4 cs = __ldg(t + p * maxpos);
+      const float2 c = make_float2(cs.x, cs.y), sn = make_float2(cs.z, cs.w);
       const float2 a = A[p], b = B[p];
-      A[p] = l_fma2(a, c, l_mul2(b, l_mul2(sn, m1)));   // a cos - b sin
-      B[p] = l_fma2(b, c, l_mul2(a, sn));               // b cos + a sin
+      A[p] = l_sub2(l_mul2(a, c), l_mul2(b, sn));   // a cos - b sin
+      B[p] = l_fma2(b, c, l_mul2(a, sn));           // b cos + a sin
     }
   }
-  float m4[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) m4[e] = fmaxf(fmaxf(xa[e], xa[e + 4]), fmaxf(xb[e], xb[e + 4]));
-  float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const float2 l2e = make_float2(LOG2E, LOG2E), off = make_float2(-mx * LOG2E, -mx * LOG2E);
+  const float k = valid ? rsqrtf(ss * (1.0f / D) + eps) * LOG2E : 0.f;
+  const float2 k2 = make_float2(k, k);
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const float2 ea = l_fma2(A[p], l2e, off), eb = l_fma2(B[p], l2e, off);
+    const float2 ea = l_mul2(A[p], k2), eb = l_mul2(B[p], k2);
     A[p] = make_float2(fast_exp2(ea.x), fast_exp2(ea.y));
     B[p] = make_float2(fast_exp2(eb.x), fast_exp2(eb.y));
   }
-  float2 t0 = l_add2(l_add2(A[0], A[1]), l_add2(A[2], A[3]));
-  const float2 t1 = l_add2(l_add2(B[0], B[1]), l_add2(B[2], B[3]));
-  t0 = l_add2(t0, t1);
-  float sum = t0.x + t0.y;
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-  const float inv = 1.0f / sum;
-  const float2 inv2 = make_float2(inv, inv);
+  if (NORMALISE) {
+    float2 t0 = l_add2(l_add2(A[0], A[1]), l_add2(A[2], A[3]));
+    const float2 t1 = l_add2(l_add2(B[0], B[1]), l_add2(B[2], B[3]));
+    t0 = l_add2(t0, t1);
+    float sum = t0.x + t0.y;
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    const float inv = valid ? __fdividef(1.0f, sum) : 0.f;   // sum lies in [64 e^-8, 64 e^8]
+    const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    A[p] = l_mul2(A[p], inv2);
-    B[p] = l_mul2(B[p], inv2);
+    for (int p = 0; p < 4; ++p) {
+      A[p] = l_mul2(A[p], inv2);
+      B[p] = l_mul2(B[p], inv2);
+    }
   }
 }
 
-
-__device__ __forceinline__ void read_q4(const unsigned char* tile, int tok, int half, int sub, float* xa, float* xb) {
-  const int ca = 4 * half + sub;
-  const uint4 wa = *reinterpret_cast<const uint4*>(tile + lswz(tok, ca));
-  const uint4 wb = *reinterpret_cast<const uint4*>(tile + lswz(tok, ca + 2));
+__device__ __forceinline__ void read_q4(const unsigned char* tile, uint32_t oa, uint32_t ob, float* xa, float* xb) {
+  const uint4 wa = *reinterpret_cast<const uint4*>(tile + oa);
+  const uint4 wb = *reinterpret_cast<const uint4*>(tile + ob);
   const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&wa);
   const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&wb);
 #pragma unroll
@@ -314,9 +272,7 @@ __device__ __forceinline__ void read_q4(const unsigned char* tile, int tok, int 
   }
 }
 
-__device__ __forceinline__ void store_q4(unsigned char* tile, int tok, int half, int sub, const float* xa,
-                                         const float* xb) {
-  const int ca = 4 * half + sub;
+__device__ __forceinline__ void store_q4(unsigned char* tile, uint32_t oa, uint32_t ob, const float* xa, const float* xb) {
   uint4 va, vb;
   __nv_bfloat162* ha = reinterpret_cast<__nv_bfloat162*>(&va);
   __nv_bfloat162* hb = reinterpret_cast<__nv_bfloat162*>(&vb);
@@ -325,9 +281,11 @@ __device__ __forceinline__ void store_q4(unsigned char* tile, int tok, int half,
     ha[e] = __floats2bfloat162_rn(xa[2 * e], xa[2 * e + 1]);
     hb[e] = __floats2bfloat162_rn(xb[2 * e], xb[2 * e + 1]);
   }
-  *reinterpret_cast<uint4*>(tile + lswz(tok, ca)) = va;
-  *reinterpret_cast<uint4*>(tile + lswz(tok, ca + 2)) = vb;
+  *reinterpret_cast<uint4*>(tile + oa) = va;
+  *reinterpret_cast<uint4*>(tile + ob) = vb;
 }
+
+__device__ __forceinline__ int ring_next(int s, int n) { return s + 1 == n ? 0 : s + 1; }
 
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __grid_constant__ LinearArgs a) {
   extern __shared__ __align__(128) unsigned char state_smem[];
@@ -348,16 +306,20 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
 
   const int nblk = (int)((n1 - n0 + 63) / 64);
+  const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
+  const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
+  const uint32_t kst = lsmem(ss.k[0]), vst = lsmem(ss.v[0]);
+  RowFetch fk(K, n0, a.ts, tok, half, sub), fv(Vt, n0, a.ts, tok, half, sub);
   int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LSTAGES - 1; ++i) {
     if (i < nblk) {
-      fetch_rows_q4(lsmem(ss.k[i]), K, n0 + 64LL * i, n1, a.ts, tok, half, sub);
-      fetch_rows_q4(lsmem(ss.v[i]), Vt, n0 + 64LL * i, n1, a.ts, tok, half, sub);
+      fk.fetch(kst + i * 8192, oa, ob, 64 * i < left);
+      fv.fetch(vst + i * 8192, oa, ob, 64 * i < left);
     }
     asm volatile("cp.async.commit_group;\n" ::);
   }
+  int st = 0, fst = LSTAGES - 1;   // ring stages of block i and of block i + LSTAGES - 1
   for (int i = 0; i < nblk; ++i) {
-    const int st = i % LSTAGES;
     // Block i's copies are the oldest but LSTAGES - 2 groups in flight. After the barrier every
     // warp is done with block i - 1 (its stage and phi), so that stage is refilled only now.
     asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 2));
@@ -365,30 +327,22 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
     {
       const int f = i + LSTAGES - 1;
       if (f < nblk) {
-        fetch_rows_q4(lsmem(ss.k[f % LSTAGES]), K, n0 + 64LL * f, n1, a.ts, tok, half, sub);
-        fetch_rows_q4(lsmem(ss.v[f % LSTAGES]), Vt, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+        fk.fetch(kst + fst * 8192, oa, ob, 64 * f < left);
+        fv.fetch(vst + fst * 8192, oa, ob, 64 * f < left);
       }
       asm volatile("cp.async.commit_group;\n" ::);
     }
-    const long long n = n0 + 64LL * i + tok;
-    const bool valid = n < n1;
+    const bool valid = 64 * i < left;
     float xa[8], xb[8];
-    read_q4(ss.k[st], tok, half, sub, xa, xb);
+    read_q4(ss.k[st], oa, ob, xa, xb);
     {
       bool sp;
       int row, col;
       view_pos(g, mod_L(g, jb + tok), sp, row, col);
       jb = mod_L(g, jb + 64);
-      if (ZEBRA_LIN_F32X2)
-        features_q4_x2(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
-      else
-        features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
-      if (!valid) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
-      }
+      features_lin<true>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, valid);
     }
-    store_q4(ss.phi, tok, half, sub, xa, xb);
+    store_q4(ss.phi, oa, ob, xa, xb);
     __syncthreads();
     const uint32_t vb = lsmem(ss.v[st]);
 #pragma unroll
@@ -410,6 +364,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
       }
       if (grp == 0) l_mma(acc[4], af, ones, ones);
     }
+    st = ring_next(st, LSTAGES);
+    fst = ring_next(fst, LSTAGES);
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
   float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
@@ -454,13 +410,17 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
   const int nblk = (int)((n1 - n0 + 63) / 64);
+  const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
+  const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
+  const uint32_t qst = lsmem(q_s[0]);
+  RowFetch fq(Q, n0, a.ts, tok, half, sub);
   int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LA_STAGES - 1; ++i) {
-    if (i < nblk) fetch_rows_q4(lsmem(q_s[i]), Q, n0 + 64LL * i, n1, a.ts, tok, half, sub);
+    if (i < nblk) fq.fetch(qst + i * 8192, oa, ob, 64 * i < left);
     asm volatile("cp.async.commit_group;\n" ::);
   }
+  int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i + LA_STAGES - 1
   for (int i = 0; i < nblk; ++i) {
-    const int st = i % LA_STAGES;
     const long long nb = n0 + 64LL * i;
     // Block i's copies are the oldest but LA_STAGES - 2 groups in flight. After the barrier every
     // warp is done with block i - 1, whose stage is refilled only now.
@@ -468,29 +428,20 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     __syncthreads();
     {
       const int f = i + LA_STAGES - 1;
-      if (f < nblk) fetch_rows_q4(lsmem(q_s[f % LA_STAGES]), Q, n0 + 64LL * f, n1, a.ts, tok, half, sub);
+      if (f < nblk) fq.fetch(qst + fst * 8192, oa, ob, 64 * f < left);
       asm volatile("cp.async.commit_group;\n" ::);
     }
-    const long long n = nb + tok;
-    const bool valid = n < n1;
     float xa[8], xb[8];
-    read_q4(q_s[st], tok, half, sub, xa, xb);
+    read_q4(q_s[st], oa, ob, xa, xb);
     {
       bool sp;
       int row, col;
       view_pos(g, mod_L(g, jb + tok), sp, row, col);
       jb = mod_L(g, jb + 64);
-      if (ZEBRA_LIN_F32X2)
-        features_q4_x2(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
-      else
-        features_q4(xa, xb, half, sub, sp, row, col, a.rope, a.eps);
-      if (!valid) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xa[e] = xb[e] = 0.f;
-      }
+      features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, 64 * i < left);
     }
     unsigned char* phi_s = q_s[st];
-    store_q4(phi_s, tok, half, sub, xa, xb);
+    store_q4(phi_s, oa, ob, xa, xb);
     __syncthreads();
     float acc[5][4];
 #pragma unroll
@@ -520,14 +471,13 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       }
     }
     // z = column 64 sits in acc[4][0] (row g4) / acc[4][2] (row g4 + 8) of the quad's first lane.
-#if ZEBRA_LIN_STAGED_OUT
     // Staged output: every warp is done reading the stage as its A operand, so
     // the bf16 output block goes there and leaves as whole 128-byte token rows.
     __syncthreads();
 #pragma unroll
     for (int half2 = 0; half2 < 2; ++half2) {
       const int r = mrow * 16 + g4 + half2 * 8;
-      const float il = 1.0f / __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3);
+      const float il = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3));
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
@@ -544,41 +494,9 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
         *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + ch * 8) =
             *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
     }
+    st = ring_next(st, LA_STAGES);
+    fst = ring_next(fst, LA_STAGES);
   }
-#else
-    // Output from registers: each quad transposes its 4 x 4 words so that lane q4 owns chunk
-    // 4 grp + q4 of both rows and stores it as one 16-byte write (8 rows x 64 bytes per warp store).
-#pragma unroll
-    for (int half2 = 0; half2 < 2; ++half2) {
-      const int r = mrow * 16 + g4 + half2 * 8;
-      const float den = __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3);
-      const float il = 1.0f / den;
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
-                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
-        w[j] = *reinterpret_cast<const uint32_t*>(&v2);
-      }
-      // lane q4 holds word q4 of every chunk j; after the exchange it holds all words of chunk q4
-      uint32_t o[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // send w[q4 ^ k] to lane q4 ^ k, receive that lane's w[q4]: word (q4 ^ k) of chunk q4
-        const int sel = q4 ^ k;
-        const uint32_t send = sel == 0 ? w[0] : sel == 1 ? w[1] : sel == 2 ? w[2] : w[3];
-        const uint32_t got = k == 0 ? send : __shfl_xor_sync(0xffffffffu, send, k);
-        if (sel == 0) o[0] = got;
-        if (sel == 1) o[1] = got;
-        if (sel == 2) o[2] = got;
-        if (sel == 3) o[3] = got;
-      }
-      const long long nn = nb + r;
-      if (nn < n1)
-        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + (4 * grp + q4) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-#endif
   asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
@@ -630,28 +548,51 @@ __global__ void __launch_bounds__(256) linear_state_simt_kernel(const __grid_con
 // --------------------------------------------------------------------------
 // 2. reduce + fold A: state[h][c][i] = sum_j S[c][j] A[i][j]; state[h][c][64] = z[c]
 // --------------------------------------------------------------------------
-// CTA = (head, 8 channel rows): sums its rows of the chunk partials in chunk
-// order (deterministic), then folds A into them.
+// CTA = (head, 8 channel rows), 4 x 130 threads. The CTA's rows are 130
+// 16-byte columns of every chunk partial; thread (slice, j) sums column j over
+// the chunks ch = slice (mod 4), several copies in flight, and the four slice
+// sums add in a fixed order (deterministic). Then the rows fold A in.
 constexpr int RED_ROWS = 8;
-__global__ void __launch_bounds__(256) linear_reduce_kernel(const __grid_constant__ LinearArgs a, int want_bf16) {
+constexpr int RED_VEC = RED_ROWS * 65 / 4;   // 130 16-byte columns
+constexpr int RED_SLICES = 4;
+constexpr int RED_THREADS = RED_VEC * RED_SLICES;
+static_assert(RED_ROWS * 65 % 4 == 0, "whole 16-byte columns");
+__global__ void __launch_bounds__(RED_THREADS) linear_reduce_kernel(const __grid_constant__ LinearArgs a, int want_bf16) {
+  __shared__ float4 P[RED_SLICES][RED_VEC];
   __shared__ float S[RED_ROWS][65];
   __shared__ float As[64][65];
   const int h = blockIdx.x, c0 = blockIdx.y * RED_ROWS, tid = threadIdx.x;
   const Geo& g = a.g;
-  for (int e = tid; e < RED_ROWS * 65; e += 256) {
-    float s = 0.f;
-    const float* p = a.part + ((size_t)h * 64 + c0) * 65 + e;
-    for (int ch = 0; ch < a.chunks; ++ch) s += p[(size_t)ch * g.H * 64 * 65];
-    S[e / 65][e % 65] = s;
+  {
+    const int sl = tid / RED_VEC, j = tid - sl * RED_VEC;
+    // rows c0.. of head h start 8 x 65 x 4 = 2,080 bytes apart: 16-byte aligned
+    const float4* p = reinterpret_cast<const float4*>(a.part + ((size_t)h * 64 + c0) * 65) + j;
+    const size_t cstride = (size_t)g.H * 64 * 65 / 4;   // 16-byte columns per chunk partial
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int ch = sl; ch < a.chunks; ch += RED_SLICES) {
+      const float4 v = __ldg(p + (size_t)ch * cstride);
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    P[sl][j] = s;
   }
-  for (int e = tid; e < 64 * 64; e += 256) {
+  for (int e = tid; e < 64 * 64; e += RED_THREADS) {
     const int i = e / 64, j = e % 64;
     As[i][j] = a.A ? a.A[(size_t)h * 64 * 64 + e] : (i == j ? 1.f : 0.f);
   }
   __syncthreads();
+  {
+    const float* q = reinterpret_cast<const float*>(&P[0][0]);
+    constexpr int E = RED_ROWS * 65;
+    for (int e = tid; e < E; e += RED_THREADS) S[e / 65][e % 65] = (q[e] + q[E + e]) + (q[2 * E + e] + q[3 * E + e]);
+  }
+  __syncthreads();
   float* st = a.state + (size_t)h * 64 * 65;
   __nv_bfloat16* sb = want_bf16 ? static_cast<__nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64 : nullptr;
-  for (int e = tid; e < RED_ROWS * NB; e += 256) {
+  for (int e = tid; e < RED_ROWS * NB; e += RED_THREADS) {
     const int r = e / NB, i = e % NB, c = c0 + r;  // channel c, output column i
     float val = 0.f;
     if (i < 64) {
@@ -716,7 +657,7 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_state_q4_kernel")) return rc;
   {
     ProfScope prof("linear_reduce", st);
-    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), 256, 0, st>>>(a, 1);
+    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), RED_THREADS, 0, st>>>(a, 1);
   }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
@@ -739,7 +680,7 @@ int launch_linear<float>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_state_simt_kernel")) return rc;
   {
     ProfScope prof("linear_reduce", st);
-    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), 256, 0, st>>>(a, 0);
+    linear_reduce_kernel<<<dim3(a.g.H, 64 / RED_ROWS), RED_THREADS, 0, st>>>(a, 0);
   }
   count_launch();
   if (int rc = check_launch("linear_reduce_kernel")) return rc;

@@ -74,12 +74,12 @@ extern "C" int zebra_linear_attn_noalloc(const zebra_geom* g, zebra_dtype dt, co
   if (int rc = check_ptr16(out, "out")) return rc;
 
   // Scratch layout: per-chunk partials, folded state, bf16 state operand,
-  // rotation table. The token chunks are those of zebra_linear_attn (so the two
+  // rotation tables. The token chunks are those of zebra_linear_attn (so the two
   // entry points sum in the same order and agree bit for bit) as long as their
   // partials fit; otherwise the chunks grow until they do.
   const int maxpos = G.Hp > G.Wp ? G.Hp : G.Wp;
   const size_t fixed = align256((size_t)G.H * 64 * 65 * 4) + align256((size_t)G.H * 72 * 64 * 2) +
-                       align256((size_t)maxpos * 16 * sizeof(float2));
+                       align256((size_t)maxpos * 16 * sizeof(float2)) + align256((size_t)maxpos * 8 * sizeof(float4));
   const size_t per_chunk = (size_t)G.H * 64 * 65 * 4;
   if (fixed + align256(per_chunk) > NOALLOC_BYTES) {
     set_error("this geometry needs more scratch than the built-in 16 MiB area; use zebra_linear_attn");
@@ -107,13 +107,14 @@ extern "C" int zebra_linear_attn_noalloc(const zebra_geom* g, zebra_dtype dt, co
   a.state = c.take<float>((size_t)G.H * 64 * 65);
   a.state_b = c.take<__nv_bfloat16>((size_t)G.H * 72 * 64);
   float2* rope = c.take<float2>((size_t)maxpos * 16);
+  float4* rope_g = c.take<float4>((size_t)maxpos * 8);
   if (c.used() > NOALLOC_BYTES) {
     set_error("scratch layout exceeds the built-in area");
     return ZEBRA_ERR_UNSUPPORTED;
   }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (int rc = launch_rope_table(rope, maxpos, (double)rope_base, st)) return rc;
+  if (int rc = launch_rope_table(rope, rope_g, maxpos, (double)rope_base, st)) return rc;
   a.g = G;
   a.q = q;
   a.k = k;
@@ -124,6 +125,8 @@ extern "C" int zebra_linear_attn_noalloc(const zebra_geom* g, zebra_dtype dt, co
   a.b = b;
   a.eps = eps;
   a.rope = rope;
+  a.rope_g = rope_g;
+  a.maxpos = maxpos;
   a.chunks = (int)chunks;
   a.chunk_tokens = (int)ct;
   a.out = out;

@@ -166,13 +166,21 @@ __global__ void __launch_bounds__(128) pack_special_kernel(SpecialArgs<T> a) {
 }
 
 // cos/sin table of the 2D rotation: tab[pos*16 + j] = (cos, sin)(pos * base^(-j/16)),
-// evaluated in double precision.
-__global__ void rope_table_kernel(float2* tab, int maxpos, double base) {
+// evaluated in double precision. tab_g (optional) holds the same values as the
+// packed-pair operands of the linear kernels, group i of the pairs j = 2i,
+// 2i + 1 before position: tab_g[i*maxpos + pos] = (cos_j, cos_j+1, sin_j, sin_j+1).
+__global__ void rope_table_kernel(float2* tab, float4* tab_g, int maxpos, double base) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= maxpos * 16) return;
   const int pos = i / 16, j = i % 16;
   const double ang = (double)pos * pow(base, -(double)j / 16.0);
-  tab[i] = make_float2((float)cos(ang), (float)sin(ang));
+  const float c = (float)cos(ang), s = (float)sin(ang);
+  tab[i] = make_float2(c, s);
+  if (tab_g) {
+    float* g = reinterpret_cast<float*>(tab_g + (size_t)(j / 2) * maxpos + pos);
+    g[j & 1] = c;
+    g[2 + (j & 1)] = s;
+  }
 }
 
 template <typename T>
@@ -197,10 +205,10 @@ int launch_pack_special(const SpecialArgs<T>& a, int ntensors, cudaStream_t st) 
   return check_launch("pack_special_kernel");
 }
 
-int launch_rope_table(float2* tab, int maxpos, double base, cudaStream_t st) {
+int launch_rope_table(float2* tab, float4* tab_g, int maxpos, double base, cudaStream_t st) {
   const int n = maxpos * 16;
   ProfScope prof("rope_table", st);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, maxpos, base);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, tab_g, maxpos, base);
   count_launch();
   return check_launch("rope_table_kernel");
 }
