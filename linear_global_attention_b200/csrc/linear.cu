@@ -26,6 +26,8 @@
 //     column, add b, stage the bf16 block in the same ring stage and store
 //     whole 128-byte token rows.
 // The fp32 variants run the same three steps with plain fp32 arithmetic.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -382,11 +384,38 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   }
 }
 
-__global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ LinearArgs a) {
+// Apply kernel shared memory: the Q ring, one output block, the B operand.
+// Every piece starts on a 1024-byte boundary, so the swizzled offsets lswz()
+// are the 128-byte swizzle of the tensor-memory-access unit's copies.
+struct ApplySmem {
+  unsigned char q[LA_STAGES][64 * 128];
+  unsigned char out[64 * 128];
+  unsigned char b[NB * 128];
+};
+struct ApplyParams {
+  CUtensorMap tout;   // out as [N][H][64] bf16, box 64 channels x 1 head x 64 tokens, 128-byte swizzle
+  LinearArgs a;
+};
+
+__device__ __forceinline__ void l_stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t l_pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ ApplyParams prm) {
   // Q ring; f(Q) of a block overwrites its own stage in place (each thread rewrites exactly the
-  // 32 bytes it read), so the MMA reads its A operand from the stage.
-  __shared__ __align__(128) unsigned char q_s[LA_STAGES][64 * 128];
-  __shared__ __align__(128) unsigned char b_s[NB * 128];
+  // 32 bytes it read), so the MMA reads its A operand from the stage. The bf16 output block
+  // goes to its own buffer, which one thread stores by a bulk tensor copy (rows past the
+  // tensor's last token are not written; chunks start on multiples of 64 tokens, so only the
+  // last chunk has such rows).
+  extern __shared__ unsigned char apply_smem_raw[];
+  ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(apply_smem_raw) + 1023) & ~uintptr_t(1023));
+  const LinearArgs& a = prm.a;
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;   // grid (head, chunk), as in the state kernel
@@ -396,11 +425,11 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
   for (int i = tid; i < NB * 8; i += LQ_THREADS) {
     const int r = i >> 3, c = i & 7;
-    *reinterpret_cast<uint4*>(b_s + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
+    *reinterpret_cast<uint4*>(sm.b + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
   }
   const int tok = tid >> 2, half = (tid >> 1) & 1, sub = tid & 1;
   const int mrow = warp & 3, grp = warp >> 2;   // token rows 16 mrow .., column group
-  const int g4 = lane >> 2, q4 = lane & 3;
+  const int q4 = lane & 3;
   float bias[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -408,11 +437,14 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     bias[2 * j] = a.b ? a.b[h * 64 + c] : 0.f;
     bias[2 * j + 1] = a.b ? a.b[h * 64 + c + 1] : 0.f;
   }
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
   const int nblk = (int)((n1 - n0 + 63) / 64);
   const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
-  const uint32_t qst = lsmem(q_s[0]);
+  const uint32_t qst = lsmem(sm.q[0]), bst = lsmem(sm.b), ost = lsmem(sm.out);
+  // stmatrix row addresses of the output block: lane 8 k + r gives row r of matrix k, matrices
+  // (rows 0-7, n-block 2x), (rows 8-15, 2x), (rows 0-7, 2x + 1), (rows 8-15, 2x + 1) of store x
+  const uint32_t o_st0 = ost + lswz(mrow * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * grp + (lane >> 4));
+  const uint32_t o_st1 = ost + lswz(mrow * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * grp + 2 + (lane >> 4));
   RowFetch fq(Q, n0, a.ts, tok, half, sub);
   int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LA_STAGES - 1; ++i) {
@@ -421,7 +453,6 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   }
   int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i + LA_STAGES - 1
   for (int i = 0; i < nblk; ++i) {
-    const long long nb = n0 + 64LL * i;
     // Block i's copies are the oldest but LA_STAGES - 2 groups in flight. After the barrier every
     // warp is done with block i - 1, whose stage is refilled only now.
     asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
@@ -432,7 +463,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       asm volatile("cp.async.commit_group;\n" ::);
     }
     float xa[8], xb[8];
-    read_q4(q_s[st], oa, ob, xa, xb);
+    read_q4(sm.q[st], oa, ob, xa, xb);
     {
       bool sp;
       int row, col;
@@ -440,9 +471,11 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       jb = mod_L(g, jb + 64);
       features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, 64 * i < left);
     }
-    unsigned char* phi_s = q_s[st];
-    store_q4(phi_s, oa, ob, xa, xb);
+    store_q4(sm.q[st], oa, ob, xa, xb);
+    // the previous block's output copy has read the output buffer before anyone rewrites it
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     __syncthreads();
+    const uint32_t phi = qst + st * 8192;
     float acc[5][4];
 #pragma unroll
     for (int j = 0; j < 5; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
@@ -451,53 +484,51 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       uint32_t af[4];
       {
         const int mi = lane >> 3, ri = lane & 7;
-        l_ldsm_x4(lsmem(phi_s) + lswz(mrow * 16 + (mi & 1) * 8 + ri, 2 * ks + (mi >> 1)), af[0], af[1], af[2],
-                  af[3]);
+        l_ldsm_x4(phi + lswz(mrow * 16 + (mi & 1) * 8 + ri, 2 * ks + (mi >> 1)), af[0], af[1], af[2], af[3]);
       }
 #pragma unroll
       for (int n2 = 0; n2 < 2; ++n2) {
         const int np = 2 * grp + n2;   // state columns 16 np .. 16 np + 15
         const int mi = lane >> 3, ri = lane & 7;
         uint32_t b0, b1, b2, b3;
-        l_ldsm_x4(lsmem(b_s) + lswz(np * 16 + (mi >> 1) * 8 + ri, 2 * ks + (mi & 1)), b0, b1, b2, b3);
+        l_ldsm_x4(bst + lswz(np * 16 + (mi >> 1) * 8 + ri, 2 * ks + (mi & 1)), b0, b1, b2, b3);
         l_mma(acc[2 * n2], af, b0, b1);
         l_mma(acc[2 * n2 + 1], af, b2, b3);
       }
       {   // the z column: both column groups compute it, so no exchange is needed
         const int mi = (lane >> 3) & 1, ri = lane & 7;
         uint32_t b0, b1;
-        l_ldsm_x2(lsmem(b_s) + lswz(64 + ri, 2 * ks + mi), b0, b1);
+        l_ldsm_x2(bst + lswz(64 + ri, 2 * ks + mi), b0, b1);
         l_mma(acc[4], af, b0, b1);
       }
     }
     // z = column 64 sits in acc[4][0] (row g4) / acc[4][2] (row g4 + 8) of the quad's first lane.
-    // Staged output: every warp is done reading the stage as its A operand, so
-    // the bf16 output block goes there and leaves as whole 128-byte token rows.
-    __syncthreads();
-#pragma unroll
-    for (int half2 = 0; half2 < 2; ++half2) {
-      const int r = mrow * 16 + g4 + half2 * 8;
-      const float il = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][half2 * 2], lane & ~3));
+    {
+      const float il0 = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][0], lane & ~3));
+      const float il1 = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][2], lane & ~3));
+      uint32_t w[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(acc[j][half2 * 2], il, bias[2 * j]),
-                                                        fmaf(acc[j][half2 * 2 + 1], il, bias[2 * j + 1]));
-        *reinterpret_cast<__nv_bfloat162*>(phi_s + lswz(r, 4 * grp + j) + 4 * q4) = v2;
+        w[j][0] = l_pack_bf16(fmaf(acc[j][0], il0, bias[2 * j]), fmaf(acc[j][1], il0, bias[2 * j + 1]));
+        w[j][1] = l_pack_bf16(fmaf(acc[j][2], il1, bias[2 * j]), fmaf(acc[j][3], il1, bias[2 * j + 1]));
       }
+      l_stsm_x4(o_st0, w[0][0], w[0][1], w[1][0], w[1][1]);
+      l_stsm_x4(o_st1, w[2][0], w[2][1], w[3][0], w[3][1]);
     }
+    // the generic-proxy writes of the block become visible to the bulk copy
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     __syncthreads();
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int idx = tid + LQ_THREADS * c, r = idx >> 3, ch = idx & 7;
-      const long long nn = nb + r;
-      if (nn < n1)
-        *reinterpret_cast<uint4*>(out + (nn * g.H + h) * D + ch * 8) =
-            *reinterpret_cast<const uint4*>(phi_s + lswz(r, ch));
+    if (tid == 0) {
+      asm volatile(
+          "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n"
+          "cp.async.bulk.commit_group;\n" ::"l"(&prm.tout), "r"(0), "r"(h), "r"((int)(n0 + 64LL * i)), "r"(ost)
+          : "memory");
     }
     st = ring_next(st, LA_STAGES);
     fst = ring_next(fst, LA_STAGES);
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
+  if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
 }
 
 // --------------------------------------------------------------------------
@@ -645,9 +676,41 @@ int linear_chunks(const Geo& g, int* chunk_tokens) {
   return (int)chunks;
 }
 
+// 3D bf16 map over out = [N][H][64] (contiguous), box 64 channels x 1 head x 64 tokens, 128-byte swizzle.
+static bool make_out_map(CUtensorMap* m, void* out, const Geo& g) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[3] = {64, (cuuint64_t)g.H, (cuuint64_t)g.N};
+  cuuint64_t strides[2] = {128, (cuuint64_t)g.H * 128};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <>
 int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
+  // the apply kernel's output copies cover whole 64-token blocks up to the tensor's end,
+  // so only the last chunk may end inside a block
+  if (a.chunk_tokens % 64) {
+    set_error("linear stage: token chunks must be multiples of 64 tokens");
+    return ZEBRA_ERR_UNSUPPORTED;
+  }
+  ApplyParams prm;
+  prm.a = a;
+  if (!make_out_map(&prm.tout, a.out, a.g)) {
+    set_error("cuTensorMapEncodeTiled failed (linear output)");
+    return ZEBRA_ERR_CUDA;
+  }
   {
     ProfScope prof("linear_state", st);
     cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
@@ -663,7 +726,9 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (int rc = check_launch("linear_reduce_kernel")) return rc;
   {
     ProfScope prof("linear_apply", st);
-    linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, 0, st>>>(a);
+    const int smem = (int)sizeof(ApplySmem) + 1024;   // + alignment of the base to 1024 bytes
+    cudaFuncSetAttribute(linear_apply_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(prm);
   }
   count_launch();
   return check_launch("linear_apply_q4_kernel");
