@@ -126,15 +126,23 @@ struct StateSmem {
   unsigned char v[LSTAGES][64 * 128];
 };
 
-// 256 threads, 64 tokens per step. Thread (tok = tid / 4, part = tid % 4) owns
+// 256 threads, 64 tokens per step. Thread (tok = token_of(tid), part = tid % 4) owns
 // 16 channels of its token that form 8 whole rotation pairs: half = part / 2
 // (channels 0-31 turn by patch row, 32-63 by column), sub = part % 2 (pairs
 // j = 8 sub .. 8 sub + 7 of the half): the "a" channels 32 half + 8 sub .. + 7
 // and their partners 16 further. The four threads of a token combine the RMS
-// norm, the maximum and the sum with two shuffles each. 8 warps split the
+// norm and the sum with two shuffles each. 8 warps split the
 // 64 x 72 contraction: rows 16 (warp % 4) .. + 15, columns 0-31 plus the
 // z column (warp / 4 = 0) or columns 32-63 (warp / 4 = 1).
 constexpr int LQ_THREADS = 256;
+// Token of thread tid: the quads of a warp take its 8 tokens in the order 0 2 1 3 4 6 5 7,
+// so the two tokens of each 8-lane phase of a 16-byte shared access are rows r and r + 2.
+// Their chunk sets {0 1 4 5} and {2 3 6 7} (before the swizzle's XOR with the row) are
+// disjoint, and the reads, writes and copies of the rows are free of bank conflicts.
+__device__ __forceinline__ int token_of(int tid) {
+  const int q = (tid >> 2) & 7;
+  return (tid >> 5) * 8 + ((q & 4) | ((q & 1) << 1) | ((q >> 1) & 1));
+}
 
 // This thread's part of its token's row in one tensor: two 16-byte pieces per
 // 64-token block (the "a" channels and, 2 chunks on, their partners), copied
@@ -157,6 +165,8 @@ struct RowFetch {
 };
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+// Inline PTX rather than the __ffma2_rn family: with those the state kernel
+// spilled and ran 3% slower.
 __device__ __forceinline__ float2 l_fma2(float2 a, float2 b, float2 c) {
   float2 d;
   asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2,%3};\n mov.b64 rb, {%4,%5};\n mov.b64 rc, {%6,%7};\n"
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
   const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
   const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v) + (long long)h * a.hs;
-  const int tok = tid >> 2, half = (tid >> 1) & 1, sub = tid & 1;
+  const int tok = token_of(tid), half = (tid >> 1) & 1, sub = tid & 1;
   const int mrow = warp & 3, grp = warp >> 2;   // channel rows 16 mrow .., column group
   float acc[5][4];
 #pragma unroll
@@ -427,7 +437,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     const int r = i >> 3, c = i & 7;
     *reinterpret_cast<uint4*>(sm.b + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
   }
-  const int tok = tid >> 2, half = (tid >> 1) & 1, sub = tid & 1;
+  const int tok = token_of(tid), half = (tid >> 1) & 1, sub = tid & 1;
   const int mrow = warp & 3, grp = warp >> 2;   // token rows 16 mrow .., column group
   const int q4 = lane & 3;
   float bias[8];
