@@ -71,8 +71,9 @@ def peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum over every launch of one call
 # at 1,024 views x 1 head: bytes per (head, query tile) work item.
 # Valid only for the kernel sources it was taken on; otherwise traffic is null.
-SPARSE_TRAFFIC = {"bytes_per_item": 672131, "sources_sha1": "2c41b12bef9f1cd386aaad02353f62ccdf391607"}
-SPARSE_SOURCES = ("linear_global_attention_b200/csrc/attn_tc.cuh", "linear_global_attention_b200/csrc/attn.cu")
+SPARSE_TRAFFIC = {"bytes_per_item": 672131, "sources_sha1": "012db3d21873ee1f105e9169eafbf2ac030aa919"}
+SPARSE_SOURCES = ("linear_global_attention_b200/csrc/attn_tc.cuh", "linear_global_attention_b200/csrc/attn.cu",
+                  "linear_global_attention_b200/csrc/tc_prims.cuh")
 
 
 def sparse_sources_sha1() -> str:

@@ -237,7 +237,11 @@ ZEBRA_API int zebra_sync_status(void* stream);
  * so that the tensor-core warp's wait for that block's keys runs out: the
  * kernel then records ZEBRA_ERR_TIMEOUT in the sticky status word, lets its
  * copies and MMAs in flight land (each wait bounded again), frees its tensor
- * memory and exits, leaving the outputs of the affected rows undefined.
+ * memory and exits, leaving the outputs of the affected rows undefined. The
+ * same call sets the wait limit of the bf16 linear stage's state kernel and,
+ * when `block` >= 0, makes it leave out the tensor-core MMAs of block `block`
+ * (64 tokens) of each token chunk, so that its wait for their completion runs
+ * out the same way (the stage's outputs are then undefined).
  * zebra_sync_status() reports the timeout. zebra_debug_inject(-1, 0) restores
  * normal operation. Every wait stays bounded, so no setting can hang the GPU.
  * Returns ZEBRA_OK, ZEBRA_ERR_CUDA or ZEBRA_ERR_UNSUPPORTED (no sm_100 device). */

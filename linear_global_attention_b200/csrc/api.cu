@@ -784,7 +784,8 @@ long long zebra_profile_report(char* buf, size_t len) {
 
 int zebra_debug_inject(int32_t block, uint64_t wait_ns) {
   ZTRY(check_device());
-  if (set_debug_inject(block, (unsigned long long)wait_ns) != ZEBRA_OK)
+  if (set_debug_inject(block, (unsigned long long)wait_ns) != ZEBRA_OK ||
+      set_linear_debug_inject(block, (unsigned long long)wait_ns) != ZEBRA_OK)
     return fail(ZEBRA_ERR_CUDA, "setting the test hook failed");
   return ZEBRA_OK;
 }
@@ -794,7 +795,10 @@ int zebra_sync_status(void* stream) {
   if (e != cudaSuccess) return fail(ZEBRA_ERR_CUDA, cudaGetErrorString(e));
   int st = 0;
   if (read_and_clear_status(&st) != ZEBRA_OK) return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
-  if (st) return fail(ZEBRA_ERR_TIMEOUT, "a device-side wait gave up (kernel aborted; outputs are invalid)");
+  int st_lin = 0;
+  if (read_and_clear_linear_status(&st_lin) != ZEBRA_OK)
+    return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
+  if (st || st_lin) return fail(ZEBRA_ERR_TIMEOUT, "a device-side wait gave up (kernel aborted; outputs are invalid)");
   if (read_and_clear_affine_status(&st) != ZEBRA_OK)
     return fail(ZEBRA_ERR_CUDA, "reading the device status word failed");
   if (st) return fail(ZEBRA_ERR_NUMERIC, "an affine fit met a system that is not positive definite (A, b are NaN)");

@@ -51,6 +51,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "tc_prims.cuh"
+
 namespace zebra {
 
 __device__ int g_status;   // sticky device status word (0 = ok)
@@ -213,47 +215,6 @@ struct alignas(64) Params {
   int item0;   // first work item of this launch; CTA b takes item0 + b
 };
 
-__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ unsigned long long gtime() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
-}
-// One test of the phase; while it is incomplete the thread sleeps in hardware
-// (up to SUSPEND_NS) and wakes when the phase completes, so waiting warps do
-// not take issue slots from the softmax warps.
-constexpr uint32_t SUSPEND_NS = 100000;
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-#ifdef ZEBRA_TC_WAIT_SPIN
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity)
-      : "memory");
-#else
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity), "r"(SUSPEND_NS)
-      : "memory");
-#endif
-  return ok != 0;
-}
-
 // Drain wait after an abort: waits for the phase whatever the abort flag says
 // (copies or MMAs still in flight must land before the CTA frees its shared
 // memory and TMEM), and gives up after `limit_ns`.
@@ -347,33 +308,6 @@ __device__ __forceinline__ int tile_groups(const Geo& g, int u) {
   return (s.rows * s.cols + 7) >> 3;
 }
 
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// shared-memory matrix descriptors (sm_100 format: start>>4 at [0,14), LBO>>4 at
-// [16,30), SBO>>4 at [32,46), version 1 at [46,48), layout at [61,64): 2 = 128B swizzle)
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// K-major 64-row tile with 128-byte rows: 8-row groups 1024 bytes apart
-__device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return desc_sw128(addr, 16, 1024); }
-// MN-major tile: the 64 N values of a K row fill one 128-byte swizzle atom,
-// K rows 128 bytes apart, 8-row groups 1024 bytes apart
-__device__ __forceinline__ uint64_t desc_mn(uint32_t addr) { return desc_sw128(addr, 8192, 1024); }
-
-// instruction descriptor of kind::f16: D fp32, A/B bf16, M = 64, N = n
-__host__ __device__ constexpr uint32_t idesc(bool b_mn_major, uint32_t n = 64) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) |
-         ((64u >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id, uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(id), "r"(accum));
-}
 // S = Q K^T (K = 64: four K = 16 steps) issued by one elected lane of the
 // converged warp, then commits to `bar0` and `bar1`. One asm block keeps the
 // issue cost per MMA low.
@@ -461,17 +395,6 @@ __device__ __forceinline__ void tmem_st_p(uint32_t taddr, const uint32_t (&pk)[8
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ bool elect_one() {
-  uint32_t e;
-  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
-  return e != 0;
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(bar))
-               : "memory");
-}
-
 // 16 TMEM lanes x 64 fp32 columns -> 32 registers (m16n8 accumulator layout per 8 columns)
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* r) {
   uint32_t* u = reinterpret_cast<uint32_t*>(r);
@@ -498,14 +421,6 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float* r) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 16 TMEM lanes x 8 fp32 columns -> 4 registers (rows g4 and g4 + 8, columns 2 q4 and 2 q4 + 1)
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
-  uint32_t* u = reinterpret_cast<uint32_t*>(r);
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
-               : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* r) {
   const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
   asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(u[0]), "r"(u[1]),

@@ -117,6 +117,9 @@ struct LinearArgs {
 };
 template <typename T> int launch_linear(const LinearArgs& a, cudaStream_t st);
 int linear_chunks(const Geo& g, int* chunk_tokens);
+// sticky status word and error-path test hook of the bf16 linear state kernel (current device)
+int read_and_clear_linear_status(int* out);
+int set_linear_debug_inject(int block, unsigned long long wait_ns);
 
 // ---- closed-form affine fit ----
 constexpr int AF_D = 64;

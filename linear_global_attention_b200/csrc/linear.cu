@@ -15,9 +15,11 @@
 //
 // Three kernels:
 //  1. state:  per (head, token chunk) CTA: prologue on K in registers (4 threads
-//     per token, 16 channels each), f(K) -> shared as bf16, then
-//     [S | z] += f(K)^T [V | 1] on mma.sync (M = 64 channels, N = 64 + 8 with a
-//     column of ones for z, K = 64 tokens), fp32 partials per chunk.
+//     per token, 16 channels each), f(K) -> its own K ring stage as bf16, then
+//     [S | z] += f(K)^T [V | ones] on the tcgen05 tensor cores (M = 64 channels,
+//     N = 64 for S and 16 for z, K = 64 tokens per block, fp32 accumulators in
+//     tensor memory; one thread issues, the next block's prologue overlaps),
+//     fp32 partials per chunk.
 //  2. reduce: per head, sums the chunk partials in a fixed order (deterministic),
 //     forms S' = S A^T, and writes the bf16 B operand [S' | z] of the apply kernel.
 //  3. apply:  per (head, token chunk) CTA: prologue on Q (f(Q) overwrites its
@@ -32,6 +34,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tc_prims.cuh"
 
 namespace zebra {
 
@@ -120,11 +123,61 @@ constexpr int LSTAGES = 3;
 #endif
 constexpr int LA_STAGES = ZEBRA_LIN_ASTAGES;   // Q ring depth of the apply kernel
 
+// State kernel shared memory (base aligned to 1024 bytes, like every tile in it):
+// the K and V rings (f(K) overwrites its own K stage), the all-ones B operand of
+// the z MMAs, the MMA completion barrier and the tensor-memory base.
 struct StateSmem {
-  unsigned char phi[64 * 128];
   unsigned char k[LSTAGES][64 * 128];
   unsigned char v[LSTAGES][64 * 128];
+  unsigned char ones[16 * 128];
+  uint64_t mma_bar;
+  uint32_t tmem_base;
+  int abort;
 };
+constexpr uint32_t STATE_TMEM_COLS = 128;   // [S | z]: columns 0-63 and 64-79
+
+// Bounded waits of the linear stage's tcgen05 kernels: the sticky status word,
+// the wait limit, and the error-path test hook (the token block of each chunk
+// whose MMAs the state kernel leaves out; -1 = none).
+__device__ int g_lin_status;
+__device__ unsigned long long g_lin_wait_ns = 2000000000ull;
+__device__ int g_lin_inject_block = -1;
+
+int set_linear_debug_inject(int block, unsigned long long wait_ns) {
+  const int b = block < 0 ? -1 : block;
+  const unsigned long long w = wait_ns ? wait_ns : 2000000000ull;
+  if (cudaMemcpyToSymbol(g_lin_inject_block, &b, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_lin_wait_ns, &w, sizeof(w)) != cudaSuccess)
+    return ZEBRA_ERR_CUDA;
+  return ZEBRA_OK;
+}
+
+int read_and_clear_linear_status(int* out) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_lin_status, sizeof(int)) != cudaSuccess) return ZEBRA_ERR_CUDA;
+  const int z = 0;
+  if (cudaMemcpyToSymbol(g_lin_status, &z, sizeof(int)) != cudaSuccess) return ZEBRA_ERR_CUDA;
+  *out = v;
+  return ZEBRA_OK;
+}
+
+// One thread waits for the phase of `parity` of `b`; after g_lin_wait_ns it
+// records ZEBRA_ERR_TIMEOUT and returns false.
+__device__ __noinline__ bool lin_wait(uint64_t* b, uint32_t parity) {
+  const unsigned long long limit = *(volatile unsigned long long*)&g_lin_wait_ns;
+  const unsigned long long t0 = tc::gtime();
+  while (!tc::mbar_try(b, parity)) {
+    if (tc::gtime() - t0 > limit) {
+      atomicExch(&g_lin_status, ZEBRA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
 
 // 256 threads, 64 tokens per step. Thread (tok = token_of(tid), part = tid % 4) owns
 // 16 channels of its token that form 8 whole rotation pairs: half = part / 2
@@ -299,9 +352,35 @@ __device__ __forceinline__ void store_q4(unsigned char* tile, uint32_t oa, uint3
 
 __device__ __forceinline__ int ring_next(int s, int n) { return s + 1 == n ? 0 : s + 1; }
 
+// [S | z] += f(K)^T [V | ones] of one 64-token block on the tensor cores: A = f(K)^T
+// (MN-major: the K stage's rows are tokens, its 64 channels the M dimension),
+// B = V (MN-major) for S (N = 64, TMEM columns 0-63) and the all-ones tile
+// (K-major, N = 16) for z (columns 64-79); K = 16 tokens per MMA, 2,048 bytes of
+// the stages per step. acc = 0 starts both accumulators. One elected lane of
+// the warp issues the eight MMAs and the commit to `bar`.
+__device__ __forceinline__ void state_mma_elect(uint32_t tmem, uint64_t fk, uint64_t v, uint64_t ones, uint32_t acc,
+                                                uint64_t* bar) {
+  constexpr uint32_t ID_S = tc::idesc(true, 64, true), ID_Z = tc::idesc(false, 16, true);
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, %16, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %14, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %9, %14, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %2, %10, %15, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %3, %11, %15, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %4, %12, %15, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %5, %13, %15, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%17];\n}\n"
+      ::"r"(tmem), "r"(tmem + 64), "l"(fk), "l"(fk + 128), "l"(fk + 256), "l"(fk + 384), "l"(v), "l"(v + 128),
+      "l"(v + 256), "l"(v + 384), "l"(ones), "l"(ones + 2), "l"(ones + 4), "l"(ones + 6), "r"(ID_S), "r"(ID_Z),
+      "r"(acc), "r"(tc::saddr(bar))
+      : "memory");
+}
+
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __grid_constant__ LinearArgs a) {
-  extern __shared__ __align__(128) unsigned char state_smem[];
-  StateSmem& ss = *reinterpret_cast<StateSmem*>(state_smem);
+  extern __shared__ unsigned char state_smem_raw[];
+  StateSmem& ss = *reinterpret_cast<StateSmem*>(align1024(state_smem_raw));
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;   // grid (head, chunk): the heads of the same tokens run together
@@ -310,19 +389,12 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(a.k) + (long long)h * a.hs;
   const __nv_bfloat16* Vt = static_cast<const __nv_bfloat16*>(a.v) + (long long)h * a.hs;
   const int tok = token_of(tid), half = (tid >> 1) & 1, sub = tid & 1;
-  const int mrow = warp & 3, grp = warp >> 2;   // channel rows 16 mrow .., column group
-  float acc[5][4];
-#pragma unroll
-  for (int j = 0; j < 5; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  const int g4 = lane >> 2;
-  const uint32_t ones = g4 == 0 ? 0x3f803f80u : 0u;  // bf16 pair (1, 1) in column 64
 
   const int nblk = (int)((n1 - n0 + 63) / 64);
   const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
   const uint32_t kst = lsmem(ss.k[0]), vst = lsmem(ss.v[0]);
   RowFetch fk(K, n0, a.ts, tok, half, sub), fv(Vt, n0, a.ts, tok, half, sub);
-  int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LSTAGES - 1; ++i) {
     if (i < nblk) {
       fk.fetch(kst + i * 8192, oa, ob, 64 * i < left);
@@ -330,20 +402,31 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
     }
     asm volatile("cp.async.commit_group;\n" ::);
   }
+  if (tid == 0) {
+    tc::mbar_init(&ss.mma_bar, 1);
+    ss.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = tid; i < 16 * 128 / 4; i += LQ_THREADS) reinterpret_cast<uint32_t*>(ss.ones)[i] = 0x3F803F80u;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the ones tile is read by the tensor cores
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(lsmem(&ss.tmem_base)),
+                 "r"(STATE_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = ss.tmem_base;
+  const uint64_t d_k0 = tc::desc_mn(kst), d_v0 = tc::desc_mn(vst), d_ones = tc::desc_k(lsmem(ss.ones));
+  const int inject = *(volatile int*)&g_lin_inject_block;
+  int issued = 0, waited = 0;   // thread 0: blocks whose MMAs went out / were seen complete
+  int jb = (int)(n0 % g.L);   // view position of the current block's first token
   int st = 0, fst = LSTAGES - 1;   // ring stages of block i and of block i + LSTAGES - 1
   for (int i = 0; i < nblk; ++i) {
-    // Block i's copies are the oldest but LSTAGES - 2 groups in flight. After the barrier every
-    // warp is done with block i - 1 (its stage and phi), so that stage is refilled only now.
+    // Block i's copies are the oldest but LSTAGES - 2 groups in flight.
     asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 2));
     __syncthreads();
-    {
-      const int f = i + LSTAGES - 1;
-      if (f < nblk) {
-        fk.fetch(kst + fst * 8192, oa, ob, 64 * f < left);
-        fv.fetch(vst + fst * 8192, oa, ob, 64 * f < left);
-      }
-      asm volatile("cp.async.commit_group;\n" ::);
-    }
     const bool valid = 64 * i < left;
     float xa[8], xb[8];
     read_q4(ss.k[st], oa, ob, xa, xb);
@@ -354,44 +437,78 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
       jb = mod_L(g, jb + 64);
       features_lin<true>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, valid);
     }
-    store_q4(ss.phi, oa, ob, xa, xb);
+    store_q4(ss.k[st], oa, ob, xa, xb);   // f(K) over its own K rows
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+    // block i - 1's MMAs are done with their stages before block i + LSTAGES - 1 refills them
+    if (tid == 0 && i > 0) {
+      if (lin_wait(&ss.mma_bar, (i - 1) & 1))
+        waited = i;
+      else
+        ss.abort = 1;
+    }
     __syncthreads();
-    const uint32_t vb = lsmem(ss.v[st]);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {   // 16 tokens per k-step
-      uint32_t af[4];
-      {
-        const int mi = lane >> 3, ri = lane & 7;
-        l_ldsm_x4_t(lsmem(ss.phi) + lswz(ks * 16 + (mi >> 1) * 8 + ri, mrow * 2 + (mi & 1)), af[0], af[1], af[2],
-                    af[3]);
+    if (ss.abort) break;
+    if (warp == 0 && i != inject) {
+      tc::fence_after();
+      state_mma_elect(tmem, d_k0 + st * 512, d_v0 + st * 512, d_ones, i > 0 ? 1u : 0u, &ss.mma_bar);
+      issued = i + 1;
+    }
+    {
+      const int f = i + LSTAGES - 1;
+      if (f < nblk) {
+        fk.fetch(kst + fst * 8192, oa, ob, 64 * f < left);
+        fv.fetch(vst + fst * 8192, oa, ob, 64 * f < left);
       }
-#pragma unroll
-      for (int d2 = 0; d2 < 2; ++d2) {
-        const int dp = 2 * grp + d2;   // V columns 16 dp .. 16 dp + 15
-        const int mi = lane >> 3, ri = lane & 7;
-        uint32_t b0, b1, b2, b3;
-        l_ldsm_x4_t(vb + lswz(ks * 16 + (mi & 1) * 8 + ri, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-        l_mma(acc[2 * d2], af, b0, b1);
-        l_mma(acc[2 * d2 + 1], af, b2, b3);
-      }
-      if (grp == 0) l_mma(acc[4], af, ones, ones);
+      asm volatile("cp.async.commit_group;\n" ::);
     }
     st = ring_next(st, LSTAGES);
     fst = ring_next(fst, LSTAGES);
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
-  float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
-  const int q4 = lane & 3;
+  if (tid == 0) {
+    if (!ss.abort && nblk > 0) {   // the last block's MMAs
+      if (lin_wait(&ss.mma_bar, (nblk - 1) & 1))
+        waited = nblk;
+      else
+        ss.abort = 1;
+    }
+    // after an abort, MMAs that went out but were not seen complete land first (bounded again)
+    if (ss.abort && issued > waited) lin_wait(&ss.mma_bar, (issued - 1) & 1);
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (!ss.abort) {
+    // warp w reads the M = 64 accumulator rows 16 (w % 4) .. + 15 from its TMEM lane quarter
+    // (16x256b shape: rows g4 and g4 + 8, columns 2 q4 and 2 q4 + 1 of each 8), columns
+    // 32 (w / 4) .. + 31, and warps 0-3 the z column 64
+    const int quarter = warp & 3, cg = warp >> 2, g4 = lane >> 2, q4 = lane & 3;
+    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+    float r[16];
+    tc::tmem_ld32(trow + 32 * cg, r);
+    float* part = a.part + ((size_t)blockIdx.y * g.H + h) * 64 * 65;
+    const int r0 = 16 * quarter + g4;
 #pragma unroll
-  for (int j = 0; j < 5; ++j) {
-    if (j == 4 && grp != 0) break;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int r = mrow * 16 + g4 + (e >> 1) * 8;
-      const int c = j < 4 ? 32 * grp + 8 * j + 2 * q4 + (e & 1) : 64 + 2 * q4 + (e & 1);
-      if (c <= 64) part[r * 65 + c] = acc[j][e];
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * cg + 8 * j + 2 * q4;
+      part[r0 * 65 + c] = r[4 * j];
+      part[r0 * 65 + c + 1] = r[4 * j + 1];
+      part[(r0 + 8) * 65 + c] = r[4 * j + 2];
+      part[(r0 + 8) * 65 + c + 1] = r[4 * j + 3];
+    }
+    if (cg == 0) {
+      float z[4];
+      tc::tmem_ld8(trow + 64, z);
+      if (q4 == 0) {
+        part[r0 * 65 + 64] = z[0];
+        part[(r0 + 8) * 65 + 64] = z[2];
+      }
     }
   }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(STATE_TMEM_COLS));
 }
 
 // Apply kernel shared memory: the Q ring, one output block, the B operand.
@@ -723,8 +840,9 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   }
   {
     ProfScope prof("linear_state", st);
-    cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(StateSmem));
-    linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, sizeof(StateSmem), st>>>(a);
+    const int smem = (int)sizeof(StateSmem) + 1024;   // + alignment of the base to 1024 bytes
+    cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(a);
   }
   count_launch();
   if (int rc = check_launch("linear_state_q4_kernel")) return rc;
