@@ -24,9 +24,10 @@
 //     forms S' = S A^T, and writes the bf16 B operand [S' | z] of the apply kernel.
 //  3. apply:  per (head, token chunk) CTA: prologue on Q (f(Q) overwrites its
 //     own ring stage; the softmax's division by its sum is left out, since it
-//     cancels in the ratio below), f(Q) [S' | z] on mma.sync, divide by the z
-//     column, add b, stage the bf16 block in the same ring stage and store
-//     whole 128-byte token rows.
+//     cancels in the ratio below), f(Q) [S' | z] on the tcgen05 tensor cores
+//     (M = 64 tokens, N = 72, accumulators in tensor memory), divide by the z
+//     column, add b, stage the bf16 block by stmatrix and store it by one bulk
+//     tensor copy.
 // The fp32 variants run the same three steps with plain fp32 arithmetic.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -511,14 +512,19 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(STATE_TMEM_COLS));
 }
 
-// Apply kernel shared memory: the Q ring, one output block, the B operand.
-// Every piece starts on a 1024-byte boundary, so the swizzled offsets lswz()
-// are the 128-byte swizzle of the tensor-memory-access unit's copies.
+// Apply kernel shared memory: the Q ring, one output block, the B operand, the
+// MMA completion barrier and the tensor-memory base. Every tile starts on a
+// 1024-byte boundary, so the swizzled offsets lswz() are the 128-byte swizzle of
+// the tensor cores' operand reads and of the bulk tensor copies.
 struct ApplySmem {
   unsigned char q[LA_STAGES][64 * 128];
   unsigned char out[64 * 128];
   unsigned char b[NB * 128];
+  uint64_t mma_bar;
+  uint32_t tmem_base;
+  int abort;
 };
+constexpr uint32_t APPLY_TMEM_COLS = 128;   // f(Q) [S' | z]: columns 0-71
 struct ApplyParams {
   CUtensorMap tout;   // out as [N][H][64] bf16, box 64 channels x 1 head x 64 tokens, 128-byte swizzle
   LinearArgs a;
@@ -534,14 +540,31 @@ __device__ __forceinline__ uint32_t l_pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// D = f(Q) [S' | z] of one 64-token block: A = f(Q) (K-major, 64 tokens x 64
+// channels), B = the [72][64] operand (K-major), N = 72, four K = 16 steps 32
+// bytes apart; one elected lane issues and commits to `bar`.
+__device__ __forceinline__ void apply_mma_elect(uint32_t d, uint64_t a, uint64_t b, uint64_t* bar) {
+  constexpr uint32_t ID = tc::idesc(false, NB, false);
+  asm volatile(
+      "{\n .reg .pred e, p0, p1;\n setp.ne.b32 p0, 0, 0;\n setp.eq.b32 p1, 0, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %9, p0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, p1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, p1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%10];\n}\n"
+      ::"r"(d), "l"(a), "l"(b), "l"(a + 2), "l"(b + 2), "l"(a + 4), "l"(b + 4), "l"(a + 6), "l"(b + 6), "r"(ID),
+      "r"(tc::saddr(bar))
+      : "memory");
+}
+
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ ApplyParams prm) {
   // Q ring; f(Q) of a block overwrites its own stage in place (each thread rewrites exactly the
-  // 32 bytes it read), so the MMA reads its A operand from the stage. The bf16 output block
-  // goes to its own buffer, which one thread stores by a bulk tensor copy (rows past the
-  // tensor's last token are not written; chunks start on multiples of 64 tokens, so only the
-  // last chunk has such rows).
+  // 32 bytes it read) and is the A operand of the block's MMAs. The bf16 output block goes to
+  // its own buffer, which one thread stores by a bulk tensor copy (rows past the tensor's last
+  // token are not written; chunks start on multiples of 64 tokens, so only the last chunk has
+  // such rows).
   extern __shared__ unsigned char apply_smem_raw[];
-  ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(apply_smem_raw) + 1023) & ~uintptr_t(1023));
+  ApplySmem& sm = *reinterpret_cast<ApplySmem*>(align1024(apply_smem_raw));
   const LinearArgs& a = prm.a;
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -550,38 +573,59 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const long long n1 = min((long long)g.N, n0 + a.chunk_tokens);
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(a.q) + (long long)h * a.hs;
   const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(a.state_b) + (size_t)h * NB * 64;
-  for (int i = tid; i < NB * 8; i += LQ_THREADS) {
-    const int r = i >> 3, c = i & 7;
-    *reinterpret_cast<uint4*>(sm.b + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
-  }
   const int tok = token_of(tid), half = (tid >> 1) & 1, sub = tid & 1;
-  const int mrow = warp & 3, grp = warp >> 2;   // token rows 16 mrow .., column group
-  const int q4 = lane & 3;
-  float bias[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int c = 32 * grp + 8 * j + 2 * q4;
-    bias[2 * j] = a.b ? a.b[h * 64 + c] : 0.f;
-    bias[2 * j + 1] = a.b ? a.b[h * 64 + c + 1] : 0.f;
-  }
   const int nblk = (int)((n1 - n0 + 63) / 64);
   const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
-  const uint32_t qst = lsmem(sm.q[0]), bst = lsmem(sm.b), ost = lsmem(sm.out);
-  // stmatrix row addresses of the output block: lane 8 k + r gives row r of matrix k, matrices
-  // (rows 0-7, n-block 2x), (rows 8-15, 2x), (rows 0-7, 2x + 1), (rows 8-15, 2x + 1) of store x
-  const uint32_t o_st0 = ost + lswz(mrow * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * grp + (lane >> 4));
-  const uint32_t o_st1 = ost + lswz(mrow * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * grp + 2 + (lane >> 4));
+  const uint32_t qst = lsmem(sm.q[0]), ost = lsmem(sm.out);
   RowFetch fq(Q, n0, a.ts, tok, half, sub);
-  int jb = (int)(n0 % g.L);   // view position of the current block's first token
   for (int i = 0; i < LA_STAGES - 1; ++i) {
     if (i < nblk) fq.fetch(qst + i * 8192, oa, ob, 64 * i < left);
     asm volatile("cp.async.commit_group;\n" ::);
   }
+  for (int i = tid; i < NB * 8; i += LQ_THREADS) {
+    const int r = i >> 3, c = i & 7;
+    *reinterpret_cast<uint4*>(sm.b + lswz(r, c)) = *reinterpret_cast<const uint4*>(sb + r * 64 + c * 8);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // B is read by the tensor cores
+  if (tid == 0) {
+    tc::mbar_init(&sm.mma_bar, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(lsmem(&sm.tmem_base)),
+                 "r"(APPLY_TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint64_t d_q0 = tc::desc_k(qst), d_b = tc::desc_k(lsmem(sm.b));
+  // epilogue: warp w reads accumulator rows 16 (w % 4) .. + 15 (its TMEM lane quarter; 16x256b
+  // shape: rows g4 and g4 + 8, columns 2 q4 and 2 q4 + 1 of each 8), columns 32 (w / 4) .. + 31
+  // and the z column 64
+  const int quarter = warp & 3, cg = warp >> 2, q4 = lane & 3;
+  const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+  float bias[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = 32 * cg + 8 * j + 2 * q4;
+    bias[2 * j] = a.b ? a.b[h * 64 + c] : 0.f;
+    bias[2 * j + 1] = a.b ? a.b[h * 64 + c + 1] : 0.f;
+  }
+  // stmatrix row addresses of the output block: lane 8 k + r gives row r of matrix k, matrices
+  // (rows 0-7, n-block 2x), (rows 8-15, 2x), (rows 0-7, 2x + 1), (rows 8-15, 2x + 1) of store x
+  const uint32_t o_st0 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + (lane >> 4));
+  const uint32_t o_st1 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + 2 + (lane >> 4));
+  int late = -1;   // thread 0: the block whose MMAs were not seen complete (abort)
+  int jb = (int)(n0 % g.L);   // view position of the current block's first token
   int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i + LA_STAGES - 1
   for (int i = 0; i < nblk; ++i) {
     // Block i's copies are the oldest but LA_STAGES - 2 groups in flight. After the barrier every
-    // warp is done with block i - 1, whose stage is refilled only now.
+    // warp is done with block i - 1 (its MMAs completed before its epilogue), whose stage is
+    // refilled only now.
     asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
     __syncthreads();
     {
@@ -599,52 +643,41 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
       features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, 64 * i < left);
     }
     store_q4(sm.q[st], oa, ob, xa, xb);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
     // the previous block's output copy has read the output buffer before anyone rewrites it
     if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     __syncthreads();
-    const uint32_t phi = qst + st * 8192;
-    float acc[5][4];
-#pragma unroll
-    for (int j = 0; j < 5; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {  // 16 channels per k-step
-      uint32_t af[4];
-      {
-        const int mi = lane >> 3, ri = lane & 7;
-        l_ldsm_x4(phi + lswz(mrow * 16 + (mi & 1) * 8 + ri, 2 * ks + (mi >> 1)), af[0], af[1], af[2], af[3]);
-      }
-#pragma unroll
-      for (int n2 = 0; n2 < 2; ++n2) {
-        const int np = 2 * grp + n2;   // state columns 16 np .. 16 np + 15
-        const int mi = lane >> 3, ri = lane & 7;
-        uint32_t b0, b1, b2, b3;
-        l_ldsm_x4(bst + lswz(np * 16 + (mi >> 1) * 8 + ri, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-        l_mma(acc[2 * n2], af, b0, b1);
-        l_mma(acc[2 * n2 + 1], af, b2, b3);
-      }
-      {   // the z column: both column groups compute it, so no exchange is needed
-        const int mi = (lane >> 3) & 1, ri = lane & 7;
-        uint32_t b0, b1;
-        l_ldsm_x2(bst + lswz(64 + ri, 2 * ks + mi), b0, b1);
-        l_mma(acc[4], af, b0, b1);
-      }
+    if (warp == 0) {
+      tc::fence_after();
+      apply_mma_elect(tmem, d_q0 + st * 512, d_b, &sm.mma_bar);
     }
-    // z = column 64 sits in acc[4][0] (row g4) / acc[4][2] (row g4 + 8) of the quad's first lane.
-    {
-      const float il0 = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][0], lane & ~3));
-      const float il1 = __fdividef(1.0f, __shfl_sync(0xffffffffu, acc[4][2], lane & ~3));
+    if (!lin_wait(&sm.mma_bar, i & 1)) {
+      sm.abort = 1;
+      if (tid == 0) late = i;
+    }
+    tc::fence_after();
+    if (!sm.abort) {
+      float r[16], z[4];
+      tc::tmem_ld32(trow + 32 * cg, r);
+      tc::tmem_ld8(trow + 64, z);
+      // z = column 64 sits in z[0] (row g4) / z[2] (row g4 + 8) of the quad's first lane
+      const float il0 = __fdividef(1.0f, __shfl_sync(0xffffffffu, z[0], lane & ~3));
+      const float il1 = __fdividef(1.0f, __shfl_sync(0xffffffffu, z[2], lane & ~3));
       uint32_t w[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        w[j][0] = l_pack_bf16(fmaf(acc[j][0], il0, bias[2 * j]), fmaf(acc[j][1], il0, bias[2 * j + 1]));
-        w[j][1] = l_pack_bf16(fmaf(acc[j][2], il1, bias[2 * j]), fmaf(acc[j][3], il1, bias[2 * j + 1]));
+        w[j][0] = l_pack_bf16(fmaf(r[4 * j], il0, bias[2 * j]), fmaf(r[4 * j + 1], il0, bias[2 * j + 1]));
+        w[j][1] = l_pack_bf16(fmaf(r[4 * j + 2], il1, bias[2 * j]), fmaf(r[4 * j + 3], il1, bias[2 * j + 1]));
       }
       l_stsm_x4(o_st0, w[0][0], w[0][1], w[1][0], w[1][1]);
       l_stsm_x4(o_st1, w[2][0], w[2][1], w[3][0], w[3][1]);
     }
-    // the generic-proxy writes of the block become visible to the bulk copy
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    // the generic-proxy writes of the block become visible to the bulk copy; the TMEM reads
+    // are done before the next block's MMAs
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc::fence_before();
     __syncthreads();
+    if (sm.abort) break;
     if (tid == 0) {
       asm volatile(
           "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n"
@@ -655,7 +688,14 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     fst = ring_next(fst, LA_STAGES);
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
-  if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+  if (tid == 0) {
+    asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+    if (late >= 0) lin_wait(&sm.mma_bar, late & 1);   // after an abort the late MMAs land first (bounded again)
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(APPLY_TMEM_COLS));
 }
 
 // --------------------------------------------------------------------------
