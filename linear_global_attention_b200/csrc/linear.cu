@@ -164,7 +164,7 @@ int read_and_clear_linear_status(int* out) {
 
 // One thread waits for the phase of `parity` of `b`; after g_lin_wait_ns it
 // records ZEBRA_ERR_TIMEOUT and returns false.
-__device__ __noinline__ bool lin_wait(uint64_t* b, uint32_t parity) {
+__device__ __noinline__ bool lin_wait_slow(uint64_t* b, uint32_t parity) {
   const unsigned long long limit = *(volatile unsigned long long*)&g_lin_wait_ns;
   const unsigned long long t0 = tc::gtime();
   while (!tc::mbar_try(b, parity)) {
@@ -174,6 +174,10 @@ __device__ __noinline__ bool lin_wait(uint64_t* b, uint32_t parity) {
     }
   }
   return true;
+}
+// the first test inline (it suspends the thread until the phase completes or the hint runs out)
+__device__ __forceinline__ bool lin_wait(uint64_t* b, uint32_t parity) {
+  return tc::mbar_try(b, parity) || lin_wait_slow(b, parity);
 }
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
