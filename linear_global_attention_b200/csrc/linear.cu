@@ -120,7 +120,7 @@ __device__ __forceinline__ void l_mma(float* c, const uint32_t* a, uint32_t b0, 
 // apply kernel, each refilled once every warp is done with the block it held.
 constexpr int LSTAGES = 3;
 #ifndef ZEBRA_LIN_ASTAGES
-#define ZEBRA_LIN_ASTAGES 4
+#define ZEBRA_LIN_ASTAGES 3
 #endif
 constexpr int LA_STAGES = ZEBRA_LIN_ASTAGES;   // Q ring depth of the apply kernel
 
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
 // the tensor cores' operand reads and of the bulk tensor copies.
 struct ApplySmem {
   unsigned char q[LA_STAGES][64 * 128];
-  unsigned char out[64 * 128];
+  unsigned char out[2][64 * 128];
   unsigned char b[NB * 128];
   uint64_t mma_bar;
   uint32_t tmem_base;
@@ -561,12 +561,30 @@ __device__ __forceinline__ void apply_mma_elect(uint32_t d, uint64_t a, uint64_t
       : "memory");
 }
 
+static_assert(4 * (sizeof(ApplySmem) + 1024 + 1024) <= 228 * 1024, "four CTAs of the apply kernel per SM");
+
+// f(Q) of block i over its own Q rows in ring stage `stage` (each thread reads and rewrites
+// only the 32 bytes it copied), made visible to the tensor cores.
+__device__ __forceinline__ void apply_prologue(const LinearArgs& a, unsigned char* stage, uint32_t oa, uint32_t ob,
+                                               int tok, int half, int sub, int jb, bool valid) {
+  const Geo& g = a.g;
+  float xa[8], xb[8];
+  read_q4(stage, oa, ob, xa, xb);
+  bool sp;
+  int row, col;
+  view_pos(g, mod_L(g, jb + tok), sp, row, col);
+  features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, valid);
+  store_q4(stage, oa, ob, xa, xb);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ ApplyParams prm) {
-  // Q ring; f(Q) of a block overwrites its own stage in place (each thread rewrites exactly the
-  // 32 bytes it read) and is the A operand of the block's MMAs. The bf16 output block goes to
-  // its own buffer, which one thread stores by a bulk tensor copy (rows past the tensor's last
-  // token are not written; chunks start on multiples of 64 tokens, so only the last chunk has
-  // such rows).
+  // Software pipeline over the chunk's 64-token blocks, one barrier per block: while the
+  // tensor cores compute block i's f(Q) [S' | z], the threads run block i + 1's prologue;
+  // then block i's epilogue reads the accumulators, stages the bf16 rows by stmatrix in
+  // output buffer i % 2, and one thread stores them by a bulk tensor copy (rows past the
+  // tensor's last token are not written; chunks start on multiples of 64 tokens, so only
+  // the last chunk has such rows) and issues block i + 1's MMAs.
   extern __shared__ unsigned char apply_smem_raw[];
   ApplySmem& sm = *reinterpret_cast<ApplySmem*>(align1024(apply_smem_raw));
   const LinearArgs& a = prm.a;
@@ -581,7 +599,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const int nblk = (int)((n1 - n0 + 63) / 64);
   const int left = (int)(n1 - n0) - tok;   // block i holds this thread's token iff 64 i < left
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
-  const uint32_t qst = lsmem(sm.q[0]), ost = lsmem(sm.out);
+  const uint32_t qst = lsmem(sm.q[0]), ost = lsmem(sm.out[0]);
   RowFetch fq(Q, n0, a.ts, tok, half, sub);
   for (int i = 0; i < LA_STAGES - 1; ++i) {
     if (i < nblk) fq.fetch(qst + i * 8192, oa, ob, 64 * i < left);
@@ -602,16 +620,10 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
                  "r"(APPLY_TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  const uint64_t d_q0 = tc::desc_k(qst), d_b = tc::desc_k(lsmem(sm.b));
   // epilogue: warp w reads accumulator rows 16 (w % 4) .. + 15 (its TMEM lane quarter; 16x256b
   // shape: rows g4 and g4 + 8, columns 2 q4 and 2 q4 + 1 of each 8), columns 32 (w / 4) .. + 31
   // and the z column 64
   const int quarter = warp & 3, cg = warp >> 2, q4 = lane & 3;
-  const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
   float bias[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -619,41 +631,39 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     bias[2 * j] = a.b ? a.b[h * 64 + c] : 0.f;
     bias[2 * j + 1] = a.b ? a.b[h * 64 + c + 1] : 0.f;
   }
-  // stmatrix row addresses of the output block: lane 8 k + r gives row r of matrix k, matrices
+  // stmatrix row addresses in output buffer 0: lane 8 k + r gives row r of matrix k, matrices
   // (rows 0-7, n-block 2x), (rows 8-15, 2x), (rows 0-7, 2x + 1), (rows 8-15, 2x + 1) of store x
   const uint32_t o_st0 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + (lane >> 4));
   const uint32_t o_st1 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + 2 + (lane >> 4));
-  int late = -1;   // thread 0: the block whose MMAs were not seen complete (abort)
-  int jb = (int)(n0 % g.L);   // view position of the current block's first token
-  int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i + LA_STAGES - 1
-  for (int i = 0; i < nblk; ++i) {
-    // Block i's copies are the oldest but LA_STAGES - 2 groups in flight. After the barrier every
-    // warp is done with block i - 1 (its MMAs completed before its epilogue), whose stage is
-    // refilled only now.
+  int jb = (int)(n0 % g.L);   // view position of the first token of the next block to prepare
+  if (nblk > 0) {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
-    __syncthreads();
-    {
+    apply_prologue(a, sm.q[0], oa, ob, tok, half, sub, jb, 0 < left);
+    jb = mod_L(g, jb + 64);
+  }
+  tc::fence_before();
+  __syncthreads();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+  const uint64_t d_q0 = tc::desc_k(qst), d_b = tc::desc_k(lsmem(sm.b));
+  if (warp == 0 && nblk > 0) {
+    tc::fence_after();
+    apply_mma_elect(tmem, d_q0, d_b, &sm.mma_bar);
+  }
+  int late = -1;   // thread 0: the block whose MMAs were not seen complete (abort)
+  int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i - 1 (refilled now)
+  for (int i = 0; i < nblk; ++i) {
+    const int nst = ring_next(st, LA_STAGES);
+    {   // block i + LA_STAGES - 1 into the stage of block i - 1 (its MMAs were seen complete
+        // before the last barrier)
       const int f = i + LA_STAGES - 1;
       if (f < nblk) fq.fetch(qst + fst * 8192, oa, ob, 64 * f < left);
       asm volatile("cp.async.commit_group;\n" ::);
     }
-    float xa[8], xb[8];
-    read_q4(sm.q[st], oa, ob, xa, xb);
-    {
-      bool sp;
-      int row, col;
-      view_pos(g, mod_L(g, jb + tok), sp, row, col);
+    if (i + 1 < nblk) {   // block i + 1's copies are the oldest but LA_STAGES - 2 groups in flight
+      asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
+      apply_prologue(a, sm.q[nst], oa, ob, tok, half, sub, jb, 64 * (i + 1) < left);
       jb = mod_L(g, jb + 64);
-      features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, 64 * i < left);
-    }
-    store_q4(sm.q[st], oa, ob, xa, xb);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
-    // the previous block's output copy has read the output buffer before anyone rewrites it
-    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-    __syncthreads();
-    if (warp == 0) {
-      tc::fence_after();
-      apply_mma_elect(tmem, d_q0 + st * 512, d_b, &sm.mma_bar);
     }
     if (!lin_wait(&sm.mma_bar, i & 1)) {
       sm.abort = 1;
@@ -673,22 +683,30 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
         w[j][0] = l_pack_bf16(fmaf(r[4 * j], il0, bias[2 * j]), fmaf(r[4 * j + 1], il0, bias[2 * j + 1]));
         w[j][1] = l_pack_bf16(fmaf(r[4 * j + 2], il1, bias[2 * j]), fmaf(r[4 * j + 3], il1, bias[2 * j + 1]));
       }
-      l_stsm_x4(o_st0, w[0][0], w[0][1], w[1][0], w[1][1]);
-      l_stsm_x4(o_st1, w[2][0], w[2][1], w[3][0], w[3][1]);
+      const uint32_t ob_off = (i & 1) * 8192;
+      l_stsm_x4(o_st0 + ob_off, w[0][0], w[0][1], w[1][0], w[1][1]);
+      l_stsm_x4(o_st1 + ob_off, w[2][0], w[2][1], w[3][0], w[3][1]);
     }
-    // the generic-proxy writes of the block become visible to the bulk copy; the TMEM reads
-    // are done before the next block's MMAs
+    // the generic-proxy writes (output rows, block i + 1's f(Q)) become visible to the bulk
+    // copy and the tensor cores; the TMEM reads are done before block i + 1's MMAs; block
+    // i - 1's output copy has read its buffer before block i + 1's epilogue rewrites it
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc::fence_before();
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
     __syncthreads();
     if (sm.abort) break;
     if (tid == 0) {
       asm volatile(
           "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n"
-          "cp.async.bulk.commit_group;\n" ::"l"(&prm.tout), "r"(0), "r"(h), "r"((int)(n0 + 64LL * i)), "r"(ost)
+          "cp.async.bulk.commit_group;\n" ::"l"(&prm.tout), "r"(0), "r"(h), "r"((int)(n0 + 64LL * i)),
+          "r"(ost + (i & 1) * 8192)
           : "memory");
     }
-    st = ring_next(st, LA_STAGES);
+    if (warp == 0 && i + 1 < nblk) {
+      tc::fence_after();
+      apply_mma_elect(tmem, d_q0 + nst * 512, d_b, &sm.mma_bar);
+    }
+    st = nst;
     fst = ring_next(fst, LA_STAGES);
   }
   asm volatile("cp.async.wait_group 0;\n" ::);
