@@ -89,28 +89,11 @@ __device__ __forceinline__ void features_full(float* x, bool special, int row, i
 }
 
 // --------------------------------------------------------------------------
-// mma helpers (same conventions as the attention kernels)
+// shared-memory addressing: 64 x 128-byte tiles with the 128-byte swizzle
+// (16-byte chunk c of row r at chunk c ^ (r % 8))
 // --------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t lsmem(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 __device__ __forceinline__ uint32_t lswz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
-__device__ __forceinline__ void l_ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void l_ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void l_ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-__device__ __forceinline__ void l_mma(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 // --------------------------------------------------------------------------
 // 1/3. state and apply (bf16), four threads per token
 // --------------------------------------------------------------------------
@@ -189,9 +172,9 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
 // (channels 0-31 turn by patch row, 32-63 by column), sub = part % 2 (pairs
 // j = 8 sub .. 8 sub + 7 of the half): the "a" channels 32 half + 8 sub .. + 7
 // and their partners 16 further. The four threads of a token combine the RMS
-// norm and the sum with two shuffles each. 8 warps split the
-// 64 x 72 contraction: rows 16 (warp % 4) .. + 15, columns 0-31 plus the
-// z column (warp / 4 = 0) or columns 32-63 (warp / 4 = 1).
+// norm and the sum with two shuffles each. The contractions run on the tensor
+// cores; to read an accumulator back, warp w takes rows 16 (w % 4) .. + 15 (its
+// tensor-memory lane quarter) and columns 32 (w / 4) .. + 31.
 constexpr int LQ_THREADS = 256;
 // Token of thread tid: the quads of a warp take its 8 tokens in the order 0 2 1 3 4 6 5 7,
 // so the two tokens of each 8-lane phase of a 16-byte shared access are rows r and r + 2.
