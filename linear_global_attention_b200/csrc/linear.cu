@@ -100,7 +100,8 @@ __device__ __forceinline__ uint32_t lswz(int row, int chunk) { return (uint32_t)
 // Raw bf16 rows of a 64-token block, one 128-byte head slice per token, land in
 // a ring of swizzled shared tiles through cp.async (padding tokens are
 // zero-filled): 3 stages of K and V in the state kernel, LA_STAGES of Q in the
-// apply kernel, each refilled once every warp is done with the block it held.
+// apply kernel, each refilled once the MMAs that read the block it held have
+// completed and every warp has passed a barrier after its own use of it.
 constexpr int LSTAGES = 3;
 #ifndef ZEBRA_LIN_ASTAGES
 #define ZEBRA_LIN_ASTAGES 3
@@ -145,8 +146,8 @@ int read_and_clear_linear_status(int* out) {
   return ZEBRA_OK;
 }
 
-// One thread waits for the phase of `parity` of `b`; after g_lin_wait_ns it
-// records ZEBRA_ERR_TIMEOUT and returns false.
+// The calling thread waits for the phase of `parity` of `b`; after
+// g_lin_wait_ns it records ZEBRA_ERR_TIMEOUT and returns false.
 __device__ __noinline__ bool lin_wait_slow(uint64_t* b, uint32_t parity) {
   const unsigned long long limit = *(volatile unsigned long long*)&g_lin_wait_ns;
   const unsigned long long t0 = tc::gtime();
