@@ -120,6 +120,9 @@ struct StateSmem {
   int abort;
 };
 constexpr uint32_t STATE_TMEM_COLS = 128;   // [S | z]: columns 0-63 and 64-79
+// 4 CTAs per SM: shared memory (+ 1 KB base alignment, + 1 KB the system keeps per CTA) and TMEM
+static_assert(4 * (sizeof(StateSmem) + 1024 + 1024) <= 228 * 1024, "four CTAs of the state kernel per SM");
+static_assert(4 * STATE_TMEM_COLS <= 512, "four CTAs' tensor memory per SM");
 
 // Bounded waits of the linear stage's tcgen05 kernels: the sticky status word,
 // the wait limit, and the error-path test hook (the token block of each chunk
@@ -513,6 +516,7 @@ struct ApplySmem {
   int abort;
 };
 constexpr uint32_t APPLY_TMEM_COLS = 128;   // f(Q) [S' | z]: columns 0-71
+static_assert(4 * APPLY_TMEM_COLS <= 512, "four CTAs' tensor memory per SM");
 struct ApplyParams {
   CUtensorMap tout;   // out as [N][H][64] bf16, box 64 channels x 1 head x 64 tokens, 128-byte swizzle
   LinearArgs a;
