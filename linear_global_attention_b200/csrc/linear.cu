@@ -115,6 +115,7 @@ struct StateSmem {
   unsigned char k[LSTAGES][64 * 128];
   unsigned char v[LSTAGES][64 * 128];
   unsigned char ones[16 * 128];
+  uint64_t full[LSTAGES];   // K and V of a stage landed (bulk tensor copies)
   uint64_t mma_bar;
   uint32_t tmem_base;
   int abort;
@@ -370,9 +371,29 @@ __device__ __forceinline__ void state_mma_elect(uint32_t tmem, uint64_t fk, uint
       : "memory");
 }
 
-__global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __grid_constant__ LinearArgs a) {
+// Tensor maps of the state kernel's K and V inputs ([N, H, 64] strided by (ts, hs)): 3D maps with
+// the channels innermost, the outer two dimensions in the order of their strides (head_outer = 0:
+// {64, H, N}, coordinates (0, h, n); 1: {64, N, H}, coordinates (0, n, h)), a box of 64 channels x
+// one head x 64 tokens and the 128-byte swizzle. Layouts a map cannot describe take the 16-byte
+// asynchronous copies instead.
+struct StateParams {
+  CUtensorMap tk, tv;
+  LinearArgs a;
+  int head_outer;
+};
+
+__device__ __forceinline__ void l_tma_3d(uint32_t dst, const CUtensorMap* map, int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(map), "r"(0), "r"(c1), "r"(c2), "r"(lsmem(bar))
+      : "memory");
+}
+
+template <bool TMA_IN>
+__global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __grid_constant__ StateParams prm) {
   extern __shared__ unsigned char state_smem_raw[];
   StateSmem& ss = *reinterpret_cast<StateSmem*>(align1024(state_smem_raw));
+  const LinearArgs& a = prm.a;
   const Geo& g = a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;   // grid (head, chunk): the heads of the same tokens run together
@@ -387,15 +408,25 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
   const uint32_t kst = lsmem(ss.k[0]), vst = lsmem(ss.v[0]);
   RowFetch fk(K, n0, a.ts, tok, half, sub), fv(Vt, n0, a.ts, tok, half, sub);
-  for (int i = 0; i < LSTAGES - 1; ++i) {
-    if (i < nblk) {
-      fk.fetch(kst + i * 8192, oa, ob, 64 * i < left);
-      fv.fetch(vst + i * 8192, oa, ob, 64 * i < left);
+  // block f into ring stage `stage`: one thread arms the stage's barrier and issues two bulk tensor
+  // copies (rows past the tensor's end are zero-filled), or every thread copies its 16-byte pieces
+  auto load = [&](int f, int stage) {
+    if constexpr (TMA_IN) {
+      if (tid == 0) {
+        const int n = (int)(n0 + 64LL * f);
+        const int c1 = prm.head_outer ? n : h, c2 = prm.head_outer ? h : n;
+        tc::mbar_expect_tx(&ss.full[stage], 2 * 64 * 128);
+        l_tma_3d(kst + stage * 8192, &prm.tk, c1, c2, &ss.full[stage]);
+        l_tma_3d(vst + stage * 8192, &prm.tv, c1, c2, &ss.full[stage]);
+      }
+    } else {
+      fk.fetch(kst + stage * 8192, oa, ob, 64 * f < left);
+      fv.fetch(vst + stage * 8192, oa, ob, 64 * f < left);
     }
-    asm volatile("cp.async.commit_group;\n" ::);
-  }
+  };
   if (tid == 0) {
     tc::mbar_init(&ss.mma_bar, 1);
+    for (int i = 0; i < LSTAGES; ++i) tc::mbar_init(&ss.full[i], 1);
     ss.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -409,15 +440,24 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
+  for (int i = 0; i < LSTAGES - 1; ++i) {   // the barriers are initialised: the first blocks go out
+    if (i < nblk) load(i, i);
+    if constexpr (!TMA_IN) asm volatile("cp.async.commit_group;\n" ::);
+  }
   const uint32_t tmem = ss.tmem_base;
   const uint64_t d_k0 = tc::desc_mn(kst), d_v0 = tc::desc_mn(vst), d_ones = tc::desc_k(lsmem(ss.ones));
   const int inject = *(volatile int*)&g_lin_inject_block;
   int issued = 0, waited = 0;   // thread 0: blocks whose MMAs went out / were seen complete
+  int consumed = 0;             // blocks whose loop iteration ran to its end
   int jb = (int)(n0 % g.L);   // view position of the current block's first token
   int st = 0, fst = LSTAGES - 1;   // ring stages of block i and of block i + LSTAGES - 1
   for (int i = 0; i < nblk; ++i) {
-    // Block i's copies are the oldest but LSTAGES - 2 groups in flight.
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 2));
+    if constexpr (TMA_IN) {
+      if (!lin_wait(&ss.full[st], (i / LSTAGES) & 1)) ss.abort = 1;
+    } else {
+      // Block i's copies are the oldest but LSTAGES - 2 groups in flight.
+      asm volatile("cp.async.wait_group %0;\n" ::"n"(LSTAGES - 2));
+    }
     __syncthreads();
     const bool valid = 64 * i < left;
     float xa[8], xb[8];
@@ -447,16 +487,21 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
     }
     {
       const int f = i + LSTAGES - 1;
-      if (f < nblk) {
-        fk.fetch(kst + fst * 8192, oa, ob, 64 * f < left);
-        fv.fetch(vst + fst * 8192, oa, ob, 64 * f < left);
-      }
-      asm volatile("cp.async.commit_group;\n" ::);
+      if (f < nblk) load(f, fst);
+      if constexpr (!TMA_IN) asm volatile("cp.async.commit_group;\n" ::);
     }
     st = ring_next(st, LSTAGES);
     fst = ring_next(fst, LSTAGES);
+    consumed = i + 1;
   }
-  asm volatile("cp.async.wait_group 0;\n" ::);
+  if constexpr (TMA_IN) {
+    // after an abort, bulk copies that went out but were not waited for land first (bounded again)
+    if (tid == 0 && ss.abort)
+      for (int f = consumed; f < min(nblk, consumed + LSTAGES - 1); ++f)
+        lin_wait(&ss.full[f % LSTAGES], (f / LSTAGES) & 1);
+  } else {
+    asm volatile("cp.async.wait_group 0;\n" ::);
+  }
   if (tid == 0) {
     if (!ss.abort && nblk > 0) {   // the last block's MMAs
       if (lin_wait(&ss.mma_bar, (nblk - 1) & 1))
@@ -873,6 +918,29 @@ static bool make_out_map(CUtensorMap* m, void* out, const Geo& g) {
          CUDA_SUCCESS;
 }
 
+// K or V ([N, H, 64] bf16 strided by ts, hs elements) as the state kernel's 3D map (see StateParams)
+static bool make_in_map(CUtensorMap* m, const void* base, const Geo& g, long long ts, long long hs, int* head_outer) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  const cuuint64_t tsb = (cuuint64_t)ts * 2, hsb = g.H > 1 ? (cuuint64_t)hs * 2 : 128;
+  if (tsb == 0 || hsb == 0 || tsb >= (1ull << 40) || hsb >= (1ull << 40)) return false;
+  *head_outer = hsb > tsb ? 1 : 0;
+  cuuint64_t dims[3] = {64, (cuuint64_t)(*head_outer ? g.N : g.H), (cuuint64_t)(*head_outer ? g.H : g.N)};
+  cuuint64_t strides[2] = {*head_outer ? tsb : hsb, *head_outer ? hsb : tsb};
+  cuuint32_t box[3] = {64, (cuuint32_t)(*head_outer ? 64 : 1), (cuuint32_t)(*head_outer ? 1 : 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <>
 int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   if (a.g.N == 0) return ZEBRA_OK;
@@ -889,10 +957,17 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
     return ZEBRA_ERR_CUDA;
   }
   {
+    StateParams sp;
+    sp.a = a;
+    int ho_k = 0, ho_v = 0;
+    const bool tma_in = make_in_map(&sp.tk, a.k, a.g, a.ts, a.hs, &ho_k) &&
+                        make_in_map(&sp.tv, a.v, a.g, a.ts, a.hs, &ho_v) && ho_k == ho_v;
+    sp.head_outer = ho_k;
     ProfScope prof("linear_state", st);
     const int smem = (int)sizeof(StateSmem) + 1024;   // + alignment of the base to 1024 bytes
-    cudaFuncSetAttribute(linear_state_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    linear_state_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(a);
+    auto kern = tma_in ? linear_state_q4_kernel<true> : linear_state_q4_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    kern<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(sp);
   }
   count_launch();
   if (int rc = check_launch("linear_state_q4_kernel")) return rc;

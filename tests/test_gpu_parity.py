@@ -376,6 +376,25 @@ def test_linear_v128_full_size_sampled():
         ph.assert_close(out[rows, h], want[:, h], "bf16", f"linear v128 head {h}")
 
 
+def test_linear_head_stride_zero_copy_path():
+    """Heads aliased by a head stride of 0: no tensor map describes that layout, so the state kernel
+    loads K and V by its 16-byte asynchronous copies instead of bulk tensor copies."""
+    g = Geom(4, 21, 19, 3)
+    rng = np.random.default_rng(17)
+    one = [synth.round_to_bf16(rng.standard_normal((g.n_tokens, 1, 64)).astype(np.float32)) for _ in range(3)]
+    q, k, v = (np.ascontiguousarray(np.broadcast_to(x, (g.n_tokens, g.heads, 64))) for x in one)
+    A, b = synth.affine(g.heads, 17)
+    zg = ph.zgeom(g)
+    qd, kd, vd = (torch.from_numpy(x).to(torch.bfloat16).cuda().expand(g.n_tokens, g.heads, 64) for x in one)
+    assert qd.stride(1) == 0
+    out = torch.empty((g.n_tokens, g.heads, 64), dtype=torch.bfloat16, device="cuda")
+    ws = zb.workspace(zg, zb.ZEBRA_OP_LINEAR, zb.ZEBRA_BF16)
+    zb.zebra_linear_attn(zg, qd, kd, vd, torch.from_numpy(A).cuda(), torch.from_numpy(b).cuda(), out, ws)
+    torch.cuda.synchronize()
+    assert zb.zebra_sync_status() == zb.ZEBRA_OK
+    ph.assert_close(ph.host(out), oracle.linear_stage(q, k, v, g, A, b), "bf16", "linear, head stride 0")
+
+
 @pytest.mark.parametrize("geom", [Geom(3, 1, 1, 2), Geom(2, 3, 5, 1, n_special=0), Geom(1, 40, 33, 2)],
                          ids=["1x1", "nospecial", "wide"])
 def test_linear_degenerate(geom):
