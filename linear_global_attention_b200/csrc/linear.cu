@@ -556,6 +556,7 @@ struct ApplySmem {
   unsigned char q[LA_STAGES][64 * 128];
   unsigned char out[2][64 * 128];
   unsigned char b[NB * 128];
+  uint64_t full[LA_STAGES];   // Q of a stage landed (bulk tensor copies)
   uint64_t mma_bar;
   uint32_t tmem_base;
   int abort;
@@ -564,7 +565,9 @@ constexpr uint32_t APPLY_TMEM_COLS = 128;   // f(Q) [S' | z]: columns 0-71
 static_assert(4 * APPLY_TMEM_COLS <= 512, "four CTAs' tensor memory per SM");
 struct ApplyParams {
   CUtensorMap tout;   // out as [N][H][64] bf16, box 64 channels x 1 head x 64 tokens, 128-byte swizzle
+  CUtensorMap tq;     // Q as the state kernel's K and V (StateParams), when a map describes it
   LinearArgs a;
+  int head_outer;
 };
 
 __device__ __forceinline__ void l_stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
@@ -611,6 +614,7 @@ __device__ __forceinline__ void apply_prologue(const LinearArgs& a, unsigned cha
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+template <bool TMA_IN>
 __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __grid_constant__ ApplyParams prm) {
   // Software pipeline over the chunk's 64-token blocks, one barrier per block: while the
   // tensor cores compute block i's f(Q) [S' | z], the threads run block i + 1's prologue;
@@ -634,9 +638,35 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const uint32_t oa = lswz(tok, 4 * half + sub), ob = lswz(tok, 4 * half + sub + 2);
   const uint32_t qst = lsmem(sm.q[0]), ost = lsmem(sm.out[0]);
   RowFetch fq(Q, n0, a.ts, tok, half, sub);
-  for (int i = 0; i < LA_STAGES - 1; ++i) {
-    if (i < nblk) fq.fetch(qst + i * 8192, oa, ob, 64 * i < left);
-    asm volatile("cp.async.commit_group;\n" ::);
+  int loaded = 0, seen = 0;   // blocks whose copies went out / whose landing this thread saw
+  // block f (= loaded) into ring stage `stage` (bulk tensor copy armed by one thread, or 16-byte copies)
+  auto load = [&](int f, int stage) {
+    if constexpr (TMA_IN) {
+      if (tid == 0) {
+        const int n = (int)(n0 + 64LL * f);
+        tc::mbar_expect_tx(&sm.full[stage], 64 * 128);
+        l_tma_3d(qst + stage * 8192, &prm.tq, prm.head_outer ? n : h, prm.head_outer ? h : n, &sm.full[stage]);
+      }
+    } else {
+      fq.fetch(qst + stage * 8192, oa, ob, 64 * f < left);
+    }
+    loaded = f + 1;
+  };
+  // block f's copies are complete for this thread (false: the wait ran out)
+  auto landed = [&](int f) -> bool {
+    if constexpr (TMA_IN) {
+      if (!lin_wait(&sm.full[f % LA_STAGES], (f / LA_STAGES) & 1)) return false;
+    } else {
+      asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
+    }
+    seen = f + 1;
+    return true;
+  };
+  if constexpr (!TMA_IN) {
+    for (int i = 0; i < LA_STAGES - 1; ++i) {
+      if (i < nblk) load(i, i);
+      asm volatile("cp.async.commit_group;\n" ::);
+    }
   }
   for (int i = tid; i < NB * 8; i += LQ_THREADS) {
     const int r = i >> 3, c = i & 7;
@@ -645,6 +675,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // B is read by the tensor cores
   if (tid == 0) {
     tc::mbar_init(&sm.mma_bar, 1);
+    for (int i = 0; i < LA_STAGES; ++i) tc::mbar_init(&sm.full[i], 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -669,8 +700,13 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const uint32_t o_st0 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + (lane >> 4));
   const uint32_t o_st1 = ost + lswz(quarter * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), 4 * cg + 2 + (lane >> 4));
   int jb = (int)(n0 % g.L);   // view position of the first token of the next block to prepare
+  if constexpr (TMA_IN) {
+    __syncthreads();   // the barriers are initialised: the first blocks go out
+    for (int i = 0; i < LA_STAGES - 1; ++i)
+      if (i < nblk) load(i, i);
+  }
   if (nblk > 0) {
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
+    if (!landed(0)) sm.abort = 1;
     apply_prologue(a, sm.q[0], oa, ob, tok, half, sub, jb, 0 < left);
     jb = mod_L(g, jb + 64);
   }
@@ -679,7 +715,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   const uint32_t tmem = sm.tmem_base;
   const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
   const uint64_t d_q0 = tc::desc_k(qst), d_b = tc::desc_k(lsmem(sm.b));
-  if (warp == 0 && nblk > 0) {
+  if (warp == 0 && nblk > 0 && !sm.abort) {
     tc::fence_after();
     apply_mma_elect(tmem, d_q0, d_b, &sm.mma_bar);
   }
@@ -687,14 +723,15 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   int st = 0, fst = LA_STAGES - 1;   // ring stages of block i and of block i - 1 (refilled now)
   for (int i = 0; i < nblk; ++i) {
     const int nst = ring_next(st, LA_STAGES);
+    if (sm.abort) break;   // (read after the last barrier: the same in every thread)
     {   // block i + LA_STAGES - 1 into the stage of block i - 1 (its MMAs were seen complete
         // before the last barrier)
       const int f = i + LA_STAGES - 1;
-      if (f < nblk) fq.fetch(qst + fst * 8192, oa, ob, 64 * f < left);
-      asm volatile("cp.async.commit_group;\n" ::);
+      if (f < nblk) load(f, fst);
+      if constexpr (!TMA_IN) asm volatile("cp.async.commit_group;\n" ::);
     }
-    if (i + 1 < nblk) {   // block i + 1's copies are the oldest but LA_STAGES - 2 groups in flight
-      asm volatile("cp.async.wait_group %0;\n" ::"n"(LA_STAGES - 2));
+    if (i + 1 < nblk) {   // block i + 1's copies (16-byte copies: the oldest but LA_STAGES - 2 groups)
+      if (!landed(i + 1)) sm.abort = 1;
       apply_prologue(a, sm.q[nst], oa, ob, tok, half, sub, jb, 64 * (i + 1) < left);
       jb = mod_L(g, jb + 64);
     }
@@ -742,7 +779,13 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     st = nst;
     fst = ring_next(fst, LA_STAGES);
   }
-  asm volatile("cp.async.wait_group 0;\n" ::);
+  if constexpr (TMA_IN) {
+    // after an abort, bulk copies that went out but were not waited for land first (bounded again)
+    if (tid == 0 && sm.abort)
+      for (int f = seen; f < loaded; ++f) lin_wait(&sm.full[f % LA_STAGES], (f / LA_STAGES) & 1);
+  } else {
+    asm volatile("cp.async.wait_group 0;\n" ::);
+  }
   if (tid == 0) {
     asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
     if (late >= 0) lin_wait(&sm.mma_bar, late & 1);   // after an abort the late MMAs land first (bounded again)
@@ -952,6 +995,7 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   }
   ApplyParams prm;
   prm.a = a;
+  const bool tma_q = make_in_map(&prm.tq, a.q, a.g, a.ts, a.hs, &prm.head_outer);
   if (!make_out_map(&prm.tout, a.out, a.g)) {
     set_error("cuTensorMapEncodeTiled failed (linear output)");
     return ZEBRA_ERR_CUDA;
@@ -980,8 +1024,9 @@ int launch_linear<__nv_bfloat16>(const LinearArgs& a, cudaStream_t st) {
   {
     ProfScope prof("linear_apply", st);
     const int smem = (int)sizeof(ApplySmem) + 1024;   // + alignment of the base to 1024 bytes
-    cudaFuncSetAttribute(linear_apply_q4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    linear_apply_q4_kernel<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(prm);
+    auto kern = tma_q ? linear_apply_q4_kernel<true> : linear_apply_q4_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    kern<<<dim3(a.g.H, a.chunks), LQ_THREADS, smem, st>>>(prm);
   }
   count_launch();
   return check_launch("linear_apply_q4_kernel");
