@@ -14,8 +14,9 @@
 // (S' = S A^T) makes the epilogue one 64x65 contraction per token.
 //
 // Three kernels:
-//  1. state:  per (head, token chunk) CTA: prologue on K in registers (4 threads
-//     per token, 16 channels each), f(K) -> its own K ring stage as bf16, then
+//  1. state:  per (head, token chunk) CTA: K and V blocks by bulk tensor copies,
+//     prologue on K in registers (4 threads per token, 16 channels each),
+//     f(K) -> its own K ring stage as bf16, then
 //     [S | z] += f(K)^T [V | ones] on the tcgen05 tensor cores (M = 64 channels,
 //     N = 64 for S and 16 for z, K = 64 tokens per block, fp32 accumulators in
 //     tensor memory; one thread issues, the next block's prologue overlaps),
@@ -98,10 +99,12 @@ __device__ __forceinline__ uint32_t lswz(int row, int chunk) { return (uint32_t)
 // 1/3. state and apply (bf16), four threads per token
 // --------------------------------------------------------------------------
 // Raw bf16 rows of a 64-token block, one 128-byte head slice per token, land in
-// a ring of swizzled shared tiles through cp.async (padding tokens are
-// zero-filled): 3 stages of K and V in the state kernel, LA_STAGES of Q in the
-// apply kernel, each refilled once the MMAs that read the block it held have
-// completed and every warp has passed a barrier after its own use of it.
+// a ring of 128-byte-swizzled shared tiles, by bulk tensor copies where a tensor
+// map describes the input layout, else by 16-byte asynchronous copies (rows past
+// the tensor's end zero-filled either way): 3 stages of K and V in the state
+// kernel, LA_STAGES of Q in the apply kernel, each refilled once the MMAs that
+// read the block it held have completed and every warp has passed a barrier
+// after its own use of it.
 constexpr int LSTAGES = 3;
 #ifndef ZEBRA_LIN_ASTAGES
 #define ZEBRA_LIN_ASTAGES 3
