@@ -60,6 +60,11 @@ __device__ __forceinline__ void view_pos(const Geo& g, int j, bool& special, int
 }
 // j mod L for 0 <= j < 2^31
 __device__ __forceinline__ int mod_L(const Geo& g, int j) { return j - fdiv(j, g.fL) * g.L; }
+// j mod L for 0 <= j < L + 64: one compare and subtract when a view has at least 64 tokens
+__device__ __forceinline__ int wrap_L(const Geo& g, int j) {
+  if (g.L >= 64) return j >= g.L ? j - g.L : j;
+  return mod_L(g, j);
+}
 
 // full 64-channel prologue in one thread (fp32 path)
 __device__ __forceinline__ void features_full(float* x, bool special, int row, int col,
@@ -468,8 +473,8 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_state_q4_kernel(const __
     {
       bool sp;
       int row, col;
-      view_pos(g, mod_L(g, jb + tok), sp, row, col);
-      jb = mod_L(g, jb + 64);
+      view_pos(g, wrap_L(g, jb + tok), sp, row, col);
+      jb = wrap_L(g, jb + 64);
       features_lin<true>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, valid);
     }
     store_q4(ss.k[st], oa, ob, xa, xb);   // f(K) over its own K rows
@@ -611,7 +616,7 @@ __device__ __forceinline__ void apply_prologue(const LinearArgs& a, unsigned cha
   read_q4(stage, oa, ob, xa, xb);
   bool sp;
   int row, col;
-  view_pos(g, mod_L(g, jb + tok), sp, row, col);
+  view_pos(g, wrap_L(g, jb + tok), sp, row, col);
   features_lin<false>(xa, xb, half, sub, sp, row, col, a.rope_g, a.maxpos, a.eps, valid);
   store_q4(stage, oa, ob, xa, xb);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -711,7 +716,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
   if (nblk > 0) {
     if (!landed(0)) sm.abort = 1;
     apply_prologue(a, sm.q[0], oa, ob, tok, half, sub, jb, 0 < left);
-    jb = mod_L(g, jb + 64);
+    jb = wrap_L(g, jb + 64);
   }
   tc::fence_before();
   __syncthreads();
@@ -736,7 +741,7 @@ __global__ void __launch_bounds__(LQ_THREADS, 4) linear_apply_q4_kernel(const __
     if (i + 1 < nblk) {   // block i + 1's copies (16-byte copies: the oldest but LA_STAGES - 2 groups)
       if (!landed(i + 1)) sm.abort = 1;
       apply_prologue(a, sm.q[nst], oa, ob, tok, half, sub, jb, 64 * (i + 1) < left);
-      jb = mod_L(g, jb + 64);
+      jb = wrap_L(g, jb + 64);
     }
     if (!lin_wait(&sm.mma_bar, i & 1)) {
       sm.abort = 1;
